@@ -1,0 +1,245 @@
+/*
+ * lsa.h -- C ABI of the Lookahead Sparse Attention (LSA) decode step on B200 (sm_100a).
+ *
+ * The method (arXiv 2606.09079, "FlashMemory-DeepSeek-V4: Lightning Index
+ * Ultra-Long Context via Lookahead Sparse Attention"):
+ *   every 64 decode steps a Neural Memory Indexer scores one compressed key
+ *   per 64-token KV chunk and keeps every chunk whose sigmoid score is at
+ *   least 0.5; inside the kept chunks the Lightning Indexer picks a finer
+ *   top-k of tokens at every step; core attention runs over those tokens plus
+ *   the always-resident most recent 8000 tokens.  Chunks outside the window
+ *   may live in pinned host memory and are copied in when kept.
+ *   (gist.science explainer, "Technisches Resuemee" section 2.1;
+ *    cjcn.com.cn article, section 2.)
+ *
+ * Conventions shared by every entry point
+ *   - bf16 data is passed as its 16-bit pattern (lsa_bf16).
+ *   - Every pointer named *_dev or taking device data is a CUDA device
+ *     pointer; *_host pointers are host memory.  The caller owns all memory:
+ *     the library never allocates, frees or retains a pointer after return.
+ *   - Work is enqueued asynchronously on the given stream.  Argument errors are
+ *     detected on the host and returned before anything is launched; the
+ *     message is available from lsa_last_error() (thread-local).
+ *   - Conditions that only the device can see (a kept list longer than its
+ *     capacity, a chunk-table entry that is -1 or out of range, a bounded wait
+ *     that ran out) are OR-ed into *dev_status as LSA_DEV_* bits when
+ *     dev_status is not NULL; the affected output is truncated or the bad row
+ *     is skipped.  No call traps or aborts.
+ *   - Scratch memory is passed in as (ws, ws_bytes); lsa_*_workspace_size()
+ *     report the size.  Workspace contents need no initialisation.
+ *   - Chunk pools: token position p of sequence b lives in row p % 64 of pool
+ *     slot chunk_table[b * table_stride + p / 64]; -1 marks a chunk that is not
+ *     on the device.  Pools are [n_slots, 64, row_width] row-major.
+ */
+#ifndef LSA_H
+#define LSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t lsa_bf16;
+typedef struct CUstream_st *lsa_stream_t;   /* same type as cudaStream_t */
+typedef struct CUevent_st *lsa_event_t;     /* same type as cudaEvent_t */
+
+#define LSA_CHUNK 64            /* tokens per KV chunk */
+
+enum {
+    LSA_OK = 0,
+    LSA_ERR_INVALID_ARG = 1,    /* null pointer, negative size, unsupported value */
+    LSA_ERR_SHAPE = 2,          /* head count / width combination not supported */
+    LSA_ERR_CUDA = 3,           /* a CUDA runtime call failed (message has the name) */
+    LSA_ERR_CAPACITY = 4,       /* an output array is too small for the request */
+    LSA_ERR_TIMEOUT = 5,
+    LSA_ERR_TABLE = 6,          /* a host-side chunk table entry is invalid */
+    LSA_ERR_WORKSPACE = 7       /* ws_bytes smaller than the workspace query */
+};
+
+/* bits OR-ed into *dev_status by kernels */
+#define LSA_DEV_CAPACITY 1      /* a list was longer than its capacity and was cut */
+#define LSA_DEV_TABLE 2         /* a needed chunk had no valid slot; its rows were skipped */
+#define LSA_DEV_TIMEOUT 4       /* a bounded device wait ran out */
+#define LSA_DEV_INDEX 8         /* an index input was out of range and was skipped */
+
+/* Message of the last error returned on this thread ("" if none). */
+const char *lsa_last_error(void);
+
+/* Library version string. */
+const char *lsa_version(void);
+
+/*
+ * a1 -- Neural Memory Indexer chunk gate.
+ * Passage: gist.science explainer 2.1 ("Scoring-Mechanismus", "Dynamisches
+ * Fetching"); cjcn.com.cn article section 2 (ReLU replaced by Sigmoid, fixed
+ * threshold 0.5, every chunk above it is fetched).
+ *
+ * For each sequence b and each of its chunks s:
+ *   logit = sum_h w[b,h] * (q[b,h,:] . khat[off[b]+s, :]),  I = sigmoid(logit)
+ *   keep s  iff  I >= 0.5  (evaluated as logit >= 0, which is the same test).
+ * Kept chunk indices (relative to the sequence) are written ascending.
+ *
+ *   q          [B, Hn, dn] bf16 (device)
+ *   w          [B, Hn]     bf16 (device), head weights
+ *   khat       [total_chunks, dn] bf16 (device), one compressed key per chunk
+ *   seq_chunk_offset [B+1] int64 (device), sequence b owns rows off[b]..off[b+1]-1
+ *   max_chunks_per_seq     host upper bound of off[b+1]-off[b]
+ *   kept_idx   [B, kept_cap] int32 (device, out): ascending; unused entries -1
+ *   kept_count [B] int32 (device, out): number written (<= kept_cap); a longer
+ *              list sets LSA_DEV_CAPACITY
+ *   logits     [total_chunks] fp32 (device, out, optional)
+ * Supported: dn in {64, 128}, Hn a multiple of 8 up to 128.
+ */
+int lsa_nmi_select(const lsa_bf16 *q, const lsa_bf16 *w, const lsa_bf16 *khat,
+                   const int64_t *seq_chunk_offset, int B, int Hn, int dn,
+                   int64_t total_chunks, int max_chunks_per_seq,
+                   int32_t *kept_idx, int32_t *kept_count, int kept_cap,
+                   float *logits, int32_t *dev_status,
+                   void *ws, size_t ws_bytes, lsa_stream_t stream);
+size_t lsa_nmi_select_workspace_size(int B, int max_chunks_per_seq);
+
+/*
+ * a2 + a3 -- Lightning-Indexer scoring and fine top-k inside the kept chunks.
+ * Passage: gist.science explainer 2.1 ("Gestufte Selektion"); cjcn.com.cn
+ * article section 2 (the native indexer takes a top-k inside the reduced set).
+ *
+ * Candidates of sequence b: every token of every kept chunk c with
+ * c < window_start[b] / 64 (chunks in the recent window are attended anyway),
+ * in ascending position.  Score of token t:
+ *   I_t = sum_h w_li[b,h] * max(0, q_li[b,h,:] . key_t)
+ * The k largest scores are kept, ties to the lower position; the kept
+ * positions are written ascending, followed by -1 up to k.
+ *
+ *   q_li      [B, Hl, dl] bf16, w_li [B, Hl] bf16 (device)
+ *   li_pool   [n_slots, 64, dl] bf16 (device): indexer key of every resident token
+ *   chunk_table [B, table_stride] int32 (device)
+ *   kept_idx  [B, kept_cap], kept_count [B] int32 (device): lsa_nmi_select output
+ *   window_start [B] int32 (device): first position of the recent window, multiple of 64
+ *   topk_idx  [B, k] int32 (device, out); topk_count [B] int32 (device, out)
+ *   scores    [B, kept_cap * 64] fp32 (device, out, optional): candidate scores
+ * Supported: dl in {64, 128}, Hl a multiple of 8 up to 128, 1 <= k <= 65536.
+ */
+int lsa_topk(const lsa_bf16 *q_li, const lsa_bf16 *w_li, const lsa_bf16 *li_pool, int64_t n_slots,
+             const int32_t *chunk_table, int table_stride,
+             const int32_t *kept_idx, const int32_t *kept_count, int kept_cap,
+             const int32_t *window_start, int B, int Hl, int dl, int k,
+             int32_t *topk_idx, int32_t *topk_count, float *scores, int32_t *dev_status,
+             void *ws, size_t ws_bytes, lsa_stream_t stream);
+size_t lsa_topk_workspace_size(int B, int kept_cap);
+
+/*
+ * a3 alone, on given fp32 scores (exact unit entry point).
+ * Sequence b owns scores[cand_offset[b] .. cand_offset[b+1]); writes the
+ * indices (relative to cand_offset[b]) of its min(k, n_b) largest scores,
+ * ties to the lower index, ascending, then -1 up to k.
+ *   cand_offset [B+1] int64 (device); max_cand host upper bound of n_b.
+ */
+int lsa_topk_from_scores(const float *scores, const int64_t *cand_offset, int B, int max_cand, int k,
+                         int32_t *topk_idx, int32_t *topk_count,
+                         void *ws, size_t ws_bytes, lsa_stream_t stream);
+
+/*
+ * a4 -- sparse decode attention over top-k rows plus the recent window.
+ * Passage: cjcn.com.cn article section 2 (core attention over the selected
+ * entries; the most recent 8000 tokens always kept on the GPU); gist.science
+ * explainer 2.1 ("Gestufte Selektion": final core-attention computation).
+ *
+ * Row set of sequence b: S = {topk_idx[b, 0..topk_count[b])} followed by the
+ * positions window_start[b] .. window_start[b] + window_len[b] - 1.  For each
+ * query head h:
+ *   o[b,h,:] = sum_{j in S} softmax_j(scale * q[b,h,:] . K_j) V_j
+ *   lse[b,h] = log sum_{j in S} exp(scale * q[b,h,:] . K_j)
+ * One KV head is shared by all query heads.  Latent layout (v_pool == NULL):
+ * K_j is the dqk-wide row of k_pool and V_j its first dv columns.  Otherwise
+ * V_j is the row of v_pool.
+ *
+ *   q       [B, Hq, dqk] bf16 (device)
+ *   k_pool  [n_slots, 64, k_row_stride] bf16; v_pool [n_slots, 64, v_row_stride] or NULL
+ *   topk_idx [B, k], topk_count [B], window_start [B], window_len [B] int32 (device)
+ *   max_window_len   host upper bound of window_len[b] (sizes the split-K grid)
+ *   out     [B, Hq, dv] fp32 (device, out); lse [B, Hq] fp32 (device, out, optional)
+ * Supported: (Hq, dqk, dv) = (16, 128, 128) with separate K/V pools, and
+ * (128 or 64, 576, 512) latent.  Strides in elements, multiples of 8.
+ */
+int lsa_sparse_decode(const lsa_bf16 *q, const lsa_bf16 *k_pool, int64_t k_row_stride,
+                      const lsa_bf16 *v_pool, int64_t v_row_stride, int64_t n_slots,
+                      const int32_t *chunk_table, int table_stride,
+                      const int32_t *topk_idx, const int32_t *topk_count, int k,
+                      const int32_t *window_start, const int32_t *window_len, int max_window_len,
+                      int B, int Hq, int dqk, int dv, float scale,
+                      float *out, float *lse, int32_t *dev_status,
+                      void *ws, size_t ws_bytes, lsa_stream_t stream);
+size_t lsa_sparse_decode_workspace_size(int B, int Hq, int dqk, int dv, int k, int max_window_len);
+
+/*
+ * a5 -- lookahead reuse: append the decoded token to the recent window.
+ * Passage: gist.science explainer 2.1 ("Periodische Triggerung", tau = 64);
+ * cjcn.com.cn article section 2 (the selection serves the next 64 steps).
+ *
+ * For each sequence b the token at position p = window_start[b] + window_len[b]
+ * gets new_k[b] (and new_v[b], new_li[b]) written into its pool row, then
+ * window_len[b] is incremented.  The chunk of p must already have a slot.
+ *   new_k [B, k_width], new_v [B, v_width] or NULL, new_li [B, dl] or NULL (device)
+ */
+int lsa_append_token(const lsa_bf16 *new_k, const lsa_bf16 *new_v, const lsa_bf16 *new_li,
+                     lsa_bf16 *k_pool, int64_t k_row_stride, int k_width,
+                     lsa_bf16 *v_pool, int64_t v_row_stride, int v_width,
+                     lsa_bf16 *li_pool, int dl, int64_t n_slots,
+                     const int32_t *chunk_table, int table_stride,
+                     const int32_t *window_start, int32_t *window_len, int B,
+                     int32_t *dev_status, lsa_stream_t stream);
+
+/*
+ * a6 -- cold-chunk fetch from the pinned host pool (one sequence).
+ * Passage: cjcn.com.cn article section 2 (unselected chunks stay in CPU
+ * memory; selected ones are moved to GPU memory); gist.science explainer 2.1
+ * ("Dynamisches Fetching" from the CPU cold pool).
+ *
+ * Every kept chunk c (from the HOST copy of the kept list) with
+ * c < first_window_chunk is given device slot first_free_slot + j (j = its
+ * rank among those chunks) in each of the n_pools pools; runs of consecutive
+ * chunks are copied with one cudaMemcpyAsync per pool on `stream`.  The slots
+ * are written into chunk_table_host (pinned, table_len entries, caller-owned),
+ * which is then copied to chunk_table_dev on the same stream, and `done` (if
+ * not NULL) is recorded after the last copy.  The caller orders later work
+ * after `done`.
+ *   host_pools[i]  pinned host base of pool i, [n_host_chunks, chunk_bytes[i]]
+ *   dev_pools[i]   device base of pool i, [n_slots, chunk_bytes[i]]
+ *   n_fetched      (host, out) number of chunks copied
+ */
+int lsa_gather_chunks(int n_pools, const void *const *host_pools, const size_t *chunk_bytes,
+                      void *const *dev_pools, int64_t n_host_chunks, int64_t n_slots,
+                      const int32_t *kept_idx_host, int kept_count_host, int first_window_chunk,
+                      int first_free_slot, int32_t *chunk_table_host, int32_t *chunk_table_dev,
+                      int table_len, lsa_stream_t stream, lsa_event_t done, int *n_fetched);
+
+/*
+ * a7 (offline) -- cross-layer majority-vote labels for one decode window.
+ * Passage: gist.science explainer 2.2 (softmax, top-p 0.6, at least theta = 3
+ * layers); cjcn.com.cn article section 3 (a chunk selected by at least 3 layers
+ * at the same time is golden; golden chunks of all steps are merged).
+ *
+ * For each layer l and step t: p = softmax(scores[l,t,:]); order chunks by
+ * score descending (ties to the lower index); keep the smallest prefix whose
+ * cumulative p reaches top_p (crossing chunk included).  count[t][c] = number
+ * of layers keeping c at step t.
+ *   mode 0: max_votes[c] = max_t count[t][c]
+ *   mode 1: max_votes[c] = number of distinct layers keeping c at any step
+ *   labels[c] = (max_votes[c] >= min_layers)
+ *   scores [n_layers, n_steps, n_chunks] fp32 (device); labels [n_chunks] uint8
+ *   (device, out); max_votes [n_chunks] int32 (device, out, optional)
+ * Supported: 1 <= n_layers <= 64, 1 <= n_chunks <= 16384.
+ */
+int lsa_label_vote(const float *scores, int n_layers, int n_steps, int n_chunks,
+                   float top_p, int min_layers, int mode,
+                   uint8_t *labels, int32_t *max_votes,
+                   void *ws, size_t ws_bytes, lsa_stream_t stream);
+size_t lsa_label_vote_workspace_size(int n_layers, int n_steps, int n_chunks);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSA_H */

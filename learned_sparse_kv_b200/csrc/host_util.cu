@@ -1,0 +1,48 @@
+// host_util.cu -- error reporting and device queries shared by the ABI entry points.
+#include <stdarg.h>
+#include <string.h>
+
+#include "common.cuh"
+
+namespace lsa {
+
+static thread_local char g_last_error[512] = "";
+
+void set_error(const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+}
+
+int fail(int code, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int check_launch(const char *what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(LSA_ERR_CUDA, "%s launch: %s", what, cudaGetErrorString(e));
+    return LSA_OK;
+}
+
+int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+}  // namespace lsa
+
+extern "C" const char *lsa_last_error(void) { return lsa::g_last_error; }
+
+extern "C" const char *lsa_version(void) { return "lsa-b200 0.1 (sm_100a)"; }

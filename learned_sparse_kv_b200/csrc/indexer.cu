@@ -1,0 +1,298 @@
+// indexer.cu -- multi-head indexer scores on tensor cores, shared by
+//   a1  the Neural Memory Indexer chunk gate (identity activation, then
+//       sigmoid >= 0.5, i.e. logit >= 0) and its order-preserving compaction;
+//   a2  the Lightning-Indexer token scores (ReLU activation) over the tokens of
+//       kept chunks that lie before the recent window.
+// Both compute score(row) = sum_h w_h * act(q_h . key_row) for 64 key rows at a
+// time: a [64 x D] . [D x H] product on mma.sync (bf16 in, fp32 accumulate),
+// then the activation and the weighted head sum in the epilogue.
+// (arXiv 2606.09079 as described by the gist.science explainer 2.1 and the
+// cjcn.com.cn article section 2.)
+#include "block_scan.cuh"
+#include "common.cuh"
+
+namespace lsa {
+
+constexpr int kRows = 64;        // key rows per tile (one chunk of tokens, or 64 chunk keys)
+constexpr int kMaxHeads = 128;
+
+struct IdxSmem {
+    // keys [64][D] and queries [H][D], rows swizzled in 16-byte chunks
+    alignas(128) uint16_t keys[kRows * 128];
+    alignas(128) uint16_t q[kMaxHeads * 128];
+    float w[kMaxHeads];
+    float score[kRows];
+};
+
+// Loads q[H][D] (bf16) and w[H] of one sequence into shared memory.
+template <int D>
+__device__ void load_queries(IdxSmem &sm, const uint16_t *q, const uint16_t *w, int H) {
+    constexpr int CPR = D * 2 / 16;  // 16-byte chunks per row
+    for (int i = threadIdx.x; i < H * CPR; i += blockDim.x) {
+        int r = i / CPR, c = i % CPR;
+        cp_async16(reinterpret_cast<char *>(sm.q) + swz(r, c, D * 2), q + (size_t)r * D + c * 8);
+    }
+    for (int h = threadIdx.x; h < H; h += blockDim.x) sm.w[h] = bf16_to_f32(w[h]);
+}
+
+// Loads up to 64 key rows; rows >= n_valid are zero-filled.  row_ptr(r) gives the global row.
+template <int D, class RowPtr>
+__device__ void load_keys(IdxSmem &sm, RowPtr row_ptr, int n_valid) {
+    constexpr int CPR = D * 2 / 16;
+    for (int i = threadIdx.x; i < kRows * CPR; i += blockDim.x) {
+        int r = i / CPR, c = i % CPR;
+        const uint16_t *src = r < n_valid ? row_ptr(r) : nullptr;
+        void *dst = reinterpret_cast<char *>(sm.keys) + swz(r, c, D * 2);
+        if (src)
+            cp_async16(dst, src + c * 8);
+        else
+            *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
+    }
+}
+
+// 4 warps: warp i scores rows 16i..16i+15.  Result in sm.score[0..63].
+template <int D, bool RELU>
+__device__ void score_tile(IdxSmem &sm, int H) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int m0 = warp * 16;
+    float acc[kMaxHeads / 8][4];
+#pragma unroll
+    for (int i = 0; i < kMaxHeads / 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+    const uint32_t kbase = smem_addr(sm.keys), qbase = smem_addr(sm.q);
+#pragma unroll
+    for (int kc = 0; kc < D / 8; kc += 2) {
+        uint32_t a[4];
+        ldmatrix_x4(a[0], a[1], a[2], a[3], kbase + swz(m0 + (lane & 15), kc + (lane >> 4), D * 2));
+#pragma unroll
+        for (int nt = 0; nt < kMaxHeads / 8; nt += 2) {
+            if (nt * 8 < H) {
+                uint32_t b0, b1, b2, b3;
+                int head = nt * 8 + (lane & 7) + ((lane >> 4) << 3);
+                int chunk = kc + ((lane >> 3) & 1);
+                ldmatrix_x4(b0, b1, b2, b3, qbase + swz(head, chunk, D * 2));
+                mma_bf16_16816(acc[nt], a, b0, b1);
+                if ((nt + 1) * 8 < H) mma_bf16_16816(acc[nt + 1], a, b2, b3);
+            }
+        }
+    }
+    const int g = lane >> 2, qd = lane & 3;
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < kMaxHeads / 8; ++nt) {
+        if (nt * 8 < H) {
+            float w0 = sm.w[nt * 8 + 2 * qd], w1 = sm.w[nt * 8 + 2 * qd + 1];
+            float v0 = acc[nt][0], v1 = acc[nt][1], v2 = acc[nt][2], v3 = acc[nt][3];
+            if (RELU) {
+                v0 = fmaxf(v0, 0.f); v1 = fmaxf(v1, 0.f); v2 = fmaxf(v2, 0.f); v3 = fmaxf(v3, 0.f);
+            }
+            s0 += w0 * v0 + w1 * v1;
+            s1 += w0 * v2 + w1 * v3;
+        }
+    }
+    s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
+    s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
+    s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+    s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+    if (qd == 0) {
+        sm.score[m0 + g] = s0;
+        sm.score[m0 + g + 8] = s1;
+    }
+}
+
+// ------------------------------------------------------------------- a1 ----
+
+// grid (tiles of 64 chunks, B).  Writes logits and one 64-bit gate mask per tile.
+template <int D>
+__global__ void __launch_bounds__(128) nmi_score_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ w,
+                                                        const uint16_t *__restrict__ khat,
+                                                        const int64_t *__restrict__ off, int H, int tiles_per_seq,
+                                                        float *__restrict__ logits, unsigned long long *__restrict__ masks) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    IdxSmem &sm = *reinterpret_cast<IdxSmem *>(smem_raw);
+    const int b = blockIdx.y, tile = blockIdx.x;
+    const int64_t first = off[b];
+    const int64_t n_ch = off[b + 1] - first;
+    const int64_t s0 = (int64_t)tile * kRows;
+    if (s0 >= n_ch) {
+        if (threadIdx.x == 0) masks[(size_t)b * tiles_per_seq + tile] = 0ull;
+        return;
+    }
+    const int n_valid = (int)(n_ch - s0 < kRows ? n_ch - s0 : kRows);
+    load_queries<D>(sm, q + (size_t)b * H * D, w + (size_t)b * H, H);
+    load_keys<D>(sm, [&](int r) { return khat + (size_t)(first + s0 + r) * D; }, n_valid);
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+    score_tile<D, false>(sm, H);
+    __syncthreads();
+    __shared__ unsigned halves[2];
+    const int r = threadIdx.x;
+    bool keep = false;
+    if (r < kRows) {
+        float l = sm.score[r];
+        keep = r < n_valid && l >= 0.f;  // sigmoid(l) >= 0.5  <=>  l >= 0
+        if (r < n_valid && logits) logits[first + s0 + r] = l;
+    }
+    unsigned bits = __ballot_sync(0xffffffffu, keep);  // warp 0: rows 0..31, warp 1: rows 32..63
+    if ((r & 31) == 0 && r < kRows) halves[r >> 5] = bits;
+    __syncthreads();
+    if (r == 0)
+        masks[(size_t)b * tiles_per_seq + tile] = (unsigned long long)halves[0] | ((unsigned long long)halves[1] << 32);
+}
+
+// grid B, 256 threads: gate masks -> ascending kept list, count, capacity flag.
+__global__ void __launch_bounds__(256) nmi_compact_kernel(const unsigned long long *__restrict__ masks,
+                                                          const int64_t *__restrict__ off, int tiles_per_seq,
+                                                          int32_t *__restrict__ kept_idx, int32_t *__restrict__ kept_count,
+                                                          int kept_cap, int32_t *status) {
+    __shared__ int warp_tot[256 / 32 + 1];
+    const int b = blockIdx.x;
+    const int64_t n_ch = off[b + 1] - off[b];
+    int n_words = (int)((n_ch + kRows - 1) / kRows);
+    if (n_words > tiles_per_seq) {  // more chunks than the host-declared maximum: score only those
+        n_words = tiles_per_seq;
+        if (threadIdx.x == 0) flag(status, LSA_DEV_INDEX);
+    }
+    const int per = (n_words + 255) / 256;
+    const int w0 = min(n_words, (int)threadIdx.x * per), w1 = min(n_words, w0 + per);
+    const unsigned long long *m = masks + (size_t)b * tiles_per_seq;
+    int mine = 0;
+    for (int i = w0; i < w1; ++i) mine += __popcll(m[i]);
+    int total;
+    int pos = block_exclusive_scan<256>(mine, warp_tot, &total);
+    int32_t *out = kept_idx + (size_t)b * kept_cap;
+    for (int i = w0; i < w1; ++i) {
+        unsigned long long bits = m[i];
+        while (bits) {
+            int bit = __ffsll((long long)bits) - 1;
+            bits &= bits - 1;
+            if (pos < kept_cap) out[pos] = i * kRows + bit;
+            ++pos;
+        }
+    }
+    for (int j = total + threadIdx.x; j < kept_cap; j += 256) out[j] = -1;
+    if (threadIdx.x == 0) {
+        kept_count[b] = min(total, kept_cap);
+        if (total > kept_cap) flag(status, LSA_DEV_CAPACITY);
+    }
+}
+
+// ------------------------------------------------------------------- a2 ----
+
+// Number of kept chunks below the window: kept lists are ascending.
+__device__ __forceinline__ int cold_kept(const int32_t *kept, int count, int first_window_chunk) {
+    int lo = 0, hi = count;
+    while (lo < hi) {
+        int mid = (lo + hi) >> 1;
+        if (kept[mid] < first_window_chunk) lo = mid + 1;
+        else hi = mid;
+    }
+    return lo;
+}
+
+// grid (G, B): CTA x of sequence b scores kept cold chunks x, x+G, ...
+template <int D>
+__global__ void __launch_bounds__(128) li_score_kernel(const uint16_t *__restrict__ q_li, const uint16_t *__restrict__ w_li,
+                                                       const uint16_t *__restrict__ li_pool, int64_t n_slots,
+                                                       const int32_t *__restrict__ table, int table_stride,
+                                                       const int32_t *__restrict__ kept_idx,
+                                                       const int32_t *__restrict__ kept_count, int kept_cap,
+                                                       const int32_t *__restrict__ window_start, int H,
+                                                       float *__restrict__ scores, int32_t *status) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    IdxSmem &sm = *reinterpret_cast<IdxSmem *>(smem_raw);
+    const int b = blockIdx.y;
+    const int32_t *kept = kept_idx + (size_t)b * kept_cap;
+    const int cnt = min(kept_count[b], kept_cap);
+    const int n_cold = cold_kept(kept, cnt, window_start[b] / LSA_CHUNK);
+    if ((int)blockIdx.x >= n_cold) return;
+    load_queries<D>(sm, q_li + (size_t)b * H * D, w_li + (size_t)b * H, H);
+    const int32_t *trow = table + (size_t)b * table_stride;
+    float *out = scores + (size_t)b * kept_cap * kRows;
+    for (int j = blockIdx.x; j < n_cold; j += gridDim.x) {
+        const int chunk = kept[j];
+        int slot = (chunk >= 0 && chunk < table_stride) ? trow[chunk] : -1;
+        const bool ok = slot >= 0 && slot < n_slots;
+        if (!ok && threadIdx.x == 0) flag(status, LSA_DEV_TABLE);
+        load_keys<D>(sm, [&](int r) { return li_pool + ((size_t)slot * kRows + r) * D; }, ok ? kRows : 0);
+        cp_async_commit();
+        cp_async_wait<0>();
+        __syncthreads();
+        score_tile<D, true>(sm, H);
+        __syncthreads();
+        if (threadIdx.x < kRows) out[(size_t)j * kRows + threadIdx.x] = ok ? sm.score[threadIdx.x] : -INFINITY;
+        __syncthreads();
+    }
+}
+
+// ------------------------------------------------------------ host launch --
+
+static bool heads_ok(int H) { return H >= 8 && H <= kMaxHeads && H % 8 == 0; }
+
+int launch_li_scores(const uint16_t *q_li, const uint16_t *w_li, const uint16_t *li_pool, int64_t n_slots,
+                     const int32_t *table, int table_stride, const int32_t *kept_idx, const int32_t *kept_count,
+                     int kept_cap, const int32_t *window_start, int B, int H, int D, float *scores,
+                     int32_t *status, cudaStream_t stream) {
+    const size_t smem = sizeof(IdxSmem);
+    int per_seq = (sm_count() * 8 + B - 1) / B;
+    per_seq = max(1, min(per_seq, kept_cap));
+    dim3 grid(per_seq, B);
+    if (D == 128) {
+        cudaFuncSetAttribute(li_score_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        li_score_kernel<128><<<grid, 128, smem, stream>>>(q_li, w_li, li_pool, n_slots, table, table_stride, kept_idx,
+                                                          kept_count, kept_cap, window_start, H, scores, status);
+    } else {
+        cudaFuncSetAttribute(li_score_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        li_score_kernel<64><<<grid, 128, smem, stream>>>(q_li, w_li, li_pool, n_slots, table, table_stride, kept_idx,
+                                                         kept_count, kept_cap, window_start, H, scores, status);
+    }
+    return check_launch("li_score_kernel");
+}
+
+bool indexer_shape_ok(int H, int D) { return heads_ok(H) && (D == 64 || D == 128); }
+
+}  // namespace lsa
+
+using namespace lsa;
+
+extern "C" size_t lsa_nmi_select_workspace_size(int B, int max_chunks_per_seq) {
+    if (B <= 0 || max_chunks_per_seq < 0) return 0;
+    Carver c(nullptr);
+    int tiles = (max_chunks_per_seq + kRows - 1) / kRows;
+    c.take<unsigned long long>((size_t)B * (tiles > 0 ? tiles : 1));
+    return align_up(c.used, 256);
+}
+
+extern "C" int lsa_nmi_select(const lsa_bf16 *q, const lsa_bf16 *w, const lsa_bf16 *khat,
+                              const int64_t *seq_chunk_offset, int B, int Hn, int dn, int64_t total_chunks,
+                              int max_chunks_per_seq, int32_t *kept_idx, int32_t *kept_count, int kept_cap,
+                              float *logits, int32_t *dev_status, void *ws, size_t ws_bytes, lsa_stream_t stream) {
+    LSA_REQUIRE(B > 0, LSA_ERR_INVALID_ARG, "lsa_nmi_select: B must be positive (got %d)", B);
+    LSA_REQUIRE(q && w && khat && seq_chunk_offset && kept_idx && kept_count, LSA_ERR_INVALID_ARG,
+                "lsa_nmi_select: null input or output pointer");
+    LSA_REQUIRE(indexer_shape_ok(Hn, dn), LSA_ERR_SHAPE,
+                "lsa_nmi_select: unsupported Hn=%d dn=%d (dn in {64,128}, Hn multiple of 8 up to 128)", Hn, dn);
+    LSA_REQUIRE(max_chunks_per_seq >= 0 && total_chunks >= 0 && kept_cap >= 1, LSA_ERR_INVALID_ARG,
+                "lsa_nmi_select: bad sizes (max_chunks_per_seq=%d total_chunks=%lld kept_cap=%d)",
+                max_chunks_per_seq, (long long)total_chunks, kept_cap);
+    LSA_REQUIRE(ws_bytes >= lsa_nmi_select_workspace_size(B, max_chunks_per_seq) && ws, LSA_ERR_WORKSPACE,
+                "lsa_nmi_select: workspace of %zu bytes, %zu needed", ws_bytes,
+                lsa_nmi_select_workspace_size(B, max_chunks_per_seq));
+    const int tiles = max(1, (max_chunks_per_seq + kRows - 1) / kRows);
+    Carver c(ws);
+    auto *masks = c.take<unsigned long long>((size_t)B * tiles);
+    const size_t smem = sizeof(IdxSmem);
+    dim3 grid(tiles, B);
+    if (dn == 128) {
+        LSA_CUDA(cudaFuncSetAttribute(nmi_score_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+        nmi_score_kernel<128><<<grid, 128, smem, stream>>>(q, w, khat, seq_chunk_offset, Hn, tiles, logits, masks);
+    } else {
+        LSA_CUDA(cudaFuncSetAttribute(nmi_score_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+        nmi_score_kernel<64><<<grid, 128, smem, stream>>>(q, w, khat, seq_chunk_offset, Hn, tiles, logits, masks);
+    }
+    int rc = check_launch("nmi_score_kernel");
+    if (rc) return rc;
+    nmi_compact_kernel<<<B, 256, 0, stream>>>(masks, seq_chunk_offset, tiles, kept_idx, kept_count, kept_cap,
+                                              dev_status);
+    return check_launch("nmi_compact_kernel");
+}

@@ -1,0 +1,241 @@
+"""ctypes binding of liblsa.so: argument marshalling only.
+
+Every step of the decode path runs in the library's CUDA kernels.  Tensors are
+torch tensors (bf16 inputs as torch.bfloat16); the binding allocates outputs
+and workspaces with torch, passes raw pointers plus the current CUDA stream,
+and turns a non-zero status into an LSAError.  There is no CPU fallback: if
+the library is missing the import fails.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblsa.so")
+
+CHUNK = 64
+DEV_CAPACITY, DEV_TABLE, DEV_TIMEOUT, DEV_INDEX = 1, 2, 4, 8
+ERRORS = {1: "INVALID_ARG", 2: "SHAPE", 3: "CUDA", 4: "CAPACITY", 5: "TIMEOUT", 6: "TABLE", 7: "WORKSPACE"}
+
+
+class LSAError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"LSA error {code} ({ERRORS.get(code, '?')}): {msg}")
+        self.code = code
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"liblsa.so not found at {LIB_PATH}; build it with "
+                          f"`python -m learned_sparse_kv_b200.build` (no CPU fallback exists)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, I64, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    sig = {
+        "lsa_nmi_select": ([P, P, P, P, I, I, I, I64, I, P, P, I, P, P, P, SZ, P], I),
+        "lsa_nmi_select_workspace_size": ([I, I], SZ),
+        "lsa_topk": ([P, P, P, I64, P, I, P, P, I, P, I, I, I, I, P, P, P, P, P, SZ, P], I),
+        "lsa_topk_workspace_size": ([I, I], SZ),
+        "lsa_topk_from_scores": ([P, P, I, I, I, P, P, P, SZ, P], I),
+        "lsa_sparse_decode": ([P, P, I64, P, I64, I64, P, I, P, P, I, P, P, I, I, I, I, I, F, P, P, P, P, SZ, P], I),
+        "lsa_sparse_decode_workspace_size": ([I, I, I, I, I, I], SZ),
+        "lsa_append_token": ([P, P, P, P, I64, I, P, I64, I, P, I, I64, P, I, P, P, I, P, P], I),
+        "lsa_gather_chunks": ([I, P, P, P, I64, I64, P, I, I, I, P, P, I, P, P, P], I),
+        "lsa_label_vote": ([P, I, I, I, F, I, I, P, P, P, SZ, P], I),
+        "lsa_label_vote_workspace_size": ([I, I, I], SZ),
+        "lsa_last_error": ([], ctypes.c_char_p),
+        "lsa_version": ([], ctypes.c_char_p),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+_lib = _load()
+
+
+def version() -> str:
+    return _lib.lsa_version().decode()
+
+
+def _check(rc):
+    if rc != 0:
+        raise LSAError(rc, _lib.lsa_last_error().decode())
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev(t, dtype, name):
+    if not (isinstance(t, torch.Tensor) and t.is_cuda):
+        raise LSAError(1, f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise LSAError(1, f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise LSAError(1, f"{name} must be contiguous")
+    return t
+
+
+def _ws(nbytes, device, ws=None):
+    if ws is not None and ws.numel() >= nbytes:
+        return ws
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+# ------------------------------------------------------------------- a1 ----
+
+def nmi_select_workspace_size(B, max_chunks_per_seq):
+    return _lib.lsa_nmi_select_workspace_size(B, max_chunks_per_seq)
+
+
+def nmi_select(q, w, khat, seq_chunk_offset, max_chunks_per_seq, kept_cap, *, logits=None, status=None,
+               kept_idx=None, kept_count=None, ws=None, stream=None):
+    """Chunk gate.  Returns (kept_idx [B, kept_cap] int32, kept_count [B] int32)."""
+    B, Hn, dn = q.shape
+    _dev(q, torch.bfloat16, "q"); _dev(w, torch.bfloat16, "w"); _dev(khat, torch.bfloat16, "khat")
+    _dev(seq_chunk_offset, torch.int64, "seq_chunk_offset")
+    dev = q.device
+    if kept_idx is None:
+        kept_idx = torch.empty(B, kept_cap, dtype=torch.int32, device=dev)
+    if kept_count is None:
+        kept_count = torch.empty(B, dtype=torch.int32, device=dev)
+    ws = _ws(nmi_select_workspace_size(B, max_chunks_per_seq), dev, ws)
+    _check(_lib.lsa_nmi_select(_ptr(q), _ptr(w), _ptr(khat), _ptr(seq_chunk_offset), B, Hn, dn, khat.shape[0],
+                               max_chunks_per_seq, _ptr(kept_idx), _ptr(kept_count), kept_cap, _ptr(logits),
+                               _ptr(status), _ptr(ws), ws.numel(), _stream(stream)))
+    return kept_idx, kept_count
+
+
+# ------------------------------------------------------------- a2 + a3 ----
+
+def topk_workspace_size(B, kept_cap):
+    return _lib.lsa_topk_workspace_size(B, kept_cap)
+
+
+def topk(q_li, w_li, li_pool, chunk_table, kept_idx, kept_count, window_start, k, *, scores=None, status=None,
+         topk_idx=None, topk_count=None, ws=None, stream=None):
+    """Lightning-indexer scores + fine top-k.  Returns (topk_idx [B,k], topk_count [B])."""
+    B, Hl, dl = q_li.shape
+    _dev(q_li, torch.bfloat16, "q_li"); _dev(w_li, torch.bfloat16, "w_li"); _dev(li_pool, torch.bfloat16, "li_pool")
+    _dev(chunk_table, torch.int32, "chunk_table"); _dev(kept_idx, torch.int32, "kept_idx")
+    _dev(kept_count, torch.int32, "kept_count"); _dev(window_start, torch.int32, "window_start")
+    dev = q_li.device
+    kept_cap = kept_idx.shape[1]
+    if topk_idx is None:
+        topk_idx = torch.empty(B, k, dtype=torch.int32, device=dev)
+    if topk_count is None:
+        topk_count = torch.empty(B, dtype=torch.int32, device=dev)
+    ws = _ws(topk_workspace_size(B, kept_cap), dev, ws) if scores is None else None
+    _check(_lib.lsa_topk(_ptr(q_li), _ptr(w_li), _ptr(li_pool), li_pool.shape[0], _ptr(chunk_table),
+                         chunk_table.shape[1], _ptr(kept_idx), _ptr(kept_count), kept_cap, _ptr(window_start),
+                         B, Hl, dl, k, _ptr(topk_idx), _ptr(topk_count), _ptr(scores), _ptr(status), _ptr(ws),
+                         0 if ws is None else ws.numel(), _stream(stream)))
+    return topk_idx, topk_count
+
+
+def topk_from_scores(scores, cand_offset, max_cand, k, *, stream=None):
+    """Exact top-k of given fp32 scores per segment.  Returns (idx [B,k], count [B])."""
+    _dev(scores, torch.float32, "scores"); _dev(cand_offset, torch.int64, "cand_offset")
+    B = cand_offset.shape[0] - 1
+    idx = torch.empty(B, k, dtype=torch.int32, device=scores.device)
+    cnt = torch.empty(B, dtype=torch.int32, device=scores.device)
+    _check(_lib.lsa_topk_from_scores(_ptr(scores), _ptr(cand_offset), B, max_cand, k, _ptr(idx), _ptr(cnt),
+                                     None, 0, _stream(stream)))
+    return idx, cnt
+
+
+# ------------------------------------------------------------------- a4 ----
+
+def sparse_decode_workspace_size(B, Hq, dqk, dv, k, max_window_len):
+    return _lib.lsa_sparse_decode_workspace_size(B, Hq, dqk, dv, k, max_window_len)
+
+
+def sparse_decode(q, k_pool, v_pool, chunk_table, topk_idx, topk_count, window_start, window_len, max_window_len,
+                  dv, scale, *, out=None, lse=None, want_lse=True, status=None, ws=None, stream=None):
+    """Attention over top-k rows + window.  k_pool [slots,64,Kw]; v_pool None (latent) or [slots,64,Vw].
+
+    Returns (out [B,Hq,dv] fp32, lse [B,Hq] fp32 or None).
+    """
+    B, Hq, dqk = q.shape
+    _dev(q, torch.bfloat16, "q"); _dev(k_pool, torch.bfloat16, "k_pool")
+    if v_pool is not None:
+        _dev(v_pool, torch.bfloat16, "v_pool")
+    for name, t in (("chunk_table", chunk_table), ("topk_idx", topk_idx), ("topk_count", topk_count),
+                    ("window_start", window_start), ("window_len", window_len)):
+        _dev(t, torch.int32, name)
+    dev = q.device
+    k = topk_idx.shape[1]
+    if out is None:
+        out = torch.empty(B, Hq, dv, dtype=torch.float32, device=dev)
+    if lse is None and want_lse:
+        lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    ws = _ws(sparse_decode_workspace_size(B, Hq, dqk, dv, k, max_window_len), dev, ws)
+    _check(_lib.lsa_sparse_decode(_ptr(q), _ptr(k_pool), k_pool.shape[-1], _ptr(v_pool),
+                                  0 if v_pool is None else v_pool.shape[-1], k_pool.shape[0], _ptr(chunk_table),
+                                  chunk_table.shape[1], _ptr(topk_idx), _ptr(topk_count), k, _ptr(window_start),
+                                  _ptr(window_len), max_window_len, B, Hq, dqk, dv, float(scale), _ptr(out), _ptr(lse),
+                                  _ptr(status), _ptr(ws), ws.numel(), _stream(stream)))
+    return out, lse
+
+
+# ------------------------------------------------------------- a5, a6 ----
+
+def append_token(new_k, new_v, new_li, k_pool, v_pool, li_pool, chunk_table, window_start, window_len, *,
+                 status=None, stream=None):
+    """Writes the decoded token's rows at window_start + window_len and bumps window_len."""
+    B, kw = new_k.shape
+    _check(_lib.lsa_append_token(_ptr(new_k), _ptr(new_v), _ptr(new_li), _ptr(k_pool), k_pool.shape[-1], kw,
+                                 _ptr(v_pool), 0 if v_pool is None else v_pool.shape[-1],
+                                 0 if new_v is None else new_v.shape[1], _ptr(li_pool),
+                                 0 if li_pool is None else li_pool.shape[-1], k_pool.shape[0], _ptr(chunk_table),
+                                 chunk_table.shape[1], _ptr(window_start), _ptr(window_len), B, _ptr(status),
+                                 _stream(stream)))
+
+
+def gather_chunks(host_pools, dev_pools, kept_idx_host, first_window_chunk, first_free_slot, chunk_table_host,
+                  chunk_table_dev, *, stream=None, done=None):
+    """Copies kept cold chunks (host-side kept list) into device slots on `stream`.
+
+    host_pools: pinned CPU tensors [n_chunks, 64, width]; dev_pools: CUDA tensors [n_slots, 64, width];
+    chunk_table_host: pinned int32 [table_len]; chunk_table_dev: int32 [table_len] (device).
+    Returns the number of chunks copied.
+    """
+    n = len(host_pools)
+    HP = (ctypes.c_void_p * n)(*[t.data_ptr() for t in host_pools])
+    DP = (ctypes.c_void_p * n)(*[t.data_ptr() for t in dev_pools])
+    CB = (ctypes.c_size_t * n)(*[t[0].numel() * t.element_size() for t in host_pools])
+    kept = kept_idx_host.to(torch.int32).contiguous()
+    nf = ctypes.c_int(0)
+    _check(_lib.lsa_gather_chunks(n, HP, CB, DP, host_pools[0].shape[0], dev_pools[0].shape[0], _ptr(kept),
+                                  kept.numel(), first_window_chunk, first_free_slot, _ptr(chunk_table_host),
+                                  _ptr(chunk_table_dev), chunk_table_host.numel(), _stream(stream),
+                                  None if done is None else ctypes.c_void_p(done.cuda_event), ctypes.byref(nf)))
+    return nf.value
+
+
+# ------------------------------------------------------------------- a7 ----
+
+def label_vote_workspace_size(n_layers, n_steps, n_chunks):
+    return _lib.lsa_label_vote_workspace_size(n_layers, n_steps, n_chunks)
+
+
+def label_vote(scores, top_p=0.6, min_layers=3, mode=0, *, ws=None, stream=None):
+    """Cross-layer majority vote.  scores [layers, steps, chunks] fp32 -> (labels uint8, max_votes int32)."""
+    _dev(scores, torch.float32, "scores")
+    L, T, N = scores.shape
+    labels = torch.empty(N, dtype=torch.uint8, device=scores.device)
+    votes = torch.empty(N, dtype=torch.int32, device=scores.device)
+    ws = _ws(label_vote_workspace_size(L, T, N), scores.device, ws)
+    _check(_lib.lsa_label_vote(_ptr(scores), L, T, N, float(top_p), int(min_layers), int(mode), _ptr(labels),
+                               _ptr(votes), _ptr(ws), ws.numel(), _stream(stream)))
+    return labels, votes

@@ -1,0 +1,96 @@
+"""Places a generated workload on a CUDA device (layout only: copies, no method arithmetic).
+
+Two phases so that a test can adjust inputs between them:
+  host = host_build(wl)          numpy bf16 bits, one array per pool in device-slot layout
+  dev = upload(host, device)     torch tensors for learned_sparse_kv_b200.decode.Window
+
+The host pools already hold the rows of the tokens appended during the window
+(positions ctx .. ctx+steps-1); the device append writes the same values again.
+For a cold workload the device pools hold only the window chunks, and
+host["oracle_pools"] / host["oracle_table"] give the fully resident view.
+"""
+import numpy as np
+import torch
+
+from .generate import (CHUNK, Workload, cold_layout, host_pool, kv_pools, nmi_inputs, resident_layout,
+                       step_inputs)
+
+
+def bf16(bits: np.ndarray, device=None) -> torch.Tensor:
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+    return t.to(device) if device is not None else t
+
+
+def i32(a, device) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
+
+
+def stacked_steps(wl: Workload, steps: int):
+    per = [step_inputs(wl, s) for s in range(steps)]
+    return {key: np.stack([p[key] for p in per]) for key in per[0]}
+
+
+def _kinds(wl):
+    return ["kv", "li"] if wl.latent else ["k", "v", "li"]
+
+
+def _write_new_rows(wl, pools, table, st, steps):
+    for s in range(steps):
+        for b in range(wl.B):
+            pos = wl.ctx[b] + s
+            slot, row = table[b, pos // CHUNK], pos % CHUNK
+            if wl.latent:
+                pools["kv"][slot, row] = st["new_kv"][s, b]
+            else:
+                pools["k"][slot, row] = st["new_k"][s, b]
+                pools["v"][slot, row] = st["new_v"][s, b]
+            pools["li"][slot, row] = st["new_li"][s, b]
+
+
+def host_build(wl: Workload, steps: int = None, nmi=None, structural: bool = True, fetch_fraction: float = 0.25):
+    steps = wl.steps if steps is None else steps
+    nm = nmi if nmi is not None else nmi_inputs(wl, structural=structural)
+    st = stacked_steps(wl, steps)
+    host = dict(wl=wl, steps=steps, nmi=nm, step=st, max_chunks=max(wl.n_ch), kept_cap=max(wl.n_ch))
+    if wl.cold:
+        lay = cold_layout(wl, kept_cap=int(np.ceil(fetch_fraction * wl.n_ch[0])))
+        fw = lay["first_window_chunk"]
+        host["pools"] = kv_pools(wl, lay, chunks_of=lambda b: np.arange(fw, wl.n_ch[b]))
+        hp = host_pool(wl, 0)
+        host["cold_pools"] = hp
+        # oracle view: chunk c at slot c, the appended chunk at slot n_ch
+        otab = np.arange(wl.n_ch[0] + 1, dtype=np.int32)[None, :]
+        opools = {k: np.concatenate([hp[k], np.zeros((1,) + hp[k].shape[1:], np.uint16)]) for k in _kinds(wl)}
+        _write_new_rows(wl, opools, otab, st, steps)
+        _write_new_rows(wl, host["pools"], lay["chunk_table"], st, steps)
+        host.update(oracle_pools=opools, oracle_table=otab, first_window_chunk=fw, first_free_slot=lay["fetch_base"])
+    else:
+        lay = resident_layout(wl)
+        host["pools"] = kv_pools(wl, lay)
+        _write_new_rows(wl, host["pools"], lay["chunk_table"], st, steps)
+        host.update(oracle_pools=host["pools"], oracle_table=lay["chunk_table"])
+    host["chunk_table"] = lay["chunk_table"]
+    host["window_start"] = np.asarray(lay["window_start"], np.int32)
+    return host
+
+
+def upload(host, device):
+    """Returns (shapes, tensors, max_chunks_per_seq, kept_cap, cold) for decode.Window."""
+    wl, nm, st = host["wl"], host["nmi"], host["step"]
+    t = {"q_nmi": bf16(nm["q"], device), "w_nmi": bf16(nm["w"], device), "khat": bf16(nm["khat"], device),
+         "seq_chunk_offset": torch.from_numpy(nm["seq_chunk_offset"]).to(device)}
+    for key, v in st.items():
+        t[key] = bf16(v, device)
+    for k, v in host["pools"].items():
+        t[k] = bf16(v, device)
+    t["chunk_table"] = i32(host["chunk_table"], device)
+    t["window_start"] = i32(host["window_start"], device)
+    cold = None
+    if wl.cold:
+        cold = dict(host_pools=[bf16(host["cold_pools"][k]).pin_memory() for k in _kinds(wl)],
+                    dev_pools=[t[k] for k in _kinds(wl)],
+                    first_window_chunk=host["first_window_chunk"], first_free_slot=host["first_free_slot"],
+                    table_host=torch.from_numpy(host["chunk_table"][0].copy()).pin_memory())
+    shapes = dict(B=wl.B, Hn=wl.Hn, dn=wl.dn, Hl=wl.Hl, dl=wl.dl, k=wl.k, Hq=wl.Hq, dqk=wl.dqk, dv=wl.dv,
+                  latent=wl.latent, window=wl.window, steps=host["steps"], scale=wl.scale)
+    return shapes, t, host["max_chunks"], host["kept_cap"], cold

@@ -1,0 +1,99 @@
+"""The C-ABI library builds, loads and exports every entry point declared in include/lsa.h,
+and its host-side argument checks reject bad calls before any launch (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from learned_sparse_kv_b200 import build as lbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lsa.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lsa_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return ctypes.CDLL(lbuild.build())
+
+
+def test_header_declares_the_boundary():
+    names = declared_symbols()
+    for required in ("lsa_nmi_select", "lsa_topk", "lsa_topk_from_scores", "lsa_sparse_decode",
+                     "lsa_append_token", "lsa_gather_chunks", "lsa_label_vote", "lsa_last_error"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [n for n in declared_symbols() if not hasattr(lib, n)]
+    assert not missing, f"not exported: {missing}"
+
+
+def test_build_targets_sm100a_only():
+    assert lbuild.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def _err(lib):
+    lib.lsa_last_error.restype = ctypes.c_char_p
+    return lib.lsa_last_error().decode()
+
+
+def test_gather_rejects_unsorted_kept_list(lib):
+    kept = (ctypes.c_int32 * 3)(5, 2, 9)
+    table = (ctypes.c_int32 * 20)()
+    hp = (ctypes.c_void_p * 1)(ctypes.addressof(table))
+    dp = (ctypes.c_void_p * 1)(ctypes.addressof(table))
+    cb = (ctypes.c_size_t * 1)(64)
+    rc = lib.lsa_gather_chunks(1, hp, cb, dp, ctypes.c_int64(20), ctypes.c_int64(20), kept, 3, 15, 0,
+                               table, table, 20, None, None, None)
+    assert rc == 1 and "ascending" in _err(lib)
+
+
+def test_gather_reports_slot_capacity(lib):
+    kept = (ctypes.c_int32 * 4)(1, 2, 3, 4)
+    table = (ctypes.c_int32 * 20)()
+    hp = (ctypes.c_void_p * 1)(ctypes.addressof(table))
+    cb = (ctypes.c_size_t * 1)(64)
+    rc = lib.lsa_gather_chunks(1, hp, cb, hp, ctypes.c_int64(20), ctypes.c_int64(5), kept, 4, 15, 2,
+                               table, table, 20, None, None, None)
+    assert rc == 4 and "fit" in _err(lib)
+
+
+def test_gather_rejects_chunk_outside_host_pool(lib):
+    kept = (ctypes.c_int32 * 2)(1, 30)
+    table = (ctypes.c_int32 * 40)()
+    hp = (ctypes.c_void_p * 1)(ctypes.addressof(table))
+    cb = (ctypes.c_size_t * 1)(64)
+    rc = lib.lsa_gather_chunks(1, hp, cb, hp, ctypes.c_int64(20), ctypes.c_int64(100), kept, 2, 35, 0,
+                               table, table, 40, None, None, None)
+    assert rc == 6
+
+
+def test_entry_points_reject_bad_shapes_before_launch(lib):
+    P = ctypes.c_void_p(16)  # never dereferenced: the calls fail validation first
+    f = lib.lsa_sparse_decode
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                  ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    rc = f(P, P, 576, None, 0, 10, P, 4, P, P, 16, P, P, 100, 1, 96, 576, 512, 0.04, P, None, None, P, 1 << 20, None)
+    assert rc == 2 and "unsupported" in _err(lib)
+    rc = lib.lsa_label_vote(P, 65, 4, 128, ctypes.c_float(0.6), 3, 0, P, None, P, ctypes.c_size_t(1 << 20), None)
+    assert rc == 2
+    rc = lib.lsa_label_vote(P, 4, 4, 128, ctypes.c_float(0.6), 3, 2, P, None, P, ctypes.c_size_t(1 << 20), None)
+    assert rc == 1
+
+
+def test_workspace_queries_are_host_only(lib):
+    lib.lsa_label_vote_workspace_size.restype = ctypes.c_size_t
+    lib.lsa_topk_workspace_size.restype = ctypes.c_size_t
+    lib.lsa_nmi_select_workspace_size.restype = ctypes.c_size_t
+    assert lib.lsa_label_vote_workspace_size(32, 64, 2048) == 64 * 2048 * 4
+    assert lib.lsa_topk_workspace_size(8, 2048) == 8 * 2048 * 64 * 4
+    assert lib.lsa_nmi_select_workspace_size(8, 2048) >= 8 * 32 * 8

@@ -1,0 +1,308 @@
+"""GPU parity of each entry point against the oracle (run on a B200 with -m gpu).
+
+Lists (kept chunks, top-k positions, vote labels) must match bit for bit;
+attention must satisfy |err| <= 2e-3 + 1e-2 |ref| element by element.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import lsa_workloads as W
+from lsa_workloads.device import bf16, host_build, i32
+from tests import helpers as H
+
+pytestmark = pytest.mark.gpu
+CH = W.CHUNK
+
+
+@pytest.fixture(scope="module")
+def L():
+    from learned_sparse_kv_b200 import lsa
+    return lsa
+
+
+def dev():
+    return torch.device("cuda:0")
+
+
+# ----------------------------------------------------------- a3 from scores --
+
+@pytest.mark.parametrize("k", [1, 17, 512, 2048])
+def test_topk_from_scores_exact(L, k):
+    rng = np.random.default_rng(k)
+    sizes = [0, 1, 300, 5000, 70000, k, k + 1]
+    segs = []
+    for i, n in enumerate(sizes):
+        s = rng.standard_normal(n).astype(np.float32)
+        if i % 2:
+            s = np.round(s * 4) / 4          # exact ties
+        segs.append(s)
+    off = np.zeros(len(segs) + 1, np.int64)
+    off[1:] = np.cumsum([s.size for s in segs])
+    flat = np.concatenate(segs)
+    idx, cnt = L.topk_from_scores(torch.from_numpy(flat).to(dev()), torch.from_numpy(off).to(dev()),
+                                  max(sizes), k)
+    idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    for b, s in enumerate(segs):
+        ref = oracle.topk_select_f32(s, k)
+        assert cnt[b] == ref.size
+        np.testing.assert_array_equal(idx[b, :ref.size], ref)
+        assert np.all(idx[b, ref.size:] == -1)
+
+
+def test_topk_from_scores_all_tied_and_signed_zero(L):
+    s = np.full(10000, 0.5, np.float32)
+    s[::3] = -0.0
+    s[1::3] = 0.0
+    off = torch.tensor([0, 10000], dtype=torch.int64, device=dev())
+    for k in (1, 999, 5000):
+        idx, cnt = L.topk_from_scores(torch.from_numpy(s).to(dev()), off, 10000, k)
+        np.testing.assert_array_equal(idx.cpu().numpy()[0, :cnt.item()], oracle.topk_select_f32(s, k))
+
+
+# ------------------------------------------------------------------- a1 ---
+
+def _nmi_gpu(L, nm, kept_cap, max_chunks):
+    d = dev()
+    status = torch.zeros(1, dtype=torch.int32, device=d)
+    logits = torch.empty(nm["khat"].shape[0], dtype=torch.float32, device=d)
+    kept, cnt = L.nmi_select(bf16(nm["q"], d), bf16(nm["w"], d), bf16(nm["khat"], d),
+                             torch.from_numpy(nm["seq_chunk_offset"]).to(d), max_chunks, kept_cap,
+                             logits=logits, status=status)
+    return kept.cpu().numpy(), cnt.cpu().numpy(), logits.cpu().numpy(), int(status.item())
+
+
+@pytest.mark.parametrize("name", ["decode_16k_b1_h16", "decode_128k_b8_mla", "decode_512k_b1_mla_cold",
+                                  "decode_ragged_b32_mla"])
+def test_nmi_select_planted_exact(L, name):
+    wl = W.workload(name)
+    nm = W.nmi_inputs(wl)
+    cap = max(wl.n_ch)
+    kept, cnt, logits, st = _nmi_gpu(L, nm, cap, max(wl.n_ch))
+    ref, ref_logits, _, rc, rcnt = oracle.nmi_select(nm["q"], nm["w"], nm["khat"], nm["seq_chunk_offset"], cap)
+    assert st == 0 and rc == 0
+    for b in range(wl.B):
+        np.testing.assert_array_equal(kept[b, :cnt[b]], ref[b])
+        np.testing.assert_array_equal(kept[b, :cnt[b]], nm["planted"][b])
+        assert np.all(kept[b, cnt[b]:] == -1)
+    np.testing.assert_allclose(logits, ref_logits, rtol=1e-4, atol=1e-3)
+
+
+@pytest.mark.parametrize("Hn,dn,n_ch", [(8, 64, (300, 1, 64, 65)), (64, 128, (2048, 777)), (24, 128, (129,))])
+def test_nmi_select_random_inputs_exact(L, Hn, dn, n_ch):
+    wl = W.workload("decode_128k_b8_mla", B=len(n_ch), ctx=tuple(c * CH for c in n_ch), Hn=Hn, dn=dn,
+                    pass_rate=(0.5,) * len(n_ch))
+    nm = W.nmi_inputs(wl, structural=False)
+    host = dict(nmi=nm, kept_cap=max(n_ch))
+    H.repair_nmi_margin(host)
+    kept, cnt, logits, st = _nmi_gpu(L, nm, max(n_ch), max(n_ch))
+    ref, ref_logits, _, _, _ = oracle.nmi_select(nm["q"], nm["w"], nm["khat"], nm["seq_chunk_offset"], max(n_ch))
+    for b in range(wl.B):
+        np.testing.assert_array_equal(kept[b, :cnt[b]], ref[b])
+    np.testing.assert_allclose(logits, ref_logits, rtol=1e-4, atol=1e-3)
+
+
+def test_nmi_select_capacity_overflow_truncates_and_flags(L):
+    wl = W.workload("decode_16k_b1_h16")
+    nm = W.nmi_inputs(wl)
+    kept, cnt, _, st = _nmi_gpu(L, nm, 10, wl.n_ch[0])
+    assert st & L.DEV_CAPACITY and cnt[0] == 10
+    np.testing.assert_array_equal(kept[0], nm["planted"][0][:10])
+
+
+# -------------------------------------------------------------- a2 + a3 ---
+
+def _small_mla(**kw):
+    base = dict(B=2, ctx=(96 * CH, 40 * CH), window=16 * CH, pass_rate=(0.3, 0.5), steps=3, seed=77)
+    base.update(kw)
+    return W.workload("decode_128k_b8_mla", **base)
+
+
+@pytest.mark.parametrize("k", [64, 700, 60000])
+def test_li_topk_exact(L, k):
+    wl = _small_mla(k=k)
+    host = host_build(wl)
+    kept, _, _, _ = H.kept_lists(host)
+    pairs = [(b, s) for b in range(wl.B) for s in range(wl.steps)]
+    H.open_topk_gap(host, kept, pairs)
+    d = dev()
+    kept_t = torch.full((wl.B, host["kept_cap"]), -1, dtype=torch.int32)
+    cnt_t = torch.zeros(wl.B, dtype=torch.int32)
+    for b in range(wl.B):
+        kept_t[b, :kept[b].size] = torch.from_numpy(kept[b])
+        cnt_t[b] = kept[b].size
+    li = bf16(host["pools"]["li"], d)
+    table = i32(host["chunk_table"], d)
+    ws = i32(host["window_start"], d)
+    scores = torch.empty(wl.B, host["kept_cap"] * CH, dtype=torch.float32, device=d)
+    for s in range(wl.steps):
+        st = host["step"]
+        status = torch.zeros(1, dtype=torch.int32, device=d)
+        idx, cnt = L.topk(bf16(st["q_li"][s], d), bf16(st["w_li"][s], d), li, table, kept_t.to(d), cnt_t.to(d),
+                          ws, k, scores=scores, status=status)
+        idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+        assert status.item() == 0
+        for b in range(wl.B):
+            pos, ref_sc = H.li_scores(host, kept[b], b, s)
+            sel = oracle.topk_select(ref_sc, k)
+            assert cnt[b] == sel.size
+            np.testing.assert_array_equal(idx[b, :cnt[b]], pos[sel])
+            assert np.all(idx[b, cnt[b]:] == -1)
+            np.testing.assert_allclose(scores[b, :pos.size].cpu().numpy(), ref_sc, rtol=1e-4, atol=1e-3)
+
+
+def test_li_topk_no_cold_candidates(L):
+    wl = _small_mla(k=32)
+    host = host_build(wl)
+    d = dev()
+    kept_t = torch.full((wl.B, host["kept_cap"]), -1, dtype=torch.int32, device=d)
+    kept_t[:, 0] = torch.tensor([wl.n_ch[0] - 1, wl.n_ch[1] - 2], dtype=torch.int32)   # window chunks only
+    cnt_t = torch.tensor([1, 1], dtype=torch.int32, device=d)
+    st = host["step"]
+    idx, cnt = L.topk(bf16(st["q_li"][0], d), bf16(st["w_li"][0], d), bf16(host["pools"]["li"], d),
+                      i32(host["chunk_table"], d), kept_t, cnt_t, i32(host["window_start"], d), 32)
+    assert cnt.cpu().tolist() == [0, 0] and bool((idx == -1).all())
+
+
+# ------------------------------------------------------------------- a4 ---
+
+def _decode_case(L, wl, kept, host, s, topk_override=None, table_override=None):
+    d = dev()
+    st = host["step"]
+    B = wl.B
+    tk = np.full((B, wl.k), -1, np.int32)
+    tc = np.zeros(B, np.int32)
+    refs = []
+    for b in range(B):
+        r = H.oracle_step(host, kept[b], b, s)
+        refs.append(r)
+        sel = r["topk"][:r["topk_count"]] if topk_override is None else topk_override[b]
+        tk[b, :len(sel)] = sel
+        tc[b] = len(sel)
+    pools = host["pools"]
+    table = host["chunk_table"] if table_override is None else table_override
+    wlen = np.full(B, wl.window + s + 1, np.int32)
+    status = torch.zeros(1, dtype=torch.int32, device=d)
+    out, lse = L.sparse_decode(bf16(st["q"][s], d), bf16(pools["kv"] if wl.latent else pools["k"], d),
+                               None if wl.latent else bf16(pools["v"], d), i32(table, d), i32(tk, d), i32(tc, d),
+                               i32(host["window_start"], d), i32(wlen, d), wl.window + wl.steps, wl.dv, wl.scale,
+                               status=status)
+    return out.cpu().numpy(), lse.cpu().numpy(), refs, int(status.item())
+
+
+@pytest.mark.parametrize("shape", ["mla128", "mla64", "sep16"])
+@pytest.mark.parametrize("q_scale", [1.0, 4.0])
+def test_sparse_decode_matches_oracle(L, shape, q_scale):
+    if shape == "sep16":
+        wl = W.workload("decode_16k_b1_h16", B=2, ctx=(80 * CH, 33 * CH), window=20 * CH, steps=2,
+                        pass_rate=(0.3, 0.4), q_scale=q_scale, k=300)
+    else:
+        wl = _small_mla(q_scale=q_scale, k=500, Hq=128 if shape == "mla128" else 64)
+    host = host_build(wl)
+    kept, _, _, _ = H.kept_lists(host)
+    for s in range(wl.steps):
+        out, lse, refs, st = _decode_case(L, wl, kept, host, s)
+        assert st == 0
+        for b in range(wl.B):
+            H.assert_close_attention(out[b], refs[b]["out"])
+            np.testing.assert_allclose(lse[b], refs[b]["lse"], rtol=1e-5, atol=2e-4)
+
+
+def test_sparse_decode_window_only(L):
+    wl = _small_mla(k=64, window=CH, steps=1)
+    host = host_build(wl)
+    kept = [np.zeros(0, np.int32)] * wl.B
+    out, lse, refs, st = _decode_case(L, wl, kept, host, 0)
+    for b in range(wl.B):
+        H.assert_close_attention(out[b], refs[b]["out"])
+
+
+def test_sparse_decode_skips_rows_without_slot_and_flags(L):
+    wl = _small_mla(k=200, steps=1)
+    host = host_build(wl)
+    kept, _, _, _ = H.kept_lists(host)
+    sel = [H.oracle_step(host, kept[b], b, 0) for b in range(wl.B)]
+    sel = [r["topk"][:r["topk_count"]] for r in sel]
+    gone = int(sel[0][0]) // CH                       # this chunk loses its slot
+    table = host["chunk_table"].copy()
+    table[0, gone] = -1
+    out, _, _, st = _decode_case(L, wl, kept, host, 0, topk_override=sel, table_override=table)
+    assert st & L.DEV_TABLE
+    # reference: the same rows minus those of the chunk without a slot
+    rows = np.array([p for p in sel[0] if p // CH != gone], np.int64)
+    w0 = int(host["window_start"][0])
+    pos = np.concatenate([rows, np.arange(w0, w0 + wl.window + 1)])
+    krow = host["oracle_pools"]["kv"][host["oracle_table"][0][pos // CH], pos % CH]
+    ref, _ = oracle.attention_dense(host["step"]["q"][0, 0], krow, np.ascontiguousarray(krow[:, :wl.dv]), wl.scale)
+    H.assert_close_attention(out[0], ref)
+
+
+# ------------------------------------------------------------------- a7 ---
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_label_vote_full_window_exact(L, mode):
+    p = W.LABEL_VOTE
+    d = W.label_vote_scores(p["layers"], p["steps"], p["chunks"], p["planted"], p["seed"])
+    H.repair_vote_margin(d, p["top_p"])
+    labels, votes = L.label_vote(torch.from_numpy(d["scores"]).to(dev()), p["top_p"], p["min_layers"], mode)
+    ref_labels, ref_votes = oracle.label_vote(d["scores"], p["top_p"], p["min_layers"], mode)
+    np.testing.assert_array_equal(votes.cpu().numpy(), ref_votes)
+    np.testing.assert_array_equal(labels.cpu().numpy(), ref_labels)
+    assert 0 < ref_labels.sum() < p["chunks"]
+
+
+def test_label_vote_ragged_chunk_count(L):
+    d = W.label_vote_scores(5, 7, 777, 40, seed=31)
+    H.repair_vote_margin(d, 0.6)
+    labels, votes = L.label_vote(torch.from_numpy(d["scores"]).to(dev()), 0.6, 3, 0)
+    ref_labels, ref_votes = oracle.label_vote(d["scores"], 0.6, 3, 0)
+    np.testing.assert_array_equal(votes.cpu().numpy(), ref_votes)
+    np.testing.assert_array_equal(labels.cpu().numpy(), ref_labels)
+
+
+# ---------------------------------------------------------------- a5, a6 --
+
+def test_append_writes_rows_and_advances_window(L):
+    d = dev()
+    B, slots, kw, dl = 3, 12, 576, 128
+    kv = torch.zeros(slots, CH, kw, dtype=torch.bfloat16, device=d)
+    li = torch.zeros(slots, CH, dl, dtype=torch.bfloat16, device=d)
+    table = torch.tensor([[0, 1, 2, 3], [4, 5, 6, 7], [8, 9, 10, 11]], dtype=torch.int32, device=d)
+    wstart = torch.tensor([64, 0, 128], dtype=torch.int32, device=d)
+    wlen = torch.tensor([63, 64, 5], dtype=torch.int32, device=d)
+    nk = torch.randn(B, kw, device=d).to(torch.bfloat16)
+    nl = torch.randn(B, dl, device=d).to(torch.bfloat16)
+    L.append_token(nk, None, nl, kv, None, li, table, wstart, wlen)
+    torch.cuda.synchronize()
+    assert wlen.cpu().tolist() == [64, 65, 6]
+    for b, pos in enumerate([127, 64, 133]):
+        slot = int(table[b, pos // CH])
+        assert torch.equal(kv[slot, pos % CH], nk[b]) and torch.equal(li[slot, pos % CH], nl[b])
+
+
+def test_gather_copies_kept_cold_chunks(L):
+    d = dev()
+    rng = np.random.default_rng(5)
+    n_ch, fw, width = 40, 30, 576
+    host_kv = torch.from_numpy(rng.integers(0, 2 ** 16, (n_ch, CH, width), dtype=np.uint16).view(np.int16)).pin_memory()
+    host_li = torch.from_numpy(rng.integers(0, 2 ** 16, (n_ch, CH, 128), dtype=np.uint16).view(np.int16)).pin_memory()
+    dev_kv = torch.zeros(20, CH, width, dtype=torch.int16, device=d)
+    dev_li = torch.zeros(20, CH, 128, dtype=torch.int16, device=d)
+    kept = torch.tensor([0, 1, 2, 7, 9, 10, 29, 31, 35], dtype=torch.int32)
+    table_host = torch.full((n_ch + 1,), 99, dtype=torch.int32).pin_memory()
+    table_host[fw:] = torch.arange(n_ch + 1 - fw, dtype=torch.int32)
+    table_dev = torch.zeros(n_ch + 1, dtype=torch.int32, device=d)
+    side = torch.cuda.Stream()
+    done = torch.cuda.Event()
+    n = L.gather_chunks([host_kv, host_li], [dev_kv, dev_li], kept, fw, 11, table_host, table_dev,
+                        stream=side, done=done)
+    done.synchronize()
+    assert n == 7
+    tab = table_dev.cpu().numpy()
+    expect = {0: 11, 1: 12, 2: 13, 7: 14, 9: 15, 10: 16, 29: 17}
+    for c in range(fw):
+        assert tab[c] == expect.get(c, -1)
+    for c, sl in expect.items():
+        assert torch.equal(dev_kv[sl].cpu(), host_kv[c]) and torch.equal(dev_li[sl].cpu(), host_li[c])
+    np.testing.assert_array_equal(tab[fw:], np.arange(n_ch + 1 - fw))

@@ -1,0 +1,141 @@
+"""End-to-end parity of whole lookahead windows on the GPU (run with -m gpu).
+
+Each workload runs select + 64 x (append, top-k, attention) through
+learned_sparse_kv_b200.decode.Window, in the launch configuration the
+benchmark times (CUDA graph).  The oracle recomputes sampled (sequence, step)
+pairs from the same inputs; every step is also checked for properties that
+hold at any size (counts, ascending positions, candidates only).
+"""
+import numpy as np
+import pytest
+import torch
+
+import lsa_workloads as W
+from lsa_workloads.device import host_build, upload
+from tests import helpers as H
+
+pytestmark = pytest.mark.gpu
+CH = W.CHUNK
+
+
+def _window(host, graph=True):
+    from learned_sparse_kv_b200.decode import Shapes, Window
+    shapes, t, max_ch, kept_cap, cold = upload(host, torch.device("cuda:0"))
+    win = Window(Shapes(**shapes), t, max_ch, kept_cap, cold)
+    if graph:
+        win.capture()
+    win.run(use_graph=graph)
+    torch.cuda.synchronize()
+    return win
+
+
+def _check_window(host, win, pairs):
+    wl = host["wl"]
+    kept, _, _, _ = H.kept_lists(host)
+    assert win.device_status() == 0
+    gk, gc = win.kept_idx.cpu().numpy(), win.kept_count.cpu().numpy()
+    for b in range(wl.B):
+        np.testing.assert_array_equal(gk[b, :gc[b]], kept[b])
+    tk, tc = win.topk_idx.cpu().numpy(), win.topk_count.cpu().numpy()
+    out = win.out.cpu().numpy()
+    # properties at every step
+    for b in range(wl.B):
+        fw = int(host["window_start"][b]) // CH
+        cold_chunks = set(int(c) for c in kept[b] if c < fw)
+        n_cand = CH * len(cold_chunks)
+        for s in range(wl.steps):
+            c = int(tc[s, b])
+            assert c == min(wl.k, n_cand)
+            sel = tk[s, b, :c]
+            assert np.all(np.diff(sel) > 0) and np.all(tk[s, b, c:] == -1)
+            assert all((int(p) // CH) in cold_chunks for p in sel[:64])
+    assert np.isfinite(out).all()
+    stats = []
+    for b, s in pairs:
+        ref = H.oracle_step(host, kept[b], b, s)
+        np.testing.assert_array_equal(tk[s, b, :tc[s, b]], ref["topk"][:ref["topk_count"]])
+        stats.append(H.assert_close_attention(out[s, b], ref["out"]))
+        np.testing.assert_allclose(win.lse[s, b].cpu().numpy(), ref["lse"], rtol=1e-5, atol=2e-4)
+    return stats
+
+
+def test_window_16k_all_steps():
+    wl = W.workload("decode_16k_b1_h16")
+    host = host_build(wl)
+    kept, _, _, _ = H.kept_lists(host)
+    pairs = [(0, s) for s in range(wl.steps)]
+    H.open_topk_gap(host, kept, pairs)
+    win = _window(host)
+    _check_window(host, win, pairs)
+
+
+def test_window_16k_peaked_attention():
+    wl = W.workload("decode_16k_b1_h16", q_scale=4.0, steps=8)
+    host = host_build(wl)
+    kept, _, _, _ = H.kept_lists(host)
+    pairs = [(0, s) for s in range(wl.steps)]
+    H.open_topk_gap(host, kept, pairs)
+    win = _window(host)
+    stats = _check_window(host, win, pairs)
+    assert max(r for _, r in stats) < 5e-3
+
+
+def test_window_128k_b8():
+    wl = W.workload("decode_128k_b8_mla")
+    host = host_build(wl)
+    kept, _, _, _ = H.kept_lists(host)
+    pairs = [(0, 0), (3, 31), (7, 63)]
+    H.open_topk_gap(host, kept, pairs)
+    win = _window(host)
+    _check_window(host, win, pairs)
+
+
+def test_window_ragged_b32():
+    wl = W.workload("decode_ragged_b32_mla")
+    host = host_build(wl)
+    kept, _, _, _ = H.kept_lists(host)
+    order = np.argsort(wl.ctx)
+    pairs = [(int(order[0]), 0), (int(order[-1]), 63), (int(order[len(order) // 2]), 17)]
+    H.open_topk_gap(host, kept, pairs)
+    win = _window(host)
+    _check_window(host, win, pairs)
+
+
+def test_window_512k_cold_pool():
+    wl = W.workload("decode_512k_b1_mla_cold")
+    host = host_build(wl)
+    kept, _, _, _ = H.kept_lists(host)
+    pairs = [(0, 0), (0, 63)]
+    H.open_topk_gap(host, kept, pairs)
+    win = _window(host)
+    n_cold = sum(1 for c in kept[0] if c < host["first_window_chunk"])
+    assert win.n_fetched == n_cold
+    # fetched slots hold the host pool's bytes
+    table = win.t["chunk_table"][0].cpu().numpy()
+    kv = win.t["kv"]
+    for c in [int(x) for x in kept[0][:5]] + [int(kept[0][n_cold - 1])]:
+        slot = int(table[c])
+        assert torch.equal(kv[slot].cpu().view(torch.int16), torch.from_numpy(host["cold_pools"]["kv"][c].view(np.int16)))
+    _check_window(host, win, pairs)
+
+
+def test_window_context_is_window_plus_one_chunk():
+    wl = W.workload("decode_128k_b8_mla", B=2, ctx=(8064, 8128), pass_rate=(1.0, 0.5), steps=4)
+    host = host_build(wl)
+    kept, _, _, _ = H.kept_lists(host)
+    pairs = [(b, s) for b in range(2) for s in range(4)]
+    H.open_topk_gap(host, kept, pairs)
+    win = _window(host)
+    _check_window(host, win, pairs)
+
+
+def test_window_is_deterministic_and_graph_matches_eager():
+    wl = W.workload("decode_128k_b8_mla", B=3, ctx=(32768, 20480, 65536), pass_rate=(0.2, 0.1, 0.15), steps=6)
+    host = host_build(wl)
+    a = _window(host, graph=True)
+    out_a, tk_a = a.out.clone(), a.topk_idx.clone()
+    a.run(use_graph=True)
+    torch.cuda.synchronize()
+    assert torch.equal(out_a, a.out) and torch.equal(tk_a, a.topk_idx)
+    b = _window(host, graph=False)
+    assert torch.equal(out_a, b.out) and torch.equal(tk_a, b.topk_idx)
