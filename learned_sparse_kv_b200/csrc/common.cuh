@@ -67,9 +67,11 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-// Order-preserving map from fp32 to uint32: a < b  <=>  key(a) < key(b).
+// Order-preserving map from fp32 to uint32: a < b  <=>  key(a) < key(b), and
+// a == b  <=>  key(a) == key(b) (-0.0 and +0.0 are the same score).
 __device__ __forceinline__ uint32_t ordered_key(float f) {
     uint32_t u = __float_as_uint(f);
+    if ((u << 1) == 0u) u = 0u;
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 

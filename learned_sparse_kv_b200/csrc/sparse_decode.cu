@@ -305,11 +305,22 @@ __global__ void lse_merge_kernel(const float *__restrict__ o_part, const float *
 using CfgSep16 = DecodeCfg<16, 128, 128, 4, false>;
 using CfgMla64 = DecodeCfg<64, 576, 512, 8, true>;
 
-enum class Variant { None, Sep16, Mla64 };
+namespace mla2 {
+int launch(const uint16_t *q, const uint16_t *kv_pool, int64_t k_stride, int64_t n_slots, const int32_t *table,
+           int table_stride, const int32_t *topk_idx, const int32_t *topk_count, int k, const int32_t *window_start,
+           const int32_t *window_len, int B, float scale, int n_splits, float *o_part, float *m_part, float *l_part,
+           int32_t *status, cudaStream_t stream);
+int max_splits(int B);
+}  // namespace mla2
+
+// Sep16: 16 heads, separate K/V rows of 128 (mma.sync).  Mla64: 64 latent heads
+// (mma.sync).  Mla128: 128 latent heads on tcgen05 with a CTA pair per split.
+enum class Variant { None, Sep16, Mla64, Mla128 };
 
 static Variant pick(int Hq, int dqk, int dv, bool latent) {
     if (!latent && Hq == 16 && dqk == 128 && dv == 128) return Variant::Sep16;
-    if (latent && (Hq == 64 || Hq == 128) && dqk == 576 && dv == 512) return Variant::Mla64;
+    if (latent && Hq == 128 && dqk == 576 && dv == 512) return Variant::Mla128;
+    if (latent && Hq == 64 && dqk == 576 && dv == 512) return Variant::Mla64;
     return Variant::None;
 }
 
@@ -337,6 +348,10 @@ static int choose_splits(int B, int Hq, int k, int max_window_len) {
 }
 
 static int splits_for(Variant v, int B, int Hq, int k, int max_window_len) {
+    if (v == Variant::Mla128) {
+        const int tiles_max = (k + 63) / 64 + (max_window_len + 63) / 64;
+        return max(1, min(mla2::max_splits(B), tiles_max));
+    }
     return v == Variant::Sep16 ? choose_splits<CfgSep16>(B, Hq, k, max_window_len)
                                : choose_splits<CfgMla64>(B, Hq, k, max_window_len);
 }
@@ -399,7 +414,10 @@ extern "C" int lsa_sparse_decode(const lsa_bf16 *q, const lsa_bf16 *k_pool, int6
     float *o_part = c.take<float>((size_t)B * ns * Hq * dv);
     float *m_part = c.take<float>((size_t)B * ns * Hq);
     float *l_part = c.take<float>((size_t)B * ns * Hq);
-    int rc = v == Variant::Sep16
+    int rc = v == Variant::Mla128
+                 ? mla2::launch(q, k_pool, k_row_stride, n_slots, chunk_table, table_stride, topk_idx, topk_count, k,
+                                window_start, window_len, B, scale, ns, o_part, m_part, l_part, dev_status, stream)
+             : v == Variant::Sep16
                  ? launch<CfgSep16>(q, k_pool, k_row_stride, v_pool, v_row_stride, n_slots, chunk_table, table_stride,
                                     topk_idx, topk_count, k, window_start, window_len, B, Hq, scale, ns, o_part, m_part,
                                     l_part, dev_status, stream)

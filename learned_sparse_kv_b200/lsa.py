@@ -216,6 +216,10 @@ def gather_chunks(host_pools, dev_pools, kept_idx_host, first_window_chunk, firs
     CB = (ctypes.c_size_t * n)(*[t[0].numel() * t.element_size() for t in host_pools])
     kept = kept_idx_host.to(torch.int32).contiguous()
     nf = ctypes.c_int(0)
+    st = stream if stream is not None else torch.cuda.current_stream()
+    if done is not None and done.cuda_event == 0:
+        done.record(st)          # torch creates the CUDA event on first record
+
     _check(_lib.lsa_gather_chunks(n, HP, CB, DP, host_pools[0].shape[0], dev_pools[0].shape[0], _ptr(kept),
                                   kept.numel(), first_window_chunk, first_free_slot, _ptr(chunk_table_host),
                                   _ptr(chunk_table_dev), chunk_table_host.numel(), _stream(stream),

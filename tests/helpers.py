@@ -56,9 +56,12 @@ def li_scores(host, kept, b, s):
     return pos, oracle.li_scores(st["q_li"][s, b], st["w_li"][s, b], keys)
 
 
-def open_topk_gap(host, kept_lists_, pairs, rel=1e-3, seed=7, max_iter=200):
+def open_topk_gap(host, kept_lists_, pairs, rel=2e-5, seed=7, max_iter=200):
     """Redraws indexer keys until, for every (b, s) in pairs, the k-th and (k+1)-th
-    largest candidate scores differ by at least rel * max(1, |s_k|)."""
+    largest candidate scores differ by at least rel * max(1, |s_k|).
+
+    The GPU scores in fp32 with tensor-core accumulation; its error is about
+    1e-6 relative, so a 2e-5 relative gap leaves a 20x margin."""
     wl = host["wl"]
     rng = np.random.default_rng(seed)
     for _ in range(max_iter):
