@@ -38,14 +38,24 @@ __device__ __forceinline__ int cold_kept_count(const int32_t *kept, int count, i
     return lo;
 }
 
+// Adds 1 to hist[bin] for every lane with `active`, one shared atomic per distinct bin.
+__device__ __forceinline__ void warp_hist_add(int *hist, uint32_t bin, bool active) {
+    const unsigned act = __ballot_sync(0xffffffffu, active);
+    if (!active) return;
+    const unsigned same = __match_any_sync(act, bin);
+    if ((threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(&hist[bin], __popc(same));
+}
+
+// Scores of one sequence: from shared memory when they were staged there, else global.
 template <class PosFn>
-__device__ void topk_block(const float *__restrict__ s, int n, int k, PosFn pos, int32_t *__restrict__ out,
-                           int32_t *__restrict__ out_count) {
+__device__ void topk_block(const float *__restrict__ s_glob, const float *s, int n, int k, PosFn pos,
+                           int32_t *__restrict__ out, int32_t *__restrict__ out_count) {
     __shared__ int hist[256];
     __shared__ int warp_tot[kTopkThreads / 32 + 1];
     __shared__ uint32_t sh_prefix;
     __shared__ int sh_remaining;
     const int t = threadIdx.x;
+    (void)s_glob;
 
     if (n <= k) {  // everything is selected, already in ascending order
         for (int j = t; j < k; j += kTopkThreads) out[j] = j < n ? pos(j) : -1;
@@ -55,13 +65,14 @@ __device__ void topk_block(const float *__restrict__ s, int n, int k, PosFn pos,
 
     uint32_t prefix = 0, pmask = 0;
     int remaining = k;
+    const int n_round = (n + kTopkThreads - 1) / kTopkThreads * kTopkThreads;   // warp-uniform trip count
 #pragma unroll 1
     for (int shift = 24; shift >= 0; shift -= 8) {
         if (t < 256) hist[t] = 0;
         __syncthreads();
-        for (int j = t; j < n; j += kTopkThreads) {
-            uint32_t u = ordered_key(s[j]);
-            if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255], 1);
+        for (int j = t; j < n_round; j += kTopkThreads) {
+            const uint32_t u = j < n ? ordered_key(s[j]) : 0u;
+            warp_hist_add(hist, (u >> shift) & 255u, j < n && (u & pmask) == prefix);
         }
         __syncthreads();
         // suffix counts over digits, highest digit first
@@ -106,29 +117,46 @@ __device__ void topk_block(const float *__restrict__ s, int n, int k, PosFn pos,
     if (t == 0) *out_count = k;
 }
 
+// Copies n scores into dynamic shared memory when they fit; returns the array to read.
+__device__ __forceinline__ const float *stage_scores(const float *__restrict__ g, int n, int cap) {
+    extern __shared__ float stage[];
+    if (n > cap) return g;
+    const int n4 = (reinterpret_cast<uintptr_t>(g) & 15) == 0 ? n / 4 : 0;
+    for (int i = threadIdx.x; i < n4; i += kTopkThreads)
+        reinterpret_cast<float4 *>(stage)[i] = reinterpret_cast<const float4 *>(g)[i];
+    for (int i = 4 * n4 + threadIdx.x; i < n; i += kTopkThreads) stage[i] = g[i];
+    __syncthreads();
+    return stage;
+}
+
 __global__ void __launch_bounds__(kTopkThreads) topk_kept_kernel(const float *__restrict__ scores, int kept_cap,
                                                                  const int32_t *__restrict__ kept_idx,
                                                                  const int32_t *__restrict__ kept_count,
                                                                  const int32_t *__restrict__ window_start, int k,
                                                                  int32_t *__restrict__ topk_idx,
-                                                                 int32_t *__restrict__ topk_count) {
+                                                                 int32_t *__restrict__ topk_count, int stage_cap) {
     const int b = blockIdx.x;
     const int32_t *kept = kept_idx + (size_t)b * kept_cap;
     const int cnt = min(kept_count[b], kept_cap);
     const int n = cold_kept_count(kept, cnt, window_start[b] / LSA_CHUNK) * LSA_CHUNK;
-    topk_block(scores + (size_t)b * kept_cap * LSA_CHUNK, n, k, CandFromKept{kept}, topk_idx + (size_t)b * k,
-               topk_count + b);
+    const float *g = scores + (size_t)b * kept_cap * LSA_CHUNK;
+    const float *s = n > k ? stage_scores(g, n, stage_cap) : g;
+    topk_block(g, s, n, k, CandFromKept{kept}, topk_idx + (size_t)b * k, topk_count + b);
 }
 
 __global__ void __launch_bounds__(kTopkThreads) topk_scores_kernel(const float *__restrict__ scores,
                                                                    const int64_t *__restrict__ off, int max_cand,
                                                                    int k, int32_t *__restrict__ topk_idx,
-                                                                   int32_t *__restrict__ topk_count) {
+                                                                   int32_t *__restrict__ topk_count, int stage_cap) {
     const int b = blockIdx.x;
     const int64_t a = off[b];
     const int n = (int)max((int64_t)0, min(off[b + 1] - a, (int64_t)max_cand));
-    topk_block(scores + a, n, k, CandIdentity{}, topk_idx + (size_t)b * k, topk_count + b);
+    const float *s = n > k ? stage_scores(scores + a, n, stage_cap) : scores + a;
+    topk_block(scores + a, s, n, k, CandIdentity{}, topk_idx + (size_t)b * k, topk_count + b);
 }
+
+// Scores staged in shared memory: up to 200 KB (51,200 candidates), never more than needed.
+static int stage_capacity(int max_n) { return max(0, min(max_n, 51200)); }
 
 }  // namespace lsa
 
@@ -163,8 +191,11 @@ extern "C" int lsa_topk(const lsa_bf16 *q_li, const lsa_bf16 *w_li, const lsa_bf
     int rc = launch_li_scores(q_li, w_li, li_pool, n_slots, chunk_table, table_stride, kept_idx, kept_count, kept_cap,
                               window_start, B, Hl, dl, buf, dev_status, stream);
     if (rc) return rc;
-    topk_kept_kernel<<<B, kTopkThreads, 0, stream>>>(buf, kept_cap, kept_idx, kept_count, window_start, k, topk_idx,
-                                                     topk_count);
+    const int cap = stage_capacity(kept_cap * LSA_CHUNK);
+    LSA_CUDA(cudaFuncSetAttribute(topk_kept_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)(cap * sizeof(float))));
+    topk_kept_kernel<<<B, kTopkThreads, cap * sizeof(float), stream>>>(buf, kept_cap, kept_idx, kept_count,
+                                                                       window_start, k, topk_idx, topk_count, cap);
     return check_launch("topk_kept_kernel");
 }
 
@@ -176,6 +207,10 @@ extern "C" int lsa_topk_from_scores(const float *scores, const int64_t *cand_off
                 "lsa_topk_from_scores: null pointer or B <= 0");
     LSA_REQUIRE(max_cand >= 0, LSA_ERR_INVALID_ARG, "lsa_topk_from_scores: max_cand must be >= 0");
     LSA_REQUIRE(k >= 1 && k <= 65536, LSA_ERR_INVALID_ARG, "lsa_topk_from_scores: k=%d outside [1, 65536]", k);
-    topk_scores_kernel<<<B, kTopkThreads, 0, stream>>>(scores, cand_offset, max_cand, k, topk_idx, topk_count);
+    const int cap = stage_capacity(max_cand);
+    LSA_CUDA(cudaFuncSetAttribute(topk_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)(cap * sizeof(float))));
+    topk_scores_kernel<<<B, kTopkThreads, cap * sizeof(float), stream>>>(scores, cand_offset, max_cand, k, topk_idx,
+                                                                         topk_count, cap);
     return check_launch("topk_scores_kernel");
 }
