@@ -238,6 +238,34 @@ int lsa_label_vote(const float *scores, int n_layers, int n_steps, int n_chunks,
                    void *ws, size_t ws_bytes, lsa_stream_t stream);
 size_t lsa_label_vote_workspace_size(int n_layers, int n_steps, int n_chunks);
 
+/*
+ * a7 without a workspace, for callers that cannot allocate device memory.
+ * No passage of the paper corresponds to this entry point: it is the same
+ * label vote as lsa_label_vote, offered to code that is not allowed to call
+ * cudaMalloc at the point where it labels -- for example a plugin that may
+ * only touch memory its host handed over, or code running while the
+ * process's device allocator must not be entered.  Such callers pass only
+ * their inputs and outputs; the vote masks live in a fixed 4 MiB array built
+ * into the library (every GPU that loads the library keeps it until exit).
+ *
+ * Same arguments, results and limits as lsa_label_vote, plus:
+ *   - n_steps * n_chunks * ceil(n_layers / 32) must not exceed 1,048,576
+ *     (LSA_LABEL_VOTE_NOALLOC_MAX_WORDS); larger problems return
+ *     LSA_ERR_CAPACITY before anything is launched.
+ *   - The call allocates nothing (no cudaMalloc, cudaFree or allocating
+ *     library routine).  It clears the part of the array it uses on `stream`
+ *     before voting.
+ *   - The first call on a device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - Every call shares the one array: calls whose GPU work overlaps (on
+ *     different streams, or from different threads) race and must be ordered
+ *     by the caller.
+ */
+#define LSA_LABEL_VOTE_NOALLOC_MAX_WORDS (1u << 20)
+int lsa_label_vote_noalloc(const float *scores, int n_layers, int n_steps, int n_chunks,
+                           float top_p, int min_layers, int mode,
+                           uint8_t *labels, int32_t *max_votes, lsa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

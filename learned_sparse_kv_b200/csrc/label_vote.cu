@@ -7,6 +7,8 @@
 // sorted order, nucleus cut at the first prefix reaching top_p * Z, and an
 // atomicOr of the layer's bit into mask[step][chunk].  Kernel 2, per chunk:
 // per-step popcounts -> votes and labels.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace lsa {
@@ -194,6 +196,72 @@ extern "C" int lsa_label_vote(const float *scores, int n_layers, int n_steps, in
     nucleus_mark_kernel<<<n_layers * n_steps, kVoteThreads, smem, stream>>>(scores, n_layers, n_steps, n_chunks, npow2,
                                                                             top_p, masks, words);
     int rc = check_launch("nucleus_mark_kernel");
+    if (rc) return rc;
+    vote_kernel<<<(n_chunks + 255) / 256, 256, 0, stream>>>(masks, n_steps, n_chunks, words, min_layers, mode, labels,
+                                                            max_votes);
+    return check_launch("vote_kernel");
+}
+
+// ----------------------------------------------------------------------------
+// Label vote for callers that cannot allocate device memory.
+//
+// The vote needs one word per (step, chunk) of scratch.  Callers that may not
+// allocate -- code that runs where the device allocator must not be entered,
+// or a host that budgets every device byte up front and hands this library
+// only its inputs and outputs -- get that scratch from the fixed array below,
+// which every GPU that loads the library holds until the process exits.
+namespace lsa {
+
+constexpr size_t kStaticVoteWords = size_t(1) << 20;   // 4 MiB of uint32 vote masks
+static __device__ __align__(256) uint32_t g_vote_scratch[kStaticVoteWords];
+
+static std::mutex g_vote_scratch_lock;
+static uint32_t *g_vote_scratch_dev[64];   // device address of g_vote_scratch, per device
+
+// Host code may not use g_vote_scratch itself (it names a host-side stand-in);
+// the device address is looked up once per device, with that device current.
+static int vote_scratch(uint32_t **out) {
+    int dev = 0;
+    LSA_CUDA(cudaGetDevice(&dev));
+    LSA_REQUIRE(dev >= 0 && dev < 64, LSA_ERR_INVALID_ARG, "lsa_label_vote_noalloc: device %d out of range", dev);
+    std::lock_guard<std::mutex> guard(g_vote_scratch_lock);
+    if (!g_vote_scratch_dev[dev]) {
+        void *p = nullptr;
+        LSA_CUDA(cudaGetSymbolAddress(&p, g_vote_scratch));
+        g_vote_scratch_dev[dev] = static_cast<uint32_t *>(p);
+    }
+    *out = g_vote_scratch_dev[dev];
+    return LSA_OK;
+}
+
+}  // namespace lsa
+
+extern "C" int lsa_label_vote_noalloc(const float *scores, int n_layers, int n_steps, int n_chunks, float top_p,
+                                      int min_layers, int mode, uint8_t *labels, int32_t *max_votes,
+                                      lsa_stream_t stream) {
+    LSA_REQUIRE(scores && labels, LSA_ERR_INVALID_ARG, "lsa_label_vote_noalloc: null pointer");
+    LSA_REQUIRE(n_layers >= 1 && n_layers <= 64 && n_steps >= 1 && n_chunks >= 1 && n_chunks <= kMaxVoteChunks,
+                LSA_ERR_SHAPE, "lsa_label_vote_noalloc: unsupported sizes (layers=%d steps=%d chunks=%d)", n_layers,
+                n_steps, n_chunks);
+    LSA_REQUIRE(mode == 0 || mode == 1, LSA_ERR_INVALID_ARG, "lsa_label_vote_noalloc: mode must be 0 or 1");
+    LSA_REQUIRE(top_p > 0.f, LSA_ERR_INVALID_ARG, "lsa_label_vote_noalloc: top_p must be positive");
+    const int words = (n_layers + 31) / 32;
+    const size_t need = (size_t)n_steps * n_chunks * words;
+    LSA_REQUIRE(need <= kStaticVoteWords, LSA_ERR_CAPACITY,
+                "lsa_label_vote_noalloc: steps x chunks x ceil(layers/32) = %zu exceeds the built-in scratch of %zu "
+                "words; use lsa_label_vote with a caller workspace",
+                need, kStaticVoteWords);
+    uint32_t *masks = nullptr;
+    int rc = vote_scratch(&masks);
+    if (rc) return rc;
+    LSA_CUDA(cudaMemsetAsync(masks, 0, need * sizeof(uint32_t), stream));   // every call starts from zero
+    int npow2 = 2;
+    while (npow2 < n_chunks) npow2 <<= 1;
+    const size_t smem = (size_t)npow2 * (sizeof(float) + sizeof(int));
+    LSA_CUDA(cudaFuncSetAttribute(nucleus_mark_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    nucleus_mark_kernel<<<n_layers * n_steps, kVoteThreads, smem, stream>>>(scores, n_layers, n_steps, n_chunks, npow2,
+                                                                            top_p, masks, words);
+    rc = check_launch("nucleus_mark_kernel");
     if (rc) return rc;
     vote_kernel<<<(n_chunks + 255) / 256, 256, 0, stream>>>(masks, n_steps, n_chunks, words, min_layers, mode, labels,
                                                             max_votes);
