@@ -224,7 +224,7 @@ def time_attention_kernels(win, windows):
                              win.window_len, status=win.status)
             lsa.topk(t["q_li"][s], t["w_li"][s], t["li"], t["chunk_table"], win.kept_idx, win.kept_count,
                      t["window_start"], sh.k, scores=win.scores, status=win.status, topk_idx=win.topk_idx[s],
-                     topk_count=win.topk_count[s])
+                     topk_count=win.topk_count[s], ws=win.ws_topk)
             rec(evs[s][0])
             lsa.sparse_decode(t["q"][s], win.k_pool, win.v_pool, t["chunk_table"], win.topk_idx[s],
                               win.topk_count[s], t["window_start"], win.window_len, win.max_window_len, sh.dv,
@@ -330,7 +330,7 @@ def run_e2e(win, wl, args, world):
                              win.window_len, status=win.status)
             lsa.topk(dev_in["q_li"], dev_in["w_li"], t["li"], t["chunk_table"], win.kept_idx, win.kept_count,
                      t["window_start"], sh.k, scores=win.scores, status=win.status, topk_idx=win.topk_idx[s],
-                     topk_count=win.topk_count[s])
+                     topk_count=win.topk_count[s], ws=win.ws_topk)
             lsa.sparse_decode(dev_in["q"], win.k_pool, win.v_pool, t["chunk_table"], win.topk_idx[s],
                               win.topk_count[s], t["window_start"], win.window_len, win.max_window_len, sh.dv,
                               sh.scale, out=win.out[s], lse=win.lse[s], status=win.status, ws=win.ws_decode)

@@ -179,32 +179,19 @@ __global__ void __launch_bounds__(256) nmi_compact_kernel(const unsigned long lo
 
 // ------------------------------------------------------------------- a2 ----
 
-// Number of kept chunks below the window: kept lists are ascending.
-__device__ __forceinline__ int cold_kept(const int32_t *kept, int count, int first_window_chunk) {
-    int lo = 0, hi = count;
-    while (lo < hi) {
-        int mid = (lo + hi) >> 1;
-        if (kept[mid] < first_window_chunk) lo = mid + 1;
-        else hi = mid;
-    }
-    return lo;
-}
-
 // grid (G, B): CTA x of sequence b scores kept cold chunks x, x+G, ...
 template <int D>
 __global__ void __launch_bounds__(128) li_score_kernel(const uint16_t *__restrict__ q_li, const uint16_t *__restrict__ w_li,
                                                        const uint16_t *__restrict__ li_pool, int64_t n_slots,
                                                        const int32_t *__restrict__ table, int table_stride,
                                                        const int32_t *__restrict__ kept_idx,
-                                                       const int32_t *__restrict__ kept_count, int kept_cap,
-                                                       const int32_t *__restrict__ window_start, int H,
+                                                       const int32_t *__restrict__ cold, int kept_cap, int H,
                                                        float *__restrict__ scores, int32_t *status) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     IdxSmem &sm = *reinterpret_cast<IdxSmem *>(smem_raw);
     const int b = blockIdx.y;
     const int32_t *kept = kept_idx + (size_t)b * kept_cap;
-    const int cnt = min(kept_count[b], kept_cap);
-    const int n_cold = cold_kept(kept, cnt, window_start[b] / LSA_CHUNK);
+    const int n_cold = cold[b];
     if ((int)blockIdx.x >= n_cold) return;
     load_queries<D>(sm, q_li + (size_t)b * H * D, w_li + (size_t)b * H, H);
     const int32_t *trow = table + (size_t)b * table_stride;
@@ -229,10 +216,21 @@ __global__ void __launch_bounds__(128) li_score_kernel(const uint16_t *__restric
 
 static bool heads_ok(int H) { return H >= 8 && H <= kMaxHeads && H % 8 == 0; }
 
+namespace li2 {
+bool shape_ok(int H, int D, int B);
+int launch(const uint16_t *q_li, const uint16_t *w_li, const uint16_t *li_pool, int64_t n_slots, const int32_t *table,
+           int table_stride, const int32_t *kept_idx, const int32_t *kept_count, int kept_cap,
+           const int32_t *cold, int B, int H, int D, float *scores, int32_t *status, cudaStream_t stream);
+}  // namespace li2
+
 int launch_li_scores(const uint16_t *q_li, const uint16_t *w_li, const uint16_t *li_pool, int64_t n_slots,
                      const int32_t *table, int table_stride, const int32_t *kept_idx, const int32_t *kept_count,
-                     int kept_cap, const int32_t *window_start, int B, int H, int D, float *scores,
-                     int32_t *status, cudaStream_t stream) {
+                     int kept_cap, const int32_t *window_start, const int32_t *cold, int B, int H, int D,
+                     float *scores, int32_t *status, cudaStream_t stream) {
+    // Head counts of 32, 64 or 128 run on tcgen05 (M = 128 tokens, N = heads); others on mma.sync.
+    if (li2::shape_ok(H, D, B))
+        return li2::launch(q_li, w_li, li_pool, n_slots, table, table_stride, kept_idx, kept_count, kept_cap,
+                           cold, B, H, D, scores, status, stream);
     const size_t smem = sizeof(IdxSmem);
     int per_seq = (sm_count() * 8 + B - 1) / B;
     per_seq = max(1, min(per_seq, kept_cap));
@@ -240,11 +238,11 @@ int launch_li_scores(const uint16_t *q_li, const uint16_t *w_li, const uint16_t 
     if (D == 128) {
         cudaFuncSetAttribute(li_score_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         li_score_kernel<128><<<grid, 128, smem, stream>>>(q_li, w_li, li_pool, n_slots, table, table_stride, kept_idx,
-                                                          kept_count, kept_cap, window_start, H, scores, status);
+                                                          cold, kept_cap, H, scores, status);
     } else {
         cudaFuncSetAttribute(li_score_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         li_score_kernel<64><<<grid, 128, smem, stream>>>(q_li, w_li, li_pool, n_slots, table, table_stride, kept_idx,
-                                                         kept_count, kept_cap, window_start, H, scores, status);
+                                                         cold, kept_cap, H, scores, status);
     }
     return check_launch("li_score_kernel");
 }

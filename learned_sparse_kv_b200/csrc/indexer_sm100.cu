@@ -1,0 +1,309 @@
+// indexer_sm100.cu -- a2 on 5th-generation tensor cores: Lightning-Indexer token
+// scores over the tokens of kept chunks that lie before the recent window.
+// (arXiv 2606.09079: the native indexer's finer top-k inside the fetched set,
+// gist.science explainer 2.1 "Gestufte Selektion"; cjcn.com.cn article section 2.)
+//
+//   score(t) = sum_h w_h * max(0, q_h . key_t)
+//
+// Persistent CTAs walk contiguous ranges of "tiles": two consecutive kept cold
+// chunks of one sequence = 128 tokens.  Per tile one tcgen05.mma chain computes
+// D[128 tokens x H heads] = keys[128 x dl] . q^T[dl x H] into tensor memory
+// (M = 128, N = H, K = dl in steps of 16); an epilogue warpgroup reads one
+// token row per thread, applies ReLU and the head weights, and writes the
+// score.  Keys arrive by TMA tile loads of whole chunk slots (64 rows x 64
+// columns, 128-byte swizzle) into a 3-stage ring; the per-sequence query heads
+// live in two buffers so a CTA can cross a sequence boundary without a stall.
+// Warp roles: 0 TMA producer, 1 MMA issuer (also allocates TMEM), 2..5 epilogue.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace lsa {
+namespace li2 {
+
+using namespace sm100;
+
+constexpr int THREADS = 192;
+constexpr int STAGES = 3;
+constexpr int MAX_H = 128, MAX_D = 128;
+constexpr uint32_t WAIT_LIMIT = 1u << 22;
+
+struct __align__(1024) Smem {
+    uint8_t keys[STAGES][MAX_D / 64][128 * 128];   // [atom][128 token rows][128 B]
+    uint8_t q[2][MAX_D / 64][MAX_H * 128];          // [buffer][atom][H rows][128 B]
+    uint64_t k_full[STAGES], k_empty[STAGES];
+    uint64_t q_full[2], q_empty[2];
+    uint64_t acc_full[2], acc_empty[2];
+    uint64_t mma_done;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+struct Params {
+    const uint16_t *w_li;
+    const int32_t *table;
+    const int32_t *kept_idx;
+    const int32_t *cold;          // kept chunks before the window, per sequence
+    float *scores;
+    int32_t *status;
+    int64_t n_slots;
+    int B, H, D, table_stride, kept_cap;
+};
+
+// 1-CTA MMA and commit
+__device__ __forceinline__ void umma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, bool acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(uint32_t(acc)));
+}
+__device__ __forceinline__ void commit(const uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void tma_load_2d_local(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(
+            smem_addr(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(smem_addr(bar))
+        : "memory");
+}
+__device__ __forceinline__ void expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_addr(bar)) : "memory");
+}
+
+// Work list shared by all roles of a CTA: tile t of the whole batch -> (sequence, first kept index).
+struct Work {
+    int tile_off[65];   // prefix of tiles per sequence (B <= 64)
+    int cold[64];
+    int first, last;    // tile range of this CTA
+};
+
+__device__ void build_work(const Params &p, Work &wk) {
+    if (threadIdx.x == 0) {
+        int acc = 0;
+        for (int b = 0; b < p.B; ++b) {
+            wk.tile_off[b] = acc;
+            wk.cold[b] = p.cold[b];
+            acc += (wk.cold[b] + 1) >> 1;
+        }
+        wk.tile_off[p.B] = acc;
+        wk.first = (int)((int64_t)blockIdx.x * acc / gridDim.x);
+        wk.last = (int)((int64_t)(blockIdx.x + 1) * acc / gridDim.x);
+    }
+}
+
+__device__ __forceinline__ int tile_seq(const Work &wk, int B, int t) {
+    int b = 0;
+    while (b + 1 < B && wk.tile_off[b + 1] <= t) ++b;
+    return b;
+}
+
+__device__ __forceinline__ bool bounded(Smem &sm, const uint64_t *bar, uint32_t parity, int32_t *status) {
+    if (sm.abort_flag) return false;
+    if (mbar_wait(bar, parity, WAIT_LIMIT)) return true;
+    sm.abort_flag = 1;
+    flag(status, LSA_DEV_TIMEOUT);
+    return false;
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+li_score_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_constant__ CUtensorMap q_map,
+                const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem &sm = *reinterpret_cast<Smem *>(smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023));
+    __shared__ Work wk;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int atoms = p.D / 64;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) { mbar_init(&sm.k_full[i], 1); mbar_init(&sm.k_empty[i], 1); }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.q_full[i], 1); mbar_init(&sm.q_empty[i], 1);
+            mbar_init(&sm.acc_full[i], 1); mbar_init(&sm.acc_empty[i], 1);
+        }
+        mbar_init(&sm.mma_done, 1);
+        sm.abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    build_work(p, wk);
+    if (warp == 1) asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
+                                    smem_addr(&sm.tmem_base)), "r"(256));
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    const int t0 = wk.first, t1 = wk.last;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        int kslot = 0;
+        uint32_t kpar = 0;
+        int cur_b = -1, qbuf = 1, qswitch = 0;
+        for (int t = t0; t < t1; ++t) {
+            const int b = tile_seq(wk, p.B, t);
+            if (b != cur_b) {                              // query heads and weights of a new sequence
+                cur_b = b;
+                qbuf ^= 1;
+                if (qswitch >= 2 && !bounded(sm, &sm.q_empty[qbuf], ((qswitch - 2) >> 1) & 1, p.status)) break;
+                ++qswitch;
+                if (lane == 0) {
+                    expect_tx(&sm.q_full[qbuf], (uint32_t)(atoms * p.H * 128));
+                    for (int a = 0; a < atoms; ++a) tma_load_2d_local(sm.q[qbuf][a], &q_map, 64 * a, b * p.H, &sm.q_full[qbuf]);
+                }
+                __syncwarp();
+            }
+            if (!bounded(sm, &sm.k_empty[kslot], kpar ^ 1u, p.status)) break;
+            if (lane == 0) {
+                const int j0 = 2 * (t - wk.tile_off[b]);
+                const int32_t *kept = p.kept_idx + (size_t)b * p.kept_cap;
+                const int nck = min(2, wk.cold[b] - j0);
+                expect_tx(&sm.k_full[kslot], (uint32_t)(nck * atoms * 64 * 128));
+                for (int i = 0; i < nck; ++i) {
+                    const int chunk = kept[j0 + i];
+                    int slot = (chunk >= 0 && chunk < p.table_stride) ? p.table[(size_t)b * p.table_stride + chunk] : -1;
+                    if (slot < 0 || slot >= p.n_slots) slot = (int)p.n_slots;   // out of range: zero fill
+                    for (int a = 0; a < atoms; ++a)
+                        tma_load_2d_local(sm.keys[kslot][a] + i * 64 * 128, &key_map, 64 * a, slot * LSA_CHUNK,
+                                          &sm.k_full[kslot]);
+                }
+            }
+            __syncwarp();
+            if (++kslot == STAGES) { kslot = 0; kpar ^= 1u; }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        const uint32_t idesc = idesc_bf16_f32(128, p.H, false, false);
+        int kslot = 0;
+        uint32_t kpar = 0;
+        int cur_b = -1, qbuf = 1, qswitch = 0;
+        bool ok = true;
+        for (int t = t0, u = 0; t < t1 && ok; ++t, ++u) {
+            const int b = tile_seq(wk, p.B, t);
+            if (b != cur_b) {
+                if (cur_b >= 0 && lane == 0) commit(&sm.q_empty[qbuf]);   // previous buffer free after its MMAs
+                cur_b = b;
+                qbuf ^= 1;
+                ok = bounded(sm, &sm.q_full[qbuf], (qswitch >> 1) & 1, p.status);
+                ++qswitch;
+                if (!ok) break;
+            }
+            const int ab = u & 1;
+            if (u >= 2 && !(ok = bounded(sm, &sm.acc_empty[ab], ((u - 2) >> 1) & 1, p.status))) break;
+            if (!(ok = bounded(sm, &sm.k_full[kslot], kpar, p.status))) break;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t d = tmem + 64 * ab * (p.H > 64 ? 2 : 1);
+                for (int a = 0; a < atoms; ++a) {
+                    const uint64_t ad = smem_desc_sw128(smem_addr(sm.keys[kslot][a]), 16, 1024);
+                    const uint64_t bd = smem_desc_sw128(smem_addr(sm.q[qbuf][a]), 16, 1024);
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) umma(d, ad + 2 * k4, bd + 2 * k4, idesc, (a | k4) != 0);
+                }
+                commit(&sm.k_empty[kslot]);
+                commit(&sm.acc_full[ab]);
+            }
+            __syncwarp();
+            if (++kslot == STAGES) { kslot = 0; kpar ^= 1u; }
+        }
+        if (cur_b >= 0 && lane == 0) commit(&sm.q_empty[qbuf]);
+        if (lane == 0) {                                   // every MMA has completed before TMEM is released
+            commit(&sm.mma_done);
+            if (!mbar_wait(&sm.mma_done, 0, WAIT_LIMIT)) flag(p.status, LSA_DEV_TIMEOUT);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------ epilogue: one token row per thread
+        const int L = threadIdx.x - 64;                       // 0..127
+        const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+        const int row = 32 * (warp & 3) + lane;               // TMEM lane = token row of the tile
+        bool ok = true;
+        for (int t = t0, u = 0; t < t1; ++t, ++u) {
+            const int b = tile_seq(wk, p.B, t);
+            const uint16_t *wb = p.w_li + (size_t)b * p.H;
+            const int ab = u & 1;
+            if (ok) ok = bounded(sm, &sm.acc_full[ab], (u >> 1) & 1, p.status);
+            tc_fence_after();
+            const uint32_t base = tmem + lane_base + 64 * ab * (p.H > 64 ? 2 : 1);
+            float acc = 0.f;
+            for (int c0 = 0; c0 < p.H; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld32(base + c0, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) acc += bf16_to_f32(wb[c0 + i]) * fmaxf(__uint_as_float(v[i]), 0.f);
+            }
+            tc_fence_before();
+            named_barrier(1, 128);
+            if (L == 0) arrive(&sm.acc_empty[ab]);
+            // write the score of this row if it belongs to a kept cold chunk of the sequence
+            const int j0 = 2 * (t - wk.tile_off[b]);
+            const int jj = j0 + (row >> 6);
+            if (ok && jj < wk.cold[b]) {
+                const int chunk = p.kept_idx[(size_t)b * p.kept_cap + jj];
+                const int slot = (chunk >= 0 && chunk < p.table_stride) ? p.table[(size_t)b * p.table_stride + chunk] : -1;
+                const bool valid = slot >= 0 && slot < p.n_slots;
+                if (!valid && (row & 63) == 0) flag(p.status, LSA_DEV_TABLE);
+                p.scores[((size_t)b * p.kept_cap + jj) * LSA_CHUNK + (row & 63)] = valid ? acc : -INFINITY;
+            }
+        }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(256));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
+    }
+}
+
+// --------------------------------------------------------------- host side --
+
+typedef CUresult (*EncodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static bool make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+    static EncodeTiled fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return false;
+        fn = reinterpret_cast<EncodeTiled>(ptr);
+    }
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t es[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool shape_ok(int H, int D, int B) { return (H == 32 || H == 64 || H == 128) && (D == 64 || D == 128) && B <= 64; }
+
+int launch(const uint16_t *q_li, const uint16_t *w_li, const uint16_t *li_pool, int64_t n_slots, const int32_t *table,
+           int table_stride, const int32_t *kept_idx, const int32_t *kept_count, int kept_cap,
+           const int32_t *cold, int B, int H, int D, float *scores, int32_t *status, cudaStream_t stream) {
+    CUtensorMap key_map, q_map;
+    if (!make_map(&key_map, li_pool, D, (uint64_t)n_slots * LSA_CHUNK, LSA_CHUNK))
+        return fail(LSA_ERR_CUDA, "lsa_topk: cuTensorMapEncodeTiled failed for the indexer key pool");
+    if (!make_map(&q_map, q_li, D, (uint64_t)B * H, H))
+        return fail(LSA_ERR_CUDA, "lsa_topk: cuTensorMapEncodeTiled failed for the indexer queries");
+    Params prm;
+    (void)kept_count;
+    prm.w_li = w_li; prm.table = table; prm.kept_idx = kept_idx; prm.cold = cold; prm.scores = scores; prm.status = status; prm.n_slots = n_slots;
+    prm.B = B; prm.H = H; prm.D = D; prm.table_stride = table_stride; prm.kept_cap = kept_cap;
+    const size_t smem = sizeof(Smem) + 1024;
+    LSA_CUDA(cudaFuncSetAttribute(li_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    li_score_kernel<<<sm_count(), THREADS, smem, stream>>>(key_map, q_map, prm);
+    return check_launch("li_score_kernel (sm100)");
+}
+
+}  // namespace li2
+}  // namespace lsa

@@ -29,13 +29,18 @@ __device__ __forceinline__ uint32_t map_to_rank(const void *p, uint32_t rank) {
     return out;
 }
 
+// Arrivals and waits use the default (CTA-scope) semantics.  The data they
+// guard is either written by TMA (complete_tx makes it visible to the waiter)
+// or by generic stores followed by fence.proxy.async before the arrive, and
+// everything the pair's tensor cores touch is ordered by tcgen05 fences; the
+// cluster-scope variants cost a fence per hand-off and halved the attention
+// throughput when measured.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_addr) : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_addr) : "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t cluster_addr, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;\n" ::"r"(cluster_addr),
-                 "r"(bytes)
+    asm volatile("mbarrier.arrive.expect_tx.shared::cluster.b64 _, [%0], %1;\n" ::"r"(cluster_addr), "r"(bytes)
                  : "memory");
 }
 
@@ -43,7 +48,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}\n"
         : "=r"(ok)
         : "r"(addr), "r"(parity)

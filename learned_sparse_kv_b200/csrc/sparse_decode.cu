@@ -300,6 +300,15 @@ __global__ void lse_merge_kernel(const float *__restrict__ o_part, const float *
             make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
     if (lse && threadIdx.x == 0)
         lse[(size_t)b * Hq + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
+    // The partial rows of this head are dead now: drop their L2 lines without
+    // writing them back, so split-K scratch costs no DRAM write bandwidth.
+    __syncthreads();
+    const int lines = DV * 4 / 128;
+    for (int i = threadIdx.x; i < n_splits * lines; i += blockDim.x) {
+        const size_t idx = ((size_t)b * n_splits + i / lines) * Hq + h;
+        const float *line = o_part + idx * DV + (i % lines) * 32;
+        asm volatile("discard.global.L2 [%0], 128;\n" ::"l"(line) : "memory");
+    }
 }
 
 using CfgSep16 = DecodeCfg<16, 128, 128, 4, false>;

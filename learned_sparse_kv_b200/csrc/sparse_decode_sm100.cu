@@ -37,7 +37,7 @@ constexpr int HQ = 128;           // heads per cluster
 constexpr int DQK = 576, DV = 512;
 constexpr int NTILE = 64;         // kv rows per tile
 constexpr int KCH = DQK / 64;     // 9 column chunks of 64
-constexpr int KST = 12;           // K ring: [32 rows x 64 cols] stages
+constexpr int KST = 16;           // K ring: [32 rows x 64 cols] stages
 constexpr int VST = 4;            // V ring: [2 atoms][64 rows][64 cols] stages
 constexpr int INFO = 4;           // tile-validity ring
 constexpr int THREADS = 256;
@@ -58,7 +58,7 @@ struct __align__(1024) Smem {
     uint64_t v_full[VST], v_empty[VST];
     uint64_t q_full;
     uint64_t s_full[2], s_empty[2], p_full[2];
-    uint64_t pv_done, mma_done;
+    uint64_t pv_done[2], mma_done;   // pv_done[s]: P.V of the tiles using P buffer s
     uint64_t info_full[INFO], info_empty[INFO];
     unsigned long long info_mask[INFO];
     float red[128];
@@ -88,6 +88,18 @@ struct SeqTiles {
         wlen = max(p.window_len[b], 0);
         t_topk = (tk + NTILE - 1) / NTILE;
         total = t_topk + (wlen + NTILE - 1) / NTILE;
+    }
+    // Window tile t (t >= t_topk) covers one whole chunk slot: first pool row of
+    // the slot (-2 if the chunk has no slot) and the number of valid rows.
+    __device__ int64_t window_slot_row(const Params &p, int b, int t, int *n_valid) const {
+        const int j = t - t_topk;
+        *n_valid = min(NTILE, wlen - NTILE * j);
+        const int chunk = (wstart >> 6) + j;
+        if (wstart < 0 || chunk >= p.table_stride) return -2;
+        const int slot = p.table[(size_t)b * p.table_stride + chunk];
+        const int64_t g = (int64_t)slot * LSA_CHUNK;
+        if (slot < 0 || g >= p.n_rows_pool) return -2;
+        return g;
     }
     // Global pool row of row i (0..63) of tile t, or -1.
     __device__ int64_t row(const Params &p, int b, int t, int i) const {
@@ -127,7 +139,8 @@ __device__ __forceinline__ bool warp_wait(Smem &sm, const uint64_t *bar, uint32_
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
-mla_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_constant__ CUtensorMap q_map,
+mla_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_constant__ CUtensorMap kv_map32,
+                  const __grid_constant__ CUtensorMap kv_map64, const __grid_constant__ CUtensorMap q_map,
                   const Params p) {
     extern __shared__ uint8_t smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>(smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023));
@@ -140,7 +153,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_const
         for (int i = 0; i < VST; ++i) { mbar_init(&sm.v_full[i], 2); mbar_init(&sm.v_empty[i], 1); }
         mbar_init(&sm.q_full, 2);
         for (int i = 0; i < 2; ++i) { mbar_init(&sm.s_full[i], 1); mbar_init(&sm.s_empty[i], 2); mbar_init(&sm.p_full[i], 2); }
-        mbar_init(&sm.pv_done, 1);
+        mbar_init(&sm.pv_done[0], 1);
+        mbar_init(&sm.pv_done[1], 1);
         mbar_init(&sm.mma_done, 1);
         for (int i = 0; i < INFO; ++i) { mbar_init(&sm.info_full[i], 1); mbar_init(&sm.info_empty[i], 1); }
         sm.abort_flag = 0;
@@ -154,9 +168,11 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_const
     const uint32_t tmem = sm.tmem_base;
 
     const SeqTiles st(p, b);
-    const int u0 = (int)((int64_t)split * st.total / p.n_splits);        // balanced contiguous ranges
-    const int u1 = (int)((int64_t)(split + 1) * st.total / p.n_splits);
-    const int n_tiles = u1 - u0;
+    // Tiles are dealt round-robin: split s takes tiles s, s + n_splits, ...  The
+    // gathered top-k tiles (first in the tile list, and dearer to load than the
+    // chunk-aligned window tiles) are thereby spread evenly over the splits.
+    const int n_tiles = split < st.total ? (st.total - 1 - split) / p.n_splits + 1 : 0;
+    const int u0 = split, ustride = p.n_splits;
 
     if (warp == 0 && n_tiles > 0) {
         // ------------------------------------------------ K producer + Q
@@ -166,118 +182,165 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_const
             for (int c = 0; c < KCH; ++c) tma_load_2d(sm.q[c], &q_map, 64 * c, b * HQ + HPC * (int)rank, qf);
         }
         uint32_t kc = 0;
+        // row indices of the next top-k tile are loaded while the current tile is issued
+        int64_t n0 = -1, n1 = -1;
+        if (u0 < st.t_topk) { n0 = st.row(p, b, u0, lane); n1 = st.row(p, b, u0, lane + 32); }
         for (int u = 0; u < n_tiles; ++u) {
-            const int t = u0 + u;
-            // rows lane and lane + 32 of the tile (validity), and this CTA's K row (32 * rank + lane)
-            const int64_t g0 = st.row(p, b, t, lane), g1 = st.row(p, b, t, lane + 32);
-            if ((g0 == -2 || g1 == -2)) flag(p.status, LSA_DEV_TABLE);
-            const unsigned lo = __ballot_sync(0xffffffffu, g0 >= 0), hi = __ballot_sync(0xffffffffu, g1 >= 0);
+            const int t = u0 + u * ustride;
+            const bool window = t >= st.t_topk;
+            const int64_t g0 = n0, g1 = n1;
+            if (u + 1 < n_tiles && t + ustride < st.t_topk) {
+                n0 = st.row(p, b, t + ustride, lane);
+                n1 = st.row(p, b, t + ustride, lane + 32);
+            }
+            unsigned long long mask;
+            int64_t slot_row = -1;
+            if (window) {
+                int nv;
+                slot_row = st.window_slot_row(p, b, t, &nv);
+                if (slot_row == -2) flag(p.status, LSA_DEV_TABLE);
+                mask = slot_row < 0 ? 0ull : (nv >= 64 ? ~0ull : ((1ull << nv) - 1ull));
+            } else {
+                if ((g0 == -2 || g1 == -2)) flag(p.status, LSA_DEV_TABLE);
+                const unsigned lo = __ballot_sync(0xffffffffu, g0 >= 0), hi = __ballot_sync(0xffffffffu, g1 >= 0);
+                mask = (unsigned long long)lo | ((unsigned long long)hi << 32);
+            }
             if (!warp_wait(sm, &sm.info_empty[u % INFO], ((u / INFO) + 1) & 1, p.status)) break;
             if (lane == 0) {
-                sm.info_mask[u % INFO] = (unsigned long long)lo | ((unsigned long long)hi << 32);
+                sm.info_mask[u % INFO] = mask;
                 asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];\n" ::"r"(smem_addr(&sm.info_full[u % INFO])) : "memory");
             }
             const int64_t mine = rank ? g1 : g0;
             const int gr = mine >= 0 ? (int)mine : (int)p.n_rows_pool;   // out of range -> zero fill
+            const int r0 = __shfl_sync(0xffffffffu, gr, (4 * lane) & 31), r1 = __shfl_sync(0xffffffffu, gr, (4 * lane + 1) & 31);
+            const int r2 = __shfl_sync(0xffffffffu, gr, (4 * lane + 2) & 31), r3 = __shfl_sync(0xffffffffu, gr, (4 * lane + 3) & 31);
+            const int wy = slot_row >= 0 ? (int)slot_row + 32 * (int)rank : (int)p.n_rows_pool;
             bool ok = true;
-            for (int c = 0; c < KCH && ok; ++c, ++kc) {
+            for (int c = 0; c < KCH; ++c, ++kc) {
                 const int s = kc % KST;
                 ok = warp_wait(sm, &sm.k_empty[s], ((kc / KST) + 1) & 1, p.status);
                 if (!ok) break;
                 const uint32_t full = map_to_rank(&sm.k_full[s], 0);
-                if (lane == 0) mbar_arrive_expect_tx_cluster(full, 32 * 128);
+                if (lane == 0) {
+                    mbar_arrive_expect_tx_cluster(full, 32 * 128);
+                    if (window) tma_load_2d(sm.k[s], &kv_map32, 64 * c, wy, full);
+                }
                 __syncwarp();
-                const int r0 = __shfl_sync(0xffffffffu, gr, (4 * lane) & 31), r1 = __shfl_sync(0xffffffffu, gr, (4 * lane + 1) & 31);
-                const int r2 = __shfl_sync(0xffffffffu, gr, (4 * lane + 2) & 31), r3 = __shfl_sync(0xffffffffu, gr, (4 * lane + 3) & 31);
-                if (lane < 8) tma_gather4(sm.k[s] + lane * 512, &kv_map, 64 * c, r0, r1, r2, r3, full);
+                if (!window && lane < 8) tma_gather4(sm.k[s] + lane * 512, &kv_map, 64 * c, r0, r1, r2, r3, full);
             }
             if (!ok) break;
         }
     } else if (warp == 1 && n_tiles > 0) {
         // ------------------------------------------------ V producer
         uint32_t vc = 0;
+        int64_t n0 = -1, n1 = -1;
+        if (u0 < st.t_topk) { n0 = st.row(p, b, u0, lane); n1 = st.row(p, b, u0, lane + 32); }
         for (int u = 0; u < n_tiles; ++u) {
-            const int t = u0 + u;
-            const int64_t g0 = st.row(p, b, t, lane), g1 = st.row(p, b, t, lane + 32);
+            const int t = u0 + u * ustride;
+            const bool window = t >= st.t_topk;
+            const int64_t g0 = n0, g1 = n1;
+            if (u + 1 < n_tiles && t + ustride < st.t_topk) {
+                n0 = st.row(p, b, t + ustride, lane);
+                n1 = st.row(p, b, t + ustride, lane + 32);
+            }
+            int wy = (int)p.n_rows_pool;
+            if (window) {
+                int nv;
+                const int64_t sr = st.window_slot_row(p, b, t, &nv);
+                if (sr >= 0) wy = (int)sr;
+            }
             const int a0 = g0 >= 0 ? (int)g0 : (int)p.n_rows_pool, a1 = g1 >= 0 ? (int)g1 : (int)p.n_rows_pool;
+            // lane -> (value atom a = lane / 16, row group gq = lane % 16: rows 4gq .. 4gq + 3)
+            const int gq = lane & 15, a = lane >> 4;
+            int r[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int row = 4 * gq + i;
+                const int x0 = __shfl_sync(0xffffffffu, a0, row & 31), x1 = __shfl_sync(0xffffffffu, a1, row & 31);
+                r[i] = row < 32 ? x0 : x1;
+            }
             bool ok = true;
             for (int j = 0; j < 2 && ok; ++j, ++vc) {
                 const int s = vc % VST;
                 ok = warp_wait(sm, &sm.v_empty[s], ((vc / VST) + 1) & 1, p.status);
                 if (!ok) break;
                 const uint32_t full = map_to_rank(&sm.v_full[s], 0);
-                if (lane == 0) mbar_arrive_expect_tx_cluster(full, 2 * NTILE * 128);
-                __syncwarp();
-                // lane -> (value atom a = lane / 16, row group gq = lane % 16: rows 4gq .. 4gq + 3)
-                const int gq = lane & 15, a = lane >> 4;
-                int r[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int row = 4 * gq + i;
-                    const int x0 = __shfl_sync(0xffffffffu, a0, row & 31), x1 = __shfl_sync(0xffffffffu, a1, row & 31);
-                    r[i] = row < 32 ? x0 : x1;
+                const int col0 = 256 * j + 128 * (int)rank;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx_cluster(full, 2 * NTILE * 128);
+                    if (window) {
+                        tma_load_2d(sm.v[s][0], &kv_map64, col0, wy, full);
+                        tma_load_2d(sm.v[s][1], &kv_map64, col0 + 64, wy, full);
+                    }
                 }
-                const int col = 256 * j + 128 * (int)rank + 64 * a;
-                tma_gather4(sm.v[s][a] + gq * 512, &kv_map, col, r[0], r[1], r[2], r[3], full);
+                __syncwarp();
+                if (!window) tma_gather4(sm.v[s][a] + gq * 512, &kv_map, col0 + 64 * a, r[0], r[1], r[2], r[3], full);
             }
             if (!ok) break;
         }
     } else if (warp == 2 && rank == 0 && n_tiles > 0) {
         // ------------------------------------------------ MMA issuer (even CTA)
-        const uint32_t idesc_qk = idesc_bf16_f32(128, NTILE, false, false);
-        const uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
+        // Descriptors are built once; a byte offset o within shared memory is
+        // o >> 4 added to the descriptor's start-address field.
+        constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, NTILE, false, false);
+        constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 256, false, true);
+        const uint64_t qd0 = smem_desc_sw128(smem_addr(sm.q[0]), 16, 1024);
+        const uint64_t kd0 = smem_desc_sw128(smem_addr(sm.k[0]), 16, 1024);
+        const uint64_t pd0 = smem_desc_sw128(smem_addr(sm.p[0]), 16, 1024);
+        const uint64_t vd0 = smem_desc_sw128(smem_addr(sm.v[0][0]), NTILE * 128, 1024);
+        constexpr uint64_t Q_CHUNK = (HPC * 128) >> 4, K_STAGE = (32 * 128) >> 4, P_BUF = (HPC * 128) >> 4;
+        constexpr uint64_t V_STAGE = (2 * NTILE * 128) >> 4, K16 = 32 >> 4, V16 = (16 * 128) >> 4;
         bool ok = warp_wait(sm, &sm.q_full, 0, p.status);
-        uint32_t kc = 0, vc = 0;
-        auto qk = [&](int u) -> bool {
-            const int s = u & 1;
-            if (!warp_wait(sm, &sm.s_empty[s], ((u >> 1) + 1) & 1, p.status)) return false;
-            tc_fence_after();
-            for (int c = 0; c < KCH; ++c, ++kc) {
-                const int ks_ = kc % KST;
-                if (!warp_wait(sm, &sm.k_full[ks_], (kc / KST) & 1, p.status)) return false;
+        int kslot = 0, vslot = 0;
+        uint32_t kpar = 0, vpar = 0;
+        for (int u = -1; u < n_tiles && ok; ++u) {
+            if (u + 1 < n_tiles) {                         // S(u+1) = Q K^T
+                const int t = u + 1, sb = t & 1;
+                ok = warp_wait(sm, &sm.s_empty[sb], ((t >> 1) + 1) & 1, p.status);
                 tc_fence_after();
-                if (lane == 0) {
-#pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) {
-                        const uint64_t ad = smem_desc_sw128(smem_addr(sm.q[c]) + 32 * k4, 16, 1024);
-                        const uint64_t bd = smem_desc_sw128(smem_addr(sm.k[ks_]) + 32 * k4, 16, 1024);
-                        umma_pair_ss(tmem + TM_S + 32 * s, ad, bd, idesc_qk, (c | k4) != 0);
+                const uint32_t d = tmem + TM_S + 32 * sb;
+                for (int c = 0; c < KCH && ok; ++c) {
+                    ok = warp_wait(sm, &sm.k_full[kslot], kpar, p.status);
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint64_t a = qd0 + Q_CHUNK * c, bb = kd0 + K_STAGE * kslot;
+                        umma_pair_ss(d, a, bb, IDESC_QK, c != 0);
+                        umma_pair_ss(d, a + K16, bb + K16, IDESC_QK, true);
+                        umma_pair_ss(d, a + 2 * K16, bb + 2 * K16, IDESC_QK, true);
+                        umma_pair_ss(d, a + 3 * K16, bb + 3 * K16, IDESC_QK, true);
+                        umma_commit_pair(&sm.k_empty[kslot], 0x3);
                     }
-                    umma_commit_pair(&sm.k_empty[ks_], 0x3);
+                    __syncwarp();
+                    if (++kslot == KST) { kslot = 0; kpar ^= 1u; }
                 }
+                if (lane == 0) umma_commit_pair(&sm.s_full[sb], 0x3);
                 __syncwarp();
             }
-            if (lane == 0) umma_commit_pair(&sm.s_full[s], 0x3);
-            __syncwarp();
-            return true;
-        };
-        auto pv = [&](int u) -> bool {
-            const int s = u & 1;
-            if (!warp_wait(sm, &sm.p_full[s], (u >> 1) & 1, p.status)) return false;
-            tc_fence_after();
-            for (int j = 0; j < 2; ++j, ++vc) {
-                const int vs = vc % VST;
-                if (!warp_wait(sm, &sm.v_full[vs], (vc / VST) & 1, p.status)) return false;
+            if (u >= 0 && ok) {                            // O += P V for tile u
+                const int sb = u & 1;
+                ok = warp_wait(sm, &sm.p_full[sb], (u >> 1) & 1, p.status);
                 tc_fence_after();
-                if (lane == 0) {
-#pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) {
-                        const uint64_t ad = smem_desc_sw128(smem_addr(sm.p[s]) + 32 * k4, 16, 1024);
-                        const uint64_t bd = smem_desc_sw128(smem_addr(sm.v[vs][0]) + 2048 * k4, NTILE * 128, 1024);
-                        umma_pair_ss(tmem + TM_O + 128 * j, ad, bd, idesc_pv, (u | k4) != 0);
+                const uint64_t a = pd0 + P_BUF * sb;
+                for (int j = 0; j < 2 && ok; ++j) {
+                    ok = warp_wait(sm, &sm.v_full[vslot], vpar, p.status);
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint64_t bb = vd0 + V_STAGE * vslot;
+                        const uint32_t d = tmem + TM_O + 128 * j;
+                        umma_pair_ss(d, a, bb, IDESC_PV, u != 0);
+                        umma_pair_ss(d, a + K16, bb + V16, IDESC_PV, true);
+                        umma_pair_ss(d, a + 2 * K16, bb + 2 * V16, IDESC_PV, true);
+                        umma_pair_ss(d, a + 3 * K16, bb + 3 * V16, IDESC_PV, true);
+                        umma_commit_pair(&sm.v_empty[vslot], 0x3);
                     }
-                    umma_commit_pair(&sm.v_empty[vs], 0x3);
+                    __syncwarp();
+                    if (++vslot == VST) { vslot = 0; vpar ^= 1u; }
                 }
+                if (lane == 0) umma_commit_pair(&sm.pv_done[sb], 0x3);
                 __syncwarp();
             }
-            if (lane == 0) umma_commit_pair(&sm.pv_done, 0x3);
-            __syncwarp();
-            return true;
-        };
-        if (ok) ok = qk(0);
-        for (int u = 0; u < n_tiles && ok; ++u) {
-            if (u + 1 < n_tiles) ok = qk(u + 1);
-            if (ok) ok = pv(u);
         }
         if (lane == 0) umma_commit_pair(&sm.mma_done, 0x3);
         __syncwarp();
@@ -317,15 +380,20 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_const
             mx = fmaxf(mx, sm.red[L ^ 64]);
             const float m_new = fmaxf(m_run, mx);
             m_run = m_new;
-            // O is stable and P buffer s is free once the previous tile's P.V completed
-            if (u > 0 && ok) {
-                ok = mbar_wait(&sm.pv_done, (u - 1) & 1, WAIT_LIMIT);
+            // P buffer s is free once P.V of tile u-2 completed.  O must be stable
+            // (P.V of tile u-1 done) only when it is rescaled, which is rare.
+            if (u > 1 && ok) {
+                ok = mbar_wait(&sm.pv_done[s], ((u - 2) >> 1) & 1, WAIT_LIMIT);
                 if (!ok && sm.abort_flag == 0) set_abort(sm, p.status);
             }
-            tc_fence_after();
             if (m_new > -INFINITY && (m_ref == -INFINITY || m_new > m_ref + RESCALE_LOG2)) {
                 const float alpha = m_ref == -INFINITY ? 0.f : exp2f(m_ref - m_new);
                 if (u > 0) {
+                    if (ok) {
+                        ok = mbar_wait(&sm.pv_done[(u - 1) & 1], ((u - 1) >> 1) & 1, WAIT_LIMIT);
+                        if (!ok && sm.abort_flag == 0) set_abort(sm, p.status);
+                    }
+                    tc_fence_after();
 #pragma unroll 1
                     for (int q = 0; q < 8; ++q) {
                         uint32_t o[32];
@@ -364,7 +432,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_const
         }
         // ---- epilogue: wait for the last P.V, then write the partial
         if (n_tiles > 0 && ok) {
-            ok = mbar_wait(&sm.pv_done, (n_tiles - 1) & 1, WAIT_LIMIT);
+            ok = mbar_wait(&sm.pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, WAIT_LIMIT);
             if (!ok && sm.abort_flag == 0) set_abort(sm, p.status);
         }
         tc_fence_after();
@@ -457,8 +525,11 @@ int launch(const uint16_t *q, const uint16_t *kv_pool, int64_t k_stride, int64_t
            int table_stride, const int32_t *topk_idx, const int32_t *topk_count, int k, const int32_t *window_start,
            const int32_t *window_len, int B, float scale, int n_splits, float *o_part, float *m_part, float *l_part,
            int32_t *status, cudaStream_t stream) {
-    CUtensorMap kv_map, q_map;
-    if (!make_map(&kv_map, kv_pool, DQK, (uint64_t)n_slots * LSA_CHUNK, (uint64_t)k_stride * 2, 64, 1))
+    CUtensorMap kv_map, kv_map32, kv_map64, q_map;
+    const uint64_t pool_rows = (uint64_t)n_slots * LSA_CHUNK;
+    if (!make_map(&kv_map, kv_pool, DQK, pool_rows, (uint64_t)k_stride * 2, 64, 1) ||
+        !make_map(&kv_map32, kv_pool, DQK, pool_rows, (uint64_t)k_stride * 2, 64, 32) ||
+        !make_map(&kv_map64, kv_pool, DQK, pool_rows, (uint64_t)k_stride * 2, 64, 64))
         return fail(LSA_ERR_CUDA, "lsa_sparse_decode: cuTensorMapEncodeTiled failed for the KV pool");
     if (!make_map(&q_map, q, DQK, (uint64_t)B * HQ, DQK * 2, 64, 64))
         return fail(LSA_ERR_CUDA, "lsa_sparse_decode: cuTensorMapEncodeTiled failed for q");
@@ -482,7 +553,7 @@ int launch(const uint16_t *q, const uint16_t *kv_pool, int64_t k_stride, int64_t
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    LSA_CUDA(cudaLaunchKernelEx(&cfg, mla_decode_kernel, kv_map, q_map, prm));
+    LSA_CUDA(cudaLaunchKernelEx(&cfg, mla_decode_kernel, kv_map, kv_map32, kv_map64, q_map, prm));
     return LSA_OK;
 }
 

@@ -16,8 +16,8 @@ namespace lsa {
 constexpr int kTopkThreads = 1024;
 
 int launch_li_scores(const uint16_t *, const uint16_t *, const uint16_t *, int64_t, const int32_t *, int,
-                     const int32_t *, const int32_t *, int, const int32_t *, int, int, int, float *, int32_t *,
-                     cudaStream_t);
+                     const int32_t *, const int32_t *, int, const int32_t *, const int32_t *, int, int, int, float *,
+                     int32_t *, cudaStream_t);
 bool indexer_shape_ok(int H, int D);
 
 struct CandFromKept {   // candidate j -> token position kept[j / 64] * 64 + j % 64
@@ -28,14 +28,28 @@ struct CandIdentity {
     __device__ int operator()(int j) const { return j; }
 };
 
-__device__ __forceinline__ int cold_kept_count(const int32_t *kept, int count, int first_window_chunk) {
-    int lo = 0, hi = count;
-    while (lo < hi) {
-        int mid = (lo + hi) >> 1;
-        if (kept[mid] < first_window_chunk) lo = mid + 1;
-        else hi = mid;
+// grid B: cold[b] = number of kept chunks of sequence b that lie before its
+// recent window (they contribute the top-k candidates).  One coalesced pass
+// over the kept list, so the kernels that follow read a single count.
+__global__ void __launch_bounds__(256) cold_count_kernel(const int32_t *__restrict__ kept_idx,
+                                                         const int32_t *__restrict__ kept_count, int kept_cap,
+                                                         const int32_t *__restrict__ window_start,
+                                                         int32_t *__restrict__ cold) {
+    __shared__ int part[8];
+    const int b = blockIdx.x;
+    const int cnt = min(max(kept_count[b], 0), kept_cap);
+    const int fw = window_start[b] / LSA_CHUNK;
+    const int32_t *kept = kept_idx + (size_t)b * kept_cap;
+    int c = 0;
+    for (int i = threadIdx.x; i < cnt; i += 256) c += kept[i] < fw;
+    c = __reduce_add_sync(0xffffffffu, c);
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = c;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int t = 0;
+        for (int w = 0; w < 8; ++w) t += part[w];
+        cold[b] = t;
     }
-    return lo;
 }
 
 // Adds 1 to hist[bin] for every lane with `active`, one shared atomic per distinct bin.
@@ -131,14 +145,12 @@ __device__ __forceinline__ const float *stage_scores(const float *__restrict__ g
 
 __global__ void __launch_bounds__(kTopkThreads) topk_kept_kernel(const float *__restrict__ scores, int kept_cap,
                                                                  const int32_t *__restrict__ kept_idx,
-                                                                 const int32_t *__restrict__ kept_count,
-                                                                 const int32_t *__restrict__ window_start, int k,
+                                                                 const int32_t *__restrict__ cold, int k,
                                                                  int32_t *__restrict__ topk_idx,
                                                                  int32_t *__restrict__ topk_count, int stage_cap) {
     const int b = blockIdx.x;
     const int32_t *kept = kept_idx + (size_t)b * kept_cap;
-    const int cnt = min(kept_count[b], kept_cap);
-    const int n = cold_kept_count(kept, cnt, window_start[b] / LSA_CHUNK) * LSA_CHUNK;
+    const int n = cold[b] * LSA_CHUNK;
     const float *g = scores + (size_t)b * kept_cap * LSA_CHUNK;
     const float *s = n > k ? stage_scores(g, n, stage_cap) : g;
     topk_block(g, s, n, k, CandFromKept{kept}, topk_idx + (size_t)b * k, topk_count + b);
@@ -164,7 +176,10 @@ using namespace lsa;
 
 extern "C" size_t lsa_topk_workspace_size(int B, int kept_cap) {
     if (B <= 0 || kept_cap <= 0) return 0;
-    return align_up((size_t)B * kept_cap * LSA_CHUNK * sizeof(float), 256);
+    Carver c(nullptr);
+    c.take<int32_t>((size_t)B);                                   // kept cold chunk count per sequence
+    c.take<float>((size_t)B * kept_cap * LSA_CHUNK);             // candidate scores (unless the caller passes them)
+    return align_up(c.used, 256);
 }
 
 extern "C" int lsa_topk(const lsa_bf16 *q_li, const lsa_bf16 *w_li, const lsa_bf16 *li_pool, int64_t n_slots,
@@ -182,20 +197,23 @@ extern "C" int lsa_topk(const lsa_bf16 *q_li, const lsa_bf16 *w_li, const lsa_bf
                 "lsa_topk: unsupported Hl=%d dl=%d (dl in {64,128}, Hl multiple of 8 up to 128)", Hl, dl);
     LSA_REQUIRE(k >= 1 && k <= 65536, LSA_ERR_INVALID_ARG, "lsa_topk: k=%d outside [1, 65536]", k);
     LSA_REQUIRE((int64_t)kept_cap * LSA_CHUNK < (int64_t)1 << 31, LSA_ERR_INVALID_ARG, "lsa_topk: kept_cap too large");
-    float *buf = scores;
-    if (!buf) {
-        LSA_REQUIRE(ws && ws_bytes >= lsa_topk_workspace_size(B, kept_cap), LSA_ERR_WORKSPACE,
-                    "lsa_topk: workspace of %zu bytes, %zu needed", ws_bytes, lsa_topk_workspace_size(B, kept_cap));
-        buf = static_cast<float *>(ws);
-    }
-    int rc = launch_li_scores(q_li, w_li, li_pool, n_slots, chunk_table, table_stride, kept_idx, kept_count, kept_cap,
-                              window_start, B, Hl, dl, buf, dev_status, stream);
+    LSA_REQUIRE(ws && ws_bytes >= lsa_topk_workspace_size(B, kept_cap), LSA_ERR_WORKSPACE,
+                "lsa_topk: workspace of %zu bytes, %zu needed", ws_bytes, lsa_topk_workspace_size(B, kept_cap));
+    Carver c(ws);
+    int32_t *cold = c.take<int32_t>((size_t)B);
+    float *buf = c.take<float>((size_t)B * kept_cap * LSA_CHUNK);
+    if (scores) buf = scores;
+    cold_count_kernel<<<B, 256, 0, stream>>>(kept_idx, kept_count, kept_cap, window_start, cold);
+    int rc = check_launch("cold_count_kernel");
+    if (rc) return rc;
+    rc = launch_li_scores(q_li, w_li, li_pool, n_slots, chunk_table, table_stride, kept_idx, kept_count, kept_cap,
+                          window_start, cold, B, Hl, dl, buf, dev_status, stream);
     if (rc) return rc;
     const int cap = stage_capacity(kept_cap * LSA_CHUNK);
     LSA_CUDA(cudaFuncSetAttribute(topk_kept_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)(cap * sizeof(float))));
-    topk_kept_kernel<<<B, kTopkThreads, cap * sizeof(float), stream>>>(buf, kept_cap, kept_idx, kept_count,
-                                                                       window_start, k, topk_idx, topk_count, cap);
+    topk_kept_kernel<<<B, kTopkThreads, cap * sizeof(float), stream>>>(buf, kept_cap, kept_idx, cold, k, topk_idx,
+                                                                       topk_count, cap);
     return check_launch("topk_kept_kernel");
 }
 

@@ -76,6 +76,7 @@ class Window:
         self.ws_select = torch.empty(max(lsa.nmi_select_workspace_size(B, max_chunks_per_seq), 256),
                                      dtype=torch.uint8, device=d)
         self.scores = torch.empty(B, kept_cap * CHUNK, dtype=torch.float32, device=d)
+        self.ws_topk = torch.empty(max(lsa.topk_workspace_size(B, kept_cap), 256), dtype=torch.uint8, device=d)
         self.ws_decode = torch.empty(max(lsa.sparse_decode_workspace_size(B, shapes.Hq, shapes.dqk, shapes.dv,
                                                                           shapes.k, self.max_window_len), 256),
                                      dtype=torch.uint8, device=d)
@@ -118,7 +119,7 @@ class Window:
                          self.window_len, status=self.status)
         lsa.topk(t["q_li"][s], t["w_li"][s], t["li"], t["chunk_table"], self.kept_idx, self.kept_count,
                  t["window_start"], sh.k, scores=self.scores, status=self.status, topk_idx=self.topk_idx[s],
-                 topk_count=self.topk_count[s])
+                 topk_count=self.topk_count[s], ws=self.ws_topk)
         lsa.sparse_decode(t["q"][s], self.k_pool, self.v_pool, t["chunk_table"], self.topk_idx[s],
                           self.topk_count[s], t["window_start"], self.window_len, self.max_window_len, sh.dv,
                           sh.scale, out=self.out[s], lse=self.lse[s], status=self.status, ws=self.ws_decode)
@@ -159,8 +160,8 @@ class Window:
             self.steps()
 
     def launches_per_window(self) -> int:
-        """Kernels this library launches per window (select: 2; per step: append 1, top-k 2, decode 2)."""
-        return 2 + self.s.steps * 5
+        """Kernels this library launches per window (select: 2; per step: append 1, top-k 3, decode 2)."""
+        return 2 + self.s.steps * 6
 
     def device_status(self) -> int:
         return int(self.status.item())

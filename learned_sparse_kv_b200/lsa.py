@@ -135,11 +135,11 @@ def topk(q_li, w_li, li_pool, chunk_table, kept_idx, kept_count, window_start, k
         topk_idx = torch.empty(B, k, dtype=torch.int32, device=dev)
     if topk_count is None:
         topk_count = torch.empty(B, dtype=torch.int32, device=dev)
-    ws = _ws(topk_workspace_size(B, kept_cap), dev, ws) if scores is None else None
+    ws = _ws(topk_workspace_size(B, kept_cap), dev, ws)
     _check(_lib.lsa_topk(_ptr(q_li), _ptr(w_li), _ptr(li_pool), li_pool.shape[0], _ptr(chunk_table),
                          chunk_table.shape[1], _ptr(kept_idx), _ptr(kept_count), kept_cap, _ptr(window_start),
                          B, Hl, dl, k, _ptr(topk_idx), _ptr(topk_count), _ptr(scores), _ptr(status), _ptr(ws),
-                         0 if ws is None else ws.numel(), _stream(stream)))
+                         ws.numel(), _stream(stream)))
     return topk_idx, topk_count
 
 

@@ -95,5 +95,5 @@ def test_workspace_queries_are_host_only(lib):
     lib.lsa_topk_workspace_size.restype = ctypes.c_size_t
     lib.lsa_nmi_select_workspace_size.restype = ctypes.c_size_t
     assert lib.lsa_label_vote_workspace_size(32, 64, 2048) == 64 * 2048 * 4
-    assert lib.lsa_topk_workspace_size(8, 2048) == 8 * 2048 * 64 * 4
+    assert lib.lsa_topk_workspace_size(8, 2048) >= 8 * 2048 * 64 * 4 + 8 * 4
     assert lib.lsa_nmi_select_workspace_size(8, 2048) >= 8 * 32 * 8
