@@ -27,7 +27,6 @@ using namespace sm100;
 constexpr int THREADS = 192;
 constexpr int STAGES = 3;
 constexpr int MAX_H = 128, MAX_D = 128;
-constexpr uint32_t WAIT_LIMIT = 1u << 22;
 
 struct __align__(1024) Smem {
     uint8_t keys[STAGES][MAX_D / 64][128 * 128];   // [atom][128 token rows][128 B]
@@ -105,7 +104,7 @@ __device__ __forceinline__ int tile_seq(const Work &wk, int B, int t) {
 
 __device__ __forceinline__ bool bounded(Smem &sm, const uint64_t *bar, uint32_t parity, int32_t *status) {
     if (sm.abort_flag) return false;
-    if (mbar_wait(bar, parity, WAIT_LIMIT)) return true;
+    if (mbar_wait(bar, parity, WAIT_NS)) return true;
     sm.abort_flag = 1;
     flag(status, LSA_DEV_TIMEOUT);
     return false;
@@ -213,7 +212,7 @@ li_score_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_consta
         if (cur_b >= 0 && lane == 0) commit(&sm.q_empty[qbuf]);
         if (lane == 0) {                                   // every MMA has completed before TMEM is released
             commit(&sm.mma_done);
-            if (!mbar_wait(&sm.mma_done, 0, WAIT_LIMIT)) flag(p.status, LSA_DEV_TIMEOUT);
+            if (!mbar_wait(&sm.mma_done, 0, WAIT_NS)) flag(p.status, LSA_DEV_TIMEOUT);
         }
         __syncwarp();
     } else {

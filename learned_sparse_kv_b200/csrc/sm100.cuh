@@ -56,13 +56,59 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
     return ok != 0;
 }
 
-// Waits for the phase with the given parity to complete; gives up after
-// `limit` polls (each try_wait itself suspends for a while) and returns false.
-__device__ __forceinline__ bool mbar_wait(const uint64_t *bar, uint32_t parity, uint32_t limit) {
+// Acquire at cluster scope: for phases completed by generic stores of the peer
+// CTA (released with mbar_arrive_release_cluster).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t addr, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ void mbar_arrive_local(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
+    return t;
+}
+
+// Every wait on an mbarrier gives up after this long (the phases it waits for
+// complete within microseconds when the pipeline is healthy).
+constexpr uint64_t WAIT_NS = 1000000000ull;
+
+// Waits for the phase with the given parity to complete; returns false once
+// `limit_ns` nanoseconds have passed without it (each try_wait may itself
+// suspend the thread for a while, so the bound is taken on the clock).
+__device__ __forceinline__ bool mbar_wait(const uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
     const uint32_t a = smem_addr(bar);
-    for (uint32_t i = 0; i < limit; ++i)
+    if (mbar_try_wait(a, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (;;) {
         if (mbar_try_wait(a, parity)) return true;
-    return false;
+        if (global_ns() - t0 > limit_ns) return false;
+    }
+}
+
+__device__ __forceinline__ bool mbar_wait_cluster(const uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+    const uint32_t a = smem_addr(bar);
+    if (mbar_try_wait_cluster(a, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (;;) {
+        if (mbar_try_wait_cluster(a, parity)) return true;
+        if (global_ns() - t0 > limit_ns) return false;
+    }
 }
 
 // ------------------------------------------------------------- cluster ----
@@ -85,6 +131,26 @@ __device__ __forceinline__ void named_barrier(int id, int count) {
     asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(count) : "memory");
 }
 
+// Named barrier that also returns the AND of `pred` over the participating threads.
+__device__ __forceinline__ bool named_barrier_and(int id, int count, bool pred) {
+    uint32_t out;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %3, 0;\n\t"
+        "bar.red.and.pred q, %1, %2, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}\n"
+        : "=r"(out)
+        : "r"(id), "r"(count), "r"(uint32_t(pred))
+        : "memory");
+    return out != 0;
+}
+
+// 16-byte global -> shared copy (L2 only); src_bytes = 0 writes zeros and reads nothing.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+// (cp_async_commit / cp_async_wait<N> come from common.cuh)
+
 // ---------------------------------------------------------------- TMA -----
 
 // 2D tile load of box at (x, y) into this CTA's shared memory; completion is
@@ -94,6 +160,23 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.cta_group::2"
         " [%0], [%1, {%2, %3}], [%4];\n" ::"r"(smem_addr(dst)),
         "l"(map), "r"(x), "r"(y), "r"(mbar_cluster)
+        : "memory");
+}
+
+// 3D / 4D boxes, same completion rule.
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int x, int y, int z, uint32_t mbar_cluster) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.cta_group::2"
+        " [%0], [%1, {%2, %3, %4}], [%5];\n" ::"r"(smem_addr(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(z), "r"(mbar_cluster)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, int x, int y, int z, int w,
+                                            uint32_t mbar_cluster) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.cta_group::2"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];\n" ::"r"(smem_addr(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(z), "r"(w), "r"(mbar_cluster)
         : "memory");
 }
 

@@ -9,15 +9,27 @@
 // 64r..64r+63 of Q and of P in its shared memory, the B operand is split by
 // N between the pair, and each CTA's tensor memory receives its own heads'
 // rows of the result.
-//   S = Q K^T   N = 64 kv rows per tile (each CTA loads 32 rows x 576 columns)
-//   O += P V    N = 256 value columns per MMA, two MMAs per tile (each CTA
-//               loads all 64 rows x its 2 x 128 value columns)
+//   S = Q K^T   N = 64 kv rows per tile (CTA r holds rows 32r..32r+31, all 576 columns)
+//   O += P V    N = 256 value columns per MMA (CTA r holds all 64 rows of value
+//               columns 128r..128r+127 and 256+128r..); P is passed as the sum
+//               of two bf16 parts, hi = bf16(P) and lo = bf16(P - hi), so every
+//               K step takes four MMAs and P keeps ~16 bits of precision
 // TMEM per CTA: two S buffers of 32 columns and O = 64 heads x 512 values in
-// 256 columns.  Rows are gathered by TMA tile::gather4 (4 rows per load,
-// 128-byte swizzle) through the chunk table.  Warp roles:
-//   0  K producer + tile-validity masks      1  V producer
-//   2  MMA issuer (even CTA only)            3  TMEM allocator
-//   4..7  softmax, O rescale, epilogue (one thread per TMEM lane)
+// 256 columns.
+//
+// Loading a tile is one operation per operand wherever the rows are a whole
+// chunk slot of the pool: a 3D TMA box {64 columns, 32 rows, 9 column chunks}
+// fetches a CTA's K rows (36 KB) and a 4D box {64, 64 rows, 2, 2} its value
+// columns (32 KB), both straight into the 128-byte-swizzled operand layout.
+// Gathered tiles (top-k rows, and window tiles that are not a whole aligned
+// chunk) are copied by a warpgroup with 16-byte cp.async into the same layout;
+// missing rows are zero-filled.  Two stages of each operand are in flight.
+// Warp roles:
+//   0      TMA producer, tile-validity masks
+//   1      S = Q K^T issuer (even CTA)        2   O += P V issuer (even CTA)
+//   3      TMEM allocator
+//   4..7   softmax, O rescale, epilogue (one thread per TMEM lane)
+//   8..11  row gather for gathered tiles
 // The online softmax is evaluated in the log2 domain; the reference maximum
 // is only moved when a row maximum grows by more than 2^8, which keeps P <= 256
 // in bf16 and makes O rescales rare.  Every mbarrier wait is bounded: on
@@ -37,12 +49,14 @@ constexpr int HQ = 128;           // heads per cluster
 constexpr int DQK = 576, DV = 512;
 constexpr int NTILE = 64;         // kv rows per tile
 constexpr int KCH = DQK / 64;     // 9 column chunks of 64
-constexpr int KST = 16;           // K ring: [32 rows x 64 cols] stages
-constexpr int VST = 4;            // V ring: [2 atoms][64 rows][64 cols] stages
+constexpr int STAGES = 2;         // tiles in flight per operand
 constexpr int INFO = 4;           // tile-validity ring
-constexpr int THREADS = 256;
+constexpr int THREADS = 384;
+constexpr int GATHER_THREADS = 128;
+constexpr uint32_t Q_BYTES = KCH * HPC * 128;          // per CTA
+constexpr uint32_t K_BYTES = KCH * 32 * 128;           // per CTA and tile
+constexpr uint32_t V_BYTES = 2 * 2 * NTILE * 128;      // per CTA and tile
 constexpr float RESCALE_LOG2 = 8.f;
-constexpr uint32_t WAIT_LIMIT = 1u << 22;   // polls before a wait gives up (~seconds)
 
 // TMEM columns
 constexpr uint32_t TM_S = 0;      // S buffers at 0 and 32
@@ -50,21 +64,24 @@ constexpr uint32_t TM_O = 64;     // O at 64..319
 constexpr uint32_t TM_COLS = 512;
 
 struct __align__(1024) Smem {
-    uint8_t q[KCH][HPC * 128];          // 9 x [64 heads][128 B], 128B-swizzled, K-major
-    uint8_t k[KST][32 * 128];           // [32 kv rows][64 cols]
-    uint8_t v[VST][2][NTILE * 128];     // [value atom][64 kv rows][64 value cols], MN-major
-    uint8_t p[2][HPC * 128];            // [64 heads][64 kv], K-major
-    uint64_t k_full[KST], k_empty[KST];
-    uint64_t v_full[VST], v_empty[VST];
+    uint8_t q[KCH][HPC * 128];                 // 9 x [64 heads][128 B], 128B-swizzled, K-major
+    uint8_t k[STAGES][KCH][32 * 128];          // [chunk][32 kv rows][64 cols]
+    uint8_t v[STAGES][2][2][NTILE * 128];      // [value block j][atom][64 kv rows][64 value cols], MN-major
+    uint8_t p[2][HPC * 128];                   // P = hi + lo: [part][64 heads][64 kv], K-major
+    uint64_t k_full[STAGES], k_empty[STAGES];
+    uint64_t v_full[STAGES], v_empty[STAGES];
+    uint64_t k_go[2], v_go[2];       // producer -> gather: stage free for the n-th gathered tile
     uint64_t q_full;
     uint64_t s_full[2], s_empty[2], p_full[2];
-    uint64_t pv_done[2], mma_done;   // pv_done[s]: P.V of the tiles using P buffer s
+    uint64_t pv_done[2], mma_done;   // pv_done[u & 1]: P.V of tile u
     uint64_t info_full[INFO], info_empty[INFO];
     unsigned long long info_mask[INFO];
+    int32_t grow[STAGES][NTILE];     // pool rows of a gathered tile (-1: zero row)
     float red[128];
     uint32_t tmem_base;
     int abort_flag;
 };
+static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory of one CTA");
 
 struct Params {
     const int32_t *table;
@@ -72,6 +89,8 @@ struct Params {
     const int32_t *topk_count;
     const int32_t *window_start;
     const int32_t *window_len;
+    const uint8_t *pool;       // KV pool base (bytes)
+    int64_t row_bytes;         // pool row stride in bytes
     float *o_part, *m_part, *l_part;
     int32_t *status;
     int64_t n_rows_pool;   // n_slots * 64
@@ -82,26 +101,31 @@ struct Params {
 // Tiles of one sequence: ceil(tk/64) top-k tiles, then the window chunk by chunk.
 struct SeqTiles {
     int tk, wstart, wlen, t_topk, total;
+    bool aligned;
     __device__ SeqTiles(const Params &p, int b) {
         tk = min(max(p.topk_count[b], 0), p.k);
         wstart = p.window_start[b];
         wlen = max(p.window_len[b], 0);
         t_topk = (tk + NTILE - 1) / NTILE;
         total = t_topk + (wlen + NTILE - 1) / NTILE;
+        aligned = (wstart & (NTILE - 1)) == 0;
     }
-    // Window tile t (t >= t_topk) covers one whole chunk slot: first pool row of
-    // the slot (-2 if the chunk has no slot) and the number of valid rows.
-    __device__ int64_t window_slot_row(const Params &p, int b, int t, int *n_valid) const {
-        const int j = t - t_topk;
-        *n_valid = min(NTILE, wlen - NTILE * j);
-        const int chunk = (wstart >> 6) + j;
+    // Top-k tiles, and window tiles that are not one whole chunk slot, are gathered row by row.
+    __device__ bool gathered(int t) const {
+        if (t < t_topk) return true;
+        return !aligned || wlen - NTILE * (t - t_topk) < NTILE;
+    }
+    // Window tile t (t >= t_topk, aligned window) covers one whole chunk slot:
+    // its first pool row, or -2 if the chunk has no slot.
+    __device__ int64_t window_slot_row(const Params &p, int b, int t) const {
+        const int chunk = (wstart >> 6) + (t - t_topk);
         if (wstart < 0 || chunk >= p.table_stride) return -2;
         const int slot = p.table[(size_t)b * p.table_stride + chunk];
         const int64_t g = (int64_t)slot * LSA_CHUNK;
         if (slot < 0 || g >= p.n_rows_pool) return -2;
         return g;
     }
-    // Global pool row of row i (0..63) of tile t, or -1.
+    // Global pool row of row i (0..63) of tile t, -1 past the end of the row set, -2 if unmapped.
     __device__ int64_t row(const Params &p, int b, int t, int i) const {
         int pos;
         if (t < t_topk) {
@@ -132,16 +156,40 @@ __device__ __forceinline__ void set_abort(Smem &sm, int32_t *status) {
 __device__ __forceinline__ bool warp_wait(Smem &sm, const uint64_t *bar, uint32_t parity, int32_t *status) {
     bool ok = true;
     if ((threadIdx.x & 31) == 0) {
-        ok = sm.abort_flag == 0 && mbar_wait(bar, parity, WAIT_LIMIT);
+        ok = sm.abort_flag == 0 && mbar_wait(bar, parity, WAIT_NS);
         if (!ok) set_abort(sm, status);
     }
     return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
+// Same, acquiring at cluster scope (phases that the peer CTA's generic stores complete).
+__device__ __forceinline__ bool warp_wait_cluster(Smem &sm, const uint64_t *bar, uint32_t parity, int32_t *status) {
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) {
+        ok = sm.abort_flag == 0 && mbar_wait_cluster(bar, parity, WAIT_NS);
+        if (!ok) set_abort(sm, status);
+    }
+    return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
+// Gather-warpgroup-uniform bounded wait: one thread polls, the group agrees by barrier reduction.
+__device__ __forceinline__ bool group_wait(Smem &sm, const uint64_t *bar, uint32_t parity, int32_t *status, int g) {
+    bool ok = true;
+    if (g == 0) {
+        ok = sm.abort_flag == 0 && mbar_wait(bar, parity, WAIT_NS);
+        if (!ok) set_abort(sm, status);
+    }
+    return named_barrier_and(2, GATHER_THREADS, ok);
+}
+
+__device__ __forceinline__ int32_t gather_row(const SeqTiles &st, const Params &p, int b, int t, int i) {
+    const int64_t g = st.row(p, b, t, i);
+    return g >= 0 ? (int32_t)g : -1;
+}
+
 __global__ void __launch_bounds__(THREADS, 1)
-mla_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_constant__ CUtensorMap kv_map32,
-                  const __grid_constant__ CUtensorMap kv_map64, const __grid_constant__ CUtensorMap q_map,
-                  const Params p) {
+mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap v_map,
+                  const __grid_constant__ CUtensorMap q_map, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>(smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -149,13 +197,16 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_const
     const int split = blockIdx.x >> 1, b = blockIdx.y;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < KST; ++i) { mbar_init(&sm.k_full[i], 2); mbar_init(&sm.k_empty[i], 1); }
-        for (int i = 0; i < VST; ++i) { mbar_init(&sm.v_full[i], 2); mbar_init(&sm.v_empty[i], 1); }
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(&sm.k_full[i], 2); mbar_init(&sm.k_empty[i], 1);
+            mbar_init(&sm.v_full[i], 2); mbar_init(&sm.v_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) { mbar_init(&sm.k_go[i], 1); mbar_init(&sm.v_go[i], 1); }
         mbar_init(&sm.q_full, 2);
         for (int i = 0; i < 2; ++i) { mbar_init(&sm.s_full[i], 1); mbar_init(&sm.s_empty[i], 2); mbar_init(&sm.p_full[i], 2); }
         mbar_init(&sm.pv_done[0], 1);
         mbar_init(&sm.pv_done[1], 1);
-        mbar_init(&sm.mma_done, 1);
+        mbar_init(&sm.mma_done, 2);   // one commit from each MMA issuer
         for (int i = 0; i < INFO; ++i) { mbar_init(&sm.info_full[i], 1); mbar_init(&sm.info_empty[i], 1); }
         sm.abort_flag = 0;
         fence_mbar_init_cluster();
@@ -175,31 +226,30 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_const
     const int u0 = split, ustride = p.n_splits;
 
     if (warp == 0 && n_tiles > 0) {
-        // ------------------------------------------------ K producer + Q
+        // ------------------------------------------------ TMA producer + tile masks
         if (lane == 0) {
             const uint32_t qf = map_to_rank(&sm.q_full, 0);
-            mbar_arrive_expect_tx_cluster(qf, KCH * HPC * 128);
-            for (int c = 0; c < KCH; ++c) tma_load_2d(sm.q[c], &q_map, 64 * c, b * HQ + HPC * (int)rank, qf);
+            mbar_arrive_expect_tx_cluster(qf, Q_BYTES);
+            tma_load_3d(sm.q[0], &q_map, 0, b * HQ + HPC * (int)rank, 0, qf);
         }
-        uint32_t kc = 0;
-        // row indices of the next top-k tile are loaded while the current tile is issued
+        // row indices of the next gathered tile are loaded while the current tile is issued
         int64_t n0 = -1, n1 = -1;
-        if (u0 < st.t_topk) { n0 = st.row(p, b, u0, lane); n1 = st.row(p, b, u0, lane + 32); }
+        if (st.gathered(u0)) { n0 = st.row(p, b, u0, lane); n1 = st.row(p, b, u0, lane + 32); }
+        int gi = 0;   // gathered tiles handed to the gather warpgroup so far
         for (int u = 0; u < n_tiles; ++u) {
             const int t = u0 + u * ustride;
-            const bool window = t >= st.t_topk;
+            const bool gath = st.gathered(t);
             const int64_t g0 = n0, g1 = n1;
-            if (u + 1 < n_tiles && t + ustride < st.t_topk) {
+            if (u + 1 < n_tiles && st.gathered(t + ustride)) {
                 n0 = st.row(p, b, t + ustride, lane);
                 n1 = st.row(p, b, t + ustride, lane + 32);
             }
             unsigned long long mask;
-            int64_t slot_row = -1;
-            if (window) {
-                int nv;
-                slot_row = st.window_slot_row(p, b, t, &nv);
+            int64_t slot_row = -2;
+            if (!gath) {
+                slot_row = st.window_slot_row(p, b, t);
                 if (slot_row == -2) flag(p.status, LSA_DEV_TABLE);
-                mask = slot_row < 0 ? 0ull : (nv >= 64 ? ~0ull : ((1ull << nv) - 1ull));
+                mask = slot_row < 0 ? 0ull : ~0ull;
             } else {
                 if ((g0 == -2 || g1 == -2)) flag(p.status, LSA_DEV_TABLE);
                 const unsigned lo = __ballot_sync(0xffffffffu, g0 >= 0), hi = __ballot_sync(0xffffffffu, g1 >= 0);
@@ -210,141 +260,179 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_const
                 sm.info_mask[u % INFO] = mask;
                 asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];\n" ::"r"(smem_addr(&sm.info_full[u % INFO])) : "memory");
             }
-            const int64_t mine = rank ? g1 : g0;
-            const int gr = mine >= 0 ? (int)mine : (int)p.n_rows_pool;   // out of range -> zero fill
-            const int r0 = __shfl_sync(0xffffffffu, gr, (4 * lane) & 31), r1 = __shfl_sync(0xffffffffu, gr, (4 * lane + 1) & 31);
-            const int r2 = __shfl_sync(0xffffffffu, gr, (4 * lane + 2) & 31), r3 = __shfl_sync(0xffffffffu, gr, (4 * lane + 3) & 31);
-            const int wy = slot_row >= 0 ? (int)slot_row + 32 * (int)rank : (int)p.n_rows_pool;
-            bool ok = true;
-            for (int c = 0; c < KCH; ++c, ++kc) {
-                const int s = kc % KST;
-                ok = warp_wait(sm, &sm.k_empty[s], ((kc / KST) + 1) & 1, p.status);
-                if (!ok) break;
-                const uint32_t full = map_to_rank(&sm.k_full[s], 0);
-                if (lane == 0) {
-                    mbar_arrive_expect_tx_cluster(full, 32 * 128);
-                    if (window) tma_load_2d(sm.k[s], &kv_map32, 64 * c, wy, full);
+            // Every tile's stage is waited for here, in tile order: a parity wait is only
+            // unambiguous one phase behind the barrier, so the gather warpgroup (which
+            // skips the TMA tiles) is handed its stages through k_go / v_go, whose
+            // phases count gathered tiles only.
+            const int s = u & 1;
+            const uint32_t par = ((u >> 1) + 1) & 1;
+            // an unmapped slot is read out of range: TMA fills zeros
+            const int wy = slot_row >= 0 ? (int)slot_row : (int)p.n_rows_pool;
+            if (!warp_wait(sm, &sm.k_empty[s], par, p.status)) break;
+            if (lane == 0) {
+                if (gath) {
+                    mbar_arrive_local(&sm.k_go[gi & 1]);
+                } else {
+                    const uint32_t full = map_to_rank(&sm.k_full[s], 0);
+                    mbar_arrive_expect_tx_cluster(full, K_BYTES);
+                    tma_load_3d(sm.k[s][0], &k_map, 0, wy + 32 * (int)rank, 0, full);
                 }
-                __syncwarp();
-                if (!window && lane < 8) tma_gather4(sm.k[s] + lane * 512, &kv_map, 64 * c, r0, r1, r2, r3, full);
             }
-            if (!ok) break;
-        }
-    } else if (warp == 1 && n_tiles > 0) {
-        // ------------------------------------------------ V producer
-        uint32_t vc = 0;
-        int64_t n0 = -1, n1 = -1;
-        if (u0 < st.t_topk) { n0 = st.row(p, b, u0, lane); n1 = st.row(p, b, u0, lane + 32); }
-        for (int u = 0; u < n_tiles; ++u) {
-            const int t = u0 + u * ustride;
-            const bool window = t >= st.t_topk;
-            const int64_t g0 = n0, g1 = n1;
-            if (u + 1 < n_tiles && t + ustride < st.t_topk) {
-                n0 = st.row(p, b, t + ustride, lane);
-                n1 = st.row(p, b, t + ustride, lane + 32);
-            }
-            int wy = (int)p.n_rows_pool;
-            if (window) {
-                int nv;
-                const int64_t sr = st.window_slot_row(p, b, t, &nv);
-                if (sr >= 0) wy = (int)sr;
-            }
-            const int a0 = g0 >= 0 ? (int)g0 : (int)p.n_rows_pool, a1 = g1 >= 0 ? (int)g1 : (int)p.n_rows_pool;
-            // lane -> (value atom a = lane / 16, row group gq = lane % 16: rows 4gq .. 4gq + 3)
-            const int gq = lane & 15, a = lane >> 4;
-            int r[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int row = 4 * gq + i;
-                const int x0 = __shfl_sync(0xffffffffu, a0, row & 31), x1 = __shfl_sync(0xffffffffu, a1, row & 31);
-                r[i] = row < 32 ? x0 : x1;
-            }
-            bool ok = true;
-            for (int j = 0; j < 2 && ok; ++j, ++vc) {
-                const int s = vc % VST;
-                ok = warp_wait(sm, &sm.v_empty[s], ((vc / VST) + 1) & 1, p.status);
-                if (!ok) break;
-                const uint32_t full = map_to_rank(&sm.v_full[s], 0);
-                const int col0 = 256 * j + 128 * (int)rank;
-                if (lane == 0) {
-                    mbar_arrive_expect_tx_cluster(full, 2 * NTILE * 128);
-                    if (window) {
-                        tma_load_2d(sm.v[s][0], &kv_map64, col0, wy, full);
-                        tma_load_2d(sm.v[s][1], &kv_map64, col0 + 64, wy, full);
-                    }
+            if (!warp_wait(sm, &sm.v_empty[s], par, p.status)) break;
+            if (lane == 0) {
+                if (gath) {
+                    mbar_arrive_local(&sm.v_go[gi & 1]);
+                } else {
+                    const uint32_t full = map_to_rank(&sm.v_full[s], 0);
+                    mbar_arrive_expect_tx_cluster(full, V_BYTES);
+                    tma_load_4d(sm.v[s][0][0], &v_map, 0, wy, 2 * (int)rank, 0, full);
                 }
-                __syncwarp();
-                if (!window) tma_gather4(sm.v[s][a] + gq * 512, &kv_map, col0 + 64 * a, r[0], r[1], r[2], r[3], full);
             }
-            if (!ok) break;
+            gi += gath ? 1 : 0;
+            __syncwarp();
         }
-    } else if (warp == 2 && rank == 0 && n_tiles > 0) {
-        // ------------------------------------------------ MMA issuer (even CTA)
+    } else if ((warp == 1 || warp == 2) && rank == 0 && n_tiles > 0) {
+        // ------------------------------------------------ MMA issuers (even CTA)
+        // Warp 1 issues S = Q K^T, warp 2 issues O += P V.  Each commits only its
+        // own MMAs, so neither chain waits behind the other's operands.
         // Descriptors are built once; a byte offset o within shared memory is
         // o >> 4 added to the descriptor's start-address field.
         constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, NTILE, false, false);
         constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 256, false, true);
-        const uint64_t qd0 = smem_desc_sw128(smem_addr(sm.q[0]), 16, 1024);
-        const uint64_t kd0 = smem_desc_sw128(smem_addr(sm.k[0]), 16, 1024);
-        const uint64_t pd0 = smem_desc_sw128(smem_addr(sm.p[0]), 16, 1024);
-        const uint64_t vd0 = smem_desc_sw128(smem_addr(sm.v[0][0]), NTILE * 128, 1024);
-        constexpr uint64_t Q_CHUNK = (HPC * 128) >> 4, K_STAGE = (32 * 128) >> 4, P_BUF = (HPC * 128) >> 4;
-        constexpr uint64_t V_STAGE = (2 * NTILE * 128) >> 4, K16 = 32 >> 4, V16 = (16 * 128) >> 4;
-        bool ok = warp_wait(sm, &sm.q_full, 0, p.status);
-        int kslot = 0, vslot = 0;
-        uint32_t kpar = 0, vpar = 0;
-        for (int u = -1; u < n_tiles && ok; ++u) {
-            if (u + 1 < n_tiles) {                         // S(u+1) = Q K^T
-                const int t = u + 1, sb = t & 1;
-                ok = warp_wait(sm, &sm.s_empty[sb], ((t >> 1) + 1) & 1, p.status);
+        constexpr uint64_t K16 = 32 >> 4;
+        bool ok = true;
+        if (warp == 1) {
+            constexpr uint64_t Q_CHUNK = (HPC * 128) >> 4, K_CHUNK = (32 * 128) >> 4, K_STAGE = K_BYTES >> 4;
+            const uint64_t qd0 = smem_desc_sw128(smem_addr(sm.q[0]), 16, 1024);
+            const uint64_t kd0 = smem_desc_sw128(smem_addr(sm.k[0][0]), 16, 1024);
+            ok = warp_wait(sm, &sm.q_full, 0, p.status);
+            for (int u = 0; u < n_tiles && ok; ++u) {      // S(u) = Q K^T
+                const int sb = u & 1;
+                ok = warp_wait(sm, &sm.s_empty[sb], ((u >> 1) + 1) & 1, p.status) &&
+                     warp_wait_cluster(sm, &sm.k_full[sb], (u >> 1) & 1, p.status);
+                if (!ok) break;
                 tc_fence_after();
-                const uint32_t d = tmem + TM_S + 32 * sb;
-                for (int c = 0; c < KCH && ok; ++c) {
-                    ok = warp_wait(sm, &sm.k_full[kslot], kpar, p.status);
-                    if (!ok) break;
-                    tc_fence_after();
-                    if (lane == 0) {
-                        const uint64_t a = qd0 + Q_CHUNK * c, bb = kd0 + K_STAGE * kslot;
-                        umma_pair_ss(d, a, bb, IDESC_QK, c != 0);
-                        umma_pair_ss(d, a + K16, bb + K16, IDESC_QK, true);
-                        umma_pair_ss(d, a + 2 * K16, bb + 2 * K16, IDESC_QK, true);
-                        umma_pair_ss(d, a + 3 * K16, bb + 3 * K16, IDESC_QK, true);
-                        umma_commit_pair(&sm.k_empty[kslot], 0x3);
-                    }
-                    __syncwarp();
-                    if (++kslot == KST) { kslot = 0; kpar ^= 1u; }
+                if (lane == 0) {
+                    const uint32_t d = tmem + TM_S + 32 * sb;
+                    const uint64_t kb = kd0 + K_STAGE * sb;
+#pragma unroll
+                    for (int c = 0; c < KCH; ++c)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_pair_ss(d, qd0 + Q_CHUNK * c + K16 * kk, kb + K_CHUNK * c + K16 * kk, IDESC_QK,
+                                         (c | kk) != 0);
+                    umma_commit_pair(&sm.k_empty[sb], 0x3);
+                    umma_commit_pair(&sm.s_full[sb], 0x3);
                 }
-                if (lane == 0) umma_commit_pair(&sm.s_full[sb], 0x3);
                 __syncwarp();
             }
-            if (u >= 0 && ok) {                            // O += P V for tile u
+        } else {
+            constexpr uint64_t P_BUF = (HPC * 128) >> 4, V_STAGE = V_BYTES >> 4, V_J = (2 * NTILE * 128) >> 4;
+            constexpr uint64_t V16 = (16 * 128) >> 4;
+            const uint64_t pd0 = smem_desc_sw128(smem_addr(sm.p[0]), 16, 1024);
+            const uint64_t vd0 = smem_desc_sw128(smem_addr(sm.v[0][0][0]), NTILE * 128, 1024);
+            for (int u = 0; u < n_tiles && ok; ++u) {      // O += P V for tile u
                 const int sb = u & 1;
-                ok = warp_wait(sm, &sm.p_full[sb], (u >> 1) & 1, p.status);
+                ok = warp_wait(sm, &sm.p_full[sb], (u >> 1) & 1, p.status) &&
+                     warp_wait_cluster(sm, &sm.v_full[sb], (u >> 1) & 1, p.status);
+                if (!ok) break;
                 tc_fence_after();
-                const uint64_t a = pd0 + P_BUF * sb;
-                for (int j = 0; j < 2 && ok; ++j) {
-                    ok = warp_wait(sm, &sm.v_full[vslot], vpar, p.status);
-                    if (!ok) break;
-                    tc_fence_after();
-                    if (lane == 0) {
-                        const uint64_t bb = vd0 + V_STAGE * vslot;
-                        const uint32_t d = tmem + TM_O + 128 * j;
-                        umma_pair_ss(d, a, bb, IDESC_PV, u != 0);
-                        umma_pair_ss(d, a + K16, bb + V16, IDESC_PV, true);
-                        umma_pair_ss(d, a + 2 * K16, bb + 2 * V16, IDESC_PV, true);
-                        umma_pair_ss(d, a + 3 * K16, bb + 3 * V16, IDESC_PV, true);
-                        umma_commit_pair(&sm.v_empty[vslot], 0x3);
-                    }
-                    __syncwarp();
-                    if (++vslot == VST) { vslot = 0; vpar ^= 1u; }
+                if (lane == 0) {
+                    const uint64_t vb = vd0 + V_STAGE * sb;
+#pragma unroll
+                    for (int j = 0; j < 2; ++j)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint64_t b = vb + V_J * j + V16 * kk;
+                            umma_pair_ss(tmem + TM_O + 128 * j, pd0 + K16 * kk, b, IDESC_PV, u > 0 || kk > 0);
+                            umma_pair_ss(tmem + TM_O + 128 * j, pd0 + P_BUF + K16 * kk, b, IDESC_PV, true);
+                        }
+                    umma_commit_pair(&sm.v_empty[sb], 0x3);
+                    umma_commit_pair(&sm.pv_done[sb], 0x3);
                 }
-                if (lane == 0) umma_commit_pair(&sm.pv_done[sb], 0x3);
                 __syncwarp();
             }
         }
         if (lane == 0) umma_commit_pair(&sm.mma_done, 0x3);
         __syncwarp();
-    } else if (warp >= 4) {
+    } else if (warp >= 8 && n_tiles > 0) {
+        // ------------------------------------------------ row gather (cp.async)
+        // Thread g copies 16-byte pieces: K pieces q = g + 128 i of the CTA's 32
+        // rows x 72 pieces, V pieces of 64 rows x 4 value atoms x 8 pieces.  A
+        // tile is signalled once its copies (and those of the tile before) have
+        // landed: after the next tile's K copies are issued when the next
+        // gathered tile follows directly, else at once.
+        const int g = threadIdx.x - 256;
+        auto next_gathered = [&](int u) {
+            for (; u < n_tiles; ++u)
+                if (st.gathered(u0 + u * ustride)) return u;
+            return n_tiles;
+        };
+        auto signal = [&](int s) {
+            cp_async_wait<0>();
+            fence_proxy_async_smem();
+            named_barrier(2, GATHER_THREADS);
+            if (g == 0) {
+                mbar_arrive_release_cluster(map_to_rank(&sm.k_full[s], 0));
+                mbar_arrive_release_cluster(map_to_rank(&sm.v_full[s], 0));
+            }
+        };
+        int u = next_gathered(0);
+        int32_t nxt = (u < n_tiles && g < NTILE) ? gather_row(st, p, b, u0 + u * ustride, g) : -1;
+        int pending = -1, gi = 0;
+        bool ok = true;
+        while (u < n_tiles) {
+            const int s = u & 1;
+            if (g < NTILE) sm.grow[s][g] = nxt;   // unmapped rows are flagged by the producer warp
+            const int un = next_gathered(u + 1);
+            if (un < n_tiles && g < NTILE) nxt = gather_row(st, p, b, u0 + un * ustride, g);
+            ok = group_wait(sm, &sm.k_go[gi & 1], (gi >> 1) & 1, p.status, g);   // also publishes grow[s]
+            if (!ok) break;
+            const int32_t *gr = sm.grow[s];
+            const uint32_t kb = smem_addr(sm.k[s][0]);
+#pragma unroll 6
+            for (int i = 0; i < 18; ++i) {
+                const int q = g + GATHER_THREADS * i;   // < 32 x 72
+                const int row = q / 72, w = q - row * 72;
+                const int32_t pr = gr[32 * (int)rank + row];
+                const uint32_t dst = kb + (w >> 3) * (32 * 128) + row * 128 + (((w & 7) ^ (row & 7)) << 4);
+                const uint8_t *src = pr >= 0 ? p.pool + (size_t)pr * p.row_bytes + w * 16 : p.pool;
+                cp_async16(dst, src, pr >= 0 ? 16u : 0u);
+            }
+            cp_async_commit();
+            if (pending >= 0) {
+                // the tile before is complete once at most this tile's K copies are in flight
+                cp_async_wait<1>();
+                fence_proxy_async_smem();
+                named_barrier(2, GATHER_THREADS);
+                if (g == 0) {
+                    mbar_arrive_release_cluster(map_to_rank(&sm.k_full[pending & 1], 0));
+                    mbar_arrive_release_cluster(map_to_rank(&sm.v_full[pending & 1], 0));
+                }
+                pending = -1;
+            }
+            ok = group_wait(sm, &sm.v_go[gi & 1], (gi >> 1) & 1, p.status, g);
+            if (!ok) break;
+            const uint32_t vb = smem_addr(sm.v[s][0][0]);
+#pragma unroll 4
+            for (int i = 0; i < 16; ++i) {
+                const int q = g + GATHER_THREADS * i;   // < 64 x 32
+                const int row = q >> 5, w = q & 31, a = w >> 3, pp = w & 7;   // a = 2 j + atom
+                const int32_t pr = gr[row];
+                const uint32_t dst = vb + a * (NTILE * 128) + row * 128 + ((pp ^ (row & 7)) << 4);
+                const int col_chunk = 4 * (a >> 1) + 2 * (int)rank + (a & 1);
+                const uint8_t *src = pr >= 0 ? p.pool + (size_t)pr * p.row_bytes + col_chunk * 128 + pp * 16 : p.pool;
+                cp_async16(dst, src, pr >= 0 ? 16u : 0u);
+            }
+            cp_async_commit();
+            if (un == u + 1) pending = u;
+            else signal(s);
+            u = un;
+            ++gi;
+        }
+        cp_async_wait<0>();   // no copy may land after the CTA has left
+        if (ok && pending >= 0) signal(pending & 1);
+    } else if (warp >= 4 && warp < 8) {
         // ------------------------------------------------ softmax + epilogue
         const int L = threadIdx.x - 128;        // TMEM lane of this thread
         const int h = L & 63, half = L >> 6;     // head within the CTA, kv half of the tile
@@ -354,9 +442,9 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_const
         for (int u = 0; u < n_tiles; ++u) {
             const int s = u & 1;
             ok = ok && sm.abort_flag == 0;
-            if (ok) ok = mbar_wait(&sm.info_full[u % INFO], (u / INFO) & 1, WAIT_LIMIT);
+            if (ok) ok = mbar_wait(&sm.info_full[u % INFO], (u / INFO) & 1, WAIT_NS);
             const uint32_t vmask = ok ? (uint32_t)(sm.info_mask[u % INFO] >> (32 * half)) : 0u;
-            if (ok) ok = mbar_wait(&sm.s_full[s], (u >> 1) & 1, WAIT_LIMIT);
+            if (ok) ok = mbar_wait(&sm.s_full[s], (u >> 1) & 1, WAIT_NS);
             if (!ok && sm.abort_flag == 0) set_abort(sm, p.status);
             tc_fence_after();
             uint32_t raw[32];
@@ -380,50 +468,54 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_const
             mx = fmaxf(mx, sm.red[L ^ 64]);
             const float m_new = fmaxf(m_run, mx);
             m_run = m_new;
-            // P buffer s is free once P.V of tile u-2 completed.  O must be stable
-            // (P.V of tile u-1 done) only when it is rescaled, which is rare.
-            if (u > 1 && ok) {
-                ok = mbar_wait(&sm.pv_done[s], ((u - 2) >> 1) & 1, WAIT_LIMIT);
-                if (!ok && sm.abort_flag == 0) set_abort(sm, p.status);
-            }
-            if (m_new > -INFINITY && (m_ref == -INFINITY || m_new > m_ref + RESCALE_LOG2)) {
-                const float alpha = m_ref == -INFINITY ? 0.f : exp2f(m_ref - m_new);
-                if (u > 0) {
-                    if (ok) {
-                        ok = mbar_wait(&sm.pv_done[(u - 1) & 1], ((u - 1) >> 1) & 1, WAIT_LIMIT);
-                        if (!ok && sm.abort_flag == 0) set_abort(sm, p.status);
-                    }
-                    tc_fence_after();
-#pragma unroll 1
-                    for (int q = 0; q < 8; ++q) {
-                        uint32_t o[32];
-                        tmem_ld32(tmem + lane_base + TM_O + 32 * q, o);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                        tmem_st32(tmem + lane_base + TM_O + 32 * q, o);
-                    }
-                    tmem_wait_st();
-                }
+            const bool move = m_new > -INFINITY && (m_ref == -INFINITY || m_new > m_ref + RESCALE_LOG2);
+            const float alpha = !move ? 1.f : (m_ref == -INFINITY ? 0.f : exp2f(m_ref - m_new));
+            if (move) {
                 l *= alpha;
                 m_ref = m_new;
             }
+            // P = hi + lo, both bf16: rounding P to one bf16 alone leaves a relative error
+            // of 2^-9 on every weight, which peaked rows carry straight into the output.
             float psum = 0.f;
-            uint32_t pk[16];
+            uint32_t pk_hi[16], pk_lo[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const float p0 = exp2f(sv[2 * i] - m_ref), p1 = exp2f(sv[2 * i + 1] - m_ref);
                 const float q0 = m_ref == -INFINITY ? 0.f : p0, q1 = m_ref == -INFINITY ? 0.f : p1;
                 psum += q0 + q1;
-                pk[i] = pack_bf16x2(q0, q1);
+                const __nv_bfloat162 hi = __floats2bfloat162_rn(q0, q1);
+                pk_hi[i] = *reinterpret_cast<const uint32_t *>(&hi);
+                pk_lo[i] = pack_bf16x2(q0 - __low2float(hi), q1 - __high2float(hi));
             }
             l += psum;
-            uint8_t *prow = sm.p[s] + h * 128;
+            // The P buffers are rewritten and O may be rescaled: P.V of tile u-1 must be done.
+            if (u > 0 && ok) {
+                ok = mbar_wait(&sm.pv_done[(u - 1) & 1], ((u - 1) >> 1) & 1, WAIT_NS);
+                if (!ok && sm.abort_flag == 0) set_abort(sm, p.status);
+            }
+            // tcgen05.ld / st are warp-collective: the whole warp takes the rescale when
+            // any of its rows moves its reference, the other rows scale by 1.
+            if (__any_sync(0xffffffffu, move) && u > 0) {
+                tc_fence_after();
+#pragma unroll 1
+                for (int q = 0; q < 8; ++q) {
+                    uint32_t o[32];
+                    tmem_ld32(tmem + lane_base + TM_O + 32 * q, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    tmem_st32(tmem + lane_base + TM_O + 32 * q, o);
+                }
+                tmem_wait_st();
+            }
+            uint8_t *prow_hi = sm.p[0] + h * 128, *prow_lo = sm.p[1] + h * 128;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                const int chunk = 4 * half + c;
-                *reinterpret_cast<uint4 *>(prow + ((chunk ^ (h & 7)) << 4)) =
-                    make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                const int chunk = 4 * half + c, off = (chunk ^ (h & 7)) << 4;
+                *reinterpret_cast<uint4 *>(prow_hi + off) =
+                    make_uint4(pk_hi[4 * c], pk_hi[4 * c + 1], pk_hi[4 * c + 2], pk_hi[4 * c + 3]);
+                *reinterpret_cast<uint4 *>(prow_lo + off) =
+                    make_uint4(pk_lo[4 * c], pk_lo[4 * c + 1], pk_lo[4 * c + 2], pk_lo[4 * c + 3]);
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -432,7 +524,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_const
         }
         // ---- epilogue: wait for the last P.V, then write the partial
         if (n_tiles > 0 && ok) {
-            ok = mbar_wait(&sm.pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, WAIT_LIMIT);
+            ok = mbar_wait(&sm.pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, WAIT_NS);
             if (!ok && sm.abort_flag == 0) set_abort(sm, p.status);
         }
         tc_fence_after();
@@ -469,8 +561,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_const
 
     // ---- teardown: every MMA finished before TMEM is released; no CTA leaves early
     if (warp == 3 && n_tiles > 0) {
-        // the even CTA's MMA thread commits mma_done to both CTAs after its last MMA
-        if (lane == 0 && !mbar_wait(&sm.mma_done, 0, WAIT_LIMIT)) set_abort(sm, p.status);
+        // each of the even CTA's two MMA threads commits mma_done to both CTAs after its last MMA
+        if (lane == 0 && !mbar_wait(&sm.mma_done, 0, WAIT_NS)) set_abort(sm, p.status);
         __syncwarp();
     }
     __syncthreads();
@@ -501,15 +593,17 @@ static EncodeTiled encoder() {
     return fn;
 }
 
-static bool make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint64_t row_bytes,
-                     uint32_t box_cols, uint32_t box_rows) {
+// bf16 tensor map of `rank` dimensions (dims[0] innermost, strides in bytes for
+// dims 1..rank-1), 128-byte swizzle, zero fill outside the tensor.
+static bool make_map(CUtensorMap *m, const void *base, int rank, const uint64_t *dims, const uint64_t *strides,
+                     const uint32_t *box) {
     EncodeTiled enc = encoder();
     if (!enc) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {row_bytes};
-    cuuint32_t box[2] = {box_cols, box_rows};
-    cuuint32_t es[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+    cuuint64_t d[5], st[4];
+    cuuint32_t bx[5], es[5];
+    for (int i = 0; i < rank; ++i) { d[i] = dims[i]; bx[i] = box[i]; es[i] = 1; }
+    for (int i = 0; i + 1 < rank; ++i) st[i] = strides[i];
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(base), d, st, bx, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -525,17 +619,31 @@ int launch(const uint16_t *q, const uint16_t *kv_pool, int64_t k_stride, int64_t
            int table_stride, const int32_t *topk_idx, const int32_t *topk_count, int k, const int32_t *window_start,
            const int32_t *window_len, int B, float scale, int n_splits, float *o_part, float *m_part, float *l_part,
            int32_t *status, cudaStream_t stream) {
-    CUtensorMap kv_map, kv_map32, kv_map64, q_map;
+    // Column chunk c of a row is 128 bytes at offset 128 c, so a row is also a
+    // [9][64] array and boxes can span chunks as a third (and fourth) dimension:
+    //   K: {64 columns, rows, 9 chunks}, box {64, 32, 9}  -> [chunk][32 rows][128 B]
+    //   V: {64 columns, rows, 4 chunks, 2 groups of 4}, box {64, 64, 2, 2} at chunk 2r
+    //      -> [group j][chunk 4j + 2r + a][64 rows][128 B]
+    //   Q: {64 columns, B x 128 heads, 9 chunks}, box {64, 64, 9}
+    CUtensorMap k_map, v_map, q_map;
     const uint64_t pool_rows = (uint64_t)n_slots * LSA_CHUNK;
-    if (!make_map(&kv_map, kv_pool, DQK, pool_rows, (uint64_t)k_stride * 2, 64, 1) ||
-        !make_map(&kv_map32, kv_pool, DQK, pool_rows, (uint64_t)k_stride * 2, 64, 32) ||
-        !make_map(&kv_map64, kv_pool, DQK, pool_rows, (uint64_t)k_stride * 2, 64, 64))
+    if (pool_rows + 64 >= (1ull << 31) || (uint64_t)B * HQ >= (1ull << 31))
+        return fail(LSA_ERR_SHAPE, "lsa_sparse_decode: pool rows must stay below 2^31 for the latent kernel");
+    const uint64_t rb = (uint64_t)k_stride * 2;
+    const uint64_t kd[3] = {64, pool_rows, KCH}, ks[2] = {rb, 128};
+    const uint32_t kbox[3] = {64, 32, KCH};
+    const uint64_t vd[4] = {64, pool_rows, 4, 2}, vs[3] = {rb, 128, 512};
+    const uint32_t vbox[4] = {64, NTILE, 2, 2};
+    const uint64_t qd[3] = {64, (uint64_t)B * HQ, KCH}, qs[2] = {DQK * 2, 128};
+    const uint32_t qbox[3] = {64, HPC, KCH};
+    if (!make_map(&k_map, kv_pool, 3, kd, ks, kbox) || !make_map(&v_map, kv_pool, 4, vd, vs, vbox))
         return fail(LSA_ERR_CUDA, "lsa_sparse_decode: cuTensorMapEncodeTiled failed for the KV pool");
-    if (!make_map(&q_map, q, DQK, (uint64_t)B * HQ, DQK * 2, 64, 64))
+    if (!make_map(&q_map, q, 3, qd, qs, qbox))
         return fail(LSA_ERR_CUDA, "lsa_sparse_decode: cuTensorMapEncodeTiled failed for q");
     Params prm;
     prm.table = table; prm.topk_idx = topk_idx; prm.topk_count = topk_count;
     prm.window_start = window_start; prm.window_len = window_len;
+    prm.pool = reinterpret_cast<const uint8_t *>(kv_pool); prm.row_bytes = (int64_t)rb;
     prm.o_part = o_part; prm.m_part = m_part; prm.l_part = l_part; prm.status = status;
     prm.n_rows_pool = n_slots * LSA_CHUNK; prm.table_stride = table_stride; prm.k = k; prm.n_splits = n_splits;
     prm.scale_log2 = scale * 1.4426950408889634f;
@@ -553,7 +661,7 @@ int launch(const uint16_t *q, const uint16_t *kv_pool, int64_t k_stride, int64_t
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    LSA_CUDA(cudaLaunchKernelEx(&cfg, mla_decode_kernel, kv_map, kv_map32, kv_map64, q_map, prm));
+    LSA_CUDA(cudaLaunchKernelEx(&cfg, mla_decode_kernel, k_map, v_map, q_map, prm));
     return LSA_OK;
 }
 

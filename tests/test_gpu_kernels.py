@@ -191,12 +191,18 @@ def _decode_case(L, wl, kept, host, s, topk_override=None, table_override=None):
     return out.cpu().numpy(), lse.cpu().numpy(), refs, int(status.item())
 
 
-@pytest.mark.parametrize("shape", ["mla128", "mla64", "sep16"])
+@pytest.mark.parametrize("shape", ["mla128", "mla128_many_tiles", "mla64", "sep16"])
 @pytest.mark.parametrize("q_scale", [1.0, 4.0])
 def test_sparse_decode_matches_oracle(L, shape, q_scale):
     if shape == "sep16":
         wl = W.workload("decode_16k_b1_h16", B=2, ctx=(80 * CH, 33 * CH), window=20 * CH, steps=2,
                         pass_rate=(0.3, 0.4), q_scale=q_scale, k=300)
+    elif shape == "mla128_many_tiles":
+        # 8 sequences -> 9 splits each, ~6 tiles per split: both K/V stages are reused and
+        # gathered (top-k, last partial chunk) and box-loaded window tiles alternate
+        ctx = tuple(c * CH for c in (96, 60, 120, 64, 80, 100, 70, 90))
+        wl = _small_mla(B=8, ctx=ctx, pass_rate=(0.3, 0.5, 0.4, 0.6, 0.35, 0.3, 0.5, 0.45), window=40 * CH,
+                        k=700, steps=2, q_scale=q_scale)
     else:
         wl = _small_mla(q_scale=q_scale, k=500, Hq=128 if shape == "mla128" else 64)
     host = host_build(wl)
@@ -236,6 +242,76 @@ def test_sparse_decode_skips_rows_without_slot_and_flags(L):
     krow = host["oracle_pools"]["kv"][host["oracle_table"][0][pos // CH], pos % CH]
     ref, _ = oracle.attention_dense(host["step"]["q"][0, 0], krow, np.ascontiguousarray(krow[:, :wl.dv]), wl.scale)
     H.assert_close_attention(out[0], ref)
+
+
+def _rows_reference(host, wl, b, pos):
+    """Oracle attention of query step 0 of sequence b over the pool rows of positions `pos`."""
+    krow = host["oracle_pools"]["kv"][host["oracle_table"][b][pos // CH], pos % CH]
+    return oracle.attention_dense(host["step"]["q"][0, b], krow, np.ascontiguousarray(krow[:, :wl.dv]), wl.scale)
+
+
+def _call_rows(L, wl, host, pools_kv, table, sel, wstart, wlen):
+    d = dev()
+    tk = np.full((wl.B, wl.k), -1, np.int32)
+    tc = np.zeros(wl.B, np.int32)
+    for b in range(wl.B):
+        tk[b, :len(sel[b])] = sel[b]
+        tc[b] = len(sel[b])
+    status = torch.zeros(1, dtype=torch.int32, device=d)
+    out, _ = L.sparse_decode(bf16(host["step"]["q"][0], d), bf16(pools_kv, d), None, i32(table, d), i32(tk, d),
+                             i32(tc, d), i32(wstart, d), i32(wlen, d), int(max(wlen)), wl.dv, wl.scale, status=status)
+    return out.cpu().numpy(), int(status.item())
+
+
+def _oracle_topk(host, wl):
+    kept, _, _, _ = H.kept_lists(host)
+    sel = [H.oracle_step(host, kept[b], b, 0) for b in range(wl.B)]
+    return [r["topk"][:r["topk_count"]].astype(np.int64) for r in sel]
+
+
+def test_sparse_decode_unaligned_window_ignores_poisoned_rows(L):
+    """A window that starts and ends inside chunks is attended row by row; the
+    rows of its first and last chunk outside the window hold NaN and must not
+    reach the output."""
+    wl = _small_mla(k=300, steps=1)
+    host = host_build(wl)
+    sel = _oracle_topk(host, wl)
+    w0 = host["window_start"].astype(np.int64)
+    wstart = (w0 + 17).astype(np.int32)
+    wlen = np.full(wl.B, wl.window - 40, np.int32)
+    pools = host["pools"]["kv"].copy()
+    table = host["chunk_table"]
+    for b in range(wl.B):
+        first, end = int(wstart[b]), int(wstart[b]) + int(wlen[b])
+        outside = np.r_[np.arange(first - first % CH, first), np.arange(end, end - end % CH + CH if end % CH else end)]
+        pools[table[b][outside // CH], outside % CH] = 0x7FC0       # bf16 NaN
+    out, st = _call_rows(L, wl, host, pools, table, sel, wstart, wlen)
+    assert st == 0
+    for b in range(wl.B):
+        pos = np.r_[sel[b], np.arange(int(wstart[b]), int(wstart[b]) + int(wlen[b]))]
+        ref, _ = _rows_reference(host, wl, b, pos)
+        assert np.isfinite(out[b]).all()
+        H.assert_close_attention(out[b], ref)
+
+
+def test_sparse_decode_window_chunk_without_slot_is_skipped(L):
+    """A whole window chunk whose table entry is -1 contributes nothing and sets LSA_DEV_TABLE."""
+    wl = _small_mla(k=200, steps=1)
+    host = host_build(wl)
+    sel = _oracle_topk(host, wl)
+    wstart = host["window_start"]
+    wlen = np.full(wl.B, wl.window, np.int32)
+    table = host["chunk_table"].copy()
+    gone = int(wstart[1]) // CH + 3
+    table[1, gone] = -1
+    out, st = _call_rows(L, wl, host, host["pools"]["kv"], table, sel, wstart, wlen)
+    assert st & L.DEV_TABLE
+    for b in range(wl.B):
+        win = np.arange(int(wstart[b]), int(wstart[b]) + int(wlen[b]))
+        if b == 1:
+            win = win[win // CH != gone]
+        ref, _ = _rows_reference(host, wl, b, np.r_[sel[b], win])
+        H.assert_close_attention(out[b], ref)
 
 
 # ------------------------------------------------------------------- a7 ---
