@@ -190,6 +190,11 @@ __device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
+// Fetches `bytes` (a multiple of 16) at a 16-byte aligned global address into L2.
+__device__ __forceinline__ void l2_prefetch(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // ------------------------------------------------------------- tcgen05 ----
 
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t *dst_smem, uint32_t ncols) {

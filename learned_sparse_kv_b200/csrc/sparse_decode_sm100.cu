@@ -25,9 +25,9 @@
 // chunk) are copied by a warpgroup with 16-byte cp.async into the same layout;
 // missing rows are zero-filled.  Two stages of each operand are in flight.
 // Warp roles:
-//   0      TMA producer, tile-validity masks
+//   0      K producer (TMA), tile-validity masks
 //   1      S = Q K^T issuer (even CTA)        2   O += P V issuer (even CTA)
-//   3      TMEM allocator
+//   3      TMEM allocator, V producer (TMA)
 //   4..7   softmax, O rescale, epilogue (one thread per TMEM lane)
 //   8..11  row gather for gathered tiles
 // The online softmax is evaluated in the log2 domain; the reference maximum
@@ -225,67 +225,71 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
     const int n_tiles = split < st.total ? (st.total - 1 - split) / p.n_splits + 1 : 0;
     const int u0 = split, ustride = p.n_splits;
 
-    if (warp == 0 && n_tiles > 0) {
-        // ------------------------------------------------ TMA producer + tile masks
-        if (lane == 0) {
+    // Every tile's stage is waited for by its producer in tile order: a parity wait is
+    // only unambiguous one phase behind the barrier, so the gather warpgroup (which
+    // skips the TMA tiles) is handed its stages through k_go / v_go, whose phases count
+    // gathered tiles only.  K (warp 0) and V (warp 3) have a producer each, so K of a
+    // later tile never waits behind the P.V that frees a V stage.
+    if ((warp == 0 || warp == 3) && n_tiles > 0) {
+        // ------------------------------------------------ TMA producers (K + masks, V)
+        const bool kprod = warp == 0;
+        if (kprod && lane == 0) {
             const uint32_t qf = map_to_rank(&sm.q_full, 0);
             mbar_arrive_expect_tx_cluster(qf, Q_BYTES);
             tma_load_3d(sm.q[0], &q_map, 0, b * HQ + HPC * (int)rank, 0, qf);
         }
         // row indices of the next gathered tile are loaded while the current tile is issued
         int64_t n0 = -1, n1 = -1;
-        if (st.gathered(u0)) { n0 = st.row(p, b, u0, lane); n1 = st.row(p, b, u0, lane + 32); }
+        if (kprod && st.gathered(u0)) { n0 = st.row(p, b, u0, lane); n1 = st.row(p, b, u0, lane + 32); }
         int gi = 0;   // gathered tiles handed to the gather warpgroup so far
         for (int u = 0; u < n_tiles; ++u) {
             const int t = u0 + u * ustride;
             const bool gath = st.gathered(t);
-            const int64_t g0 = n0, g1 = n1;
-            if (u + 1 < n_tiles && st.gathered(t + ustride)) {
-                n0 = st.row(p, b, t + ustride, lane);
-                n1 = st.row(p, b, t + ustride, lane + 32);
-            }
-            unsigned long long mask;
-            int64_t slot_row = -2;
-            if (!gath) {
-                slot_row = st.window_slot_row(p, b, t);
-                if (slot_row == -2) flag(p.status, LSA_DEV_TABLE);
-                mask = slot_row < 0 ? 0ull : ~0ull;
-            } else {
-                if ((g0 == -2 || g1 == -2)) flag(p.status, LSA_DEV_TABLE);
-                const unsigned lo = __ballot_sync(0xffffffffu, g0 >= 0), hi = __ballot_sync(0xffffffffu, g1 >= 0);
-                mask = (unsigned long long)lo | ((unsigned long long)hi << 32);
-            }
-            if (!warp_wait(sm, &sm.info_empty[u % INFO], ((u / INFO) + 1) & 1, p.status)) break;
-            if (lane == 0) {
-                sm.info_mask[u % INFO] = mask;
-                asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];\n" ::"r"(smem_addr(&sm.info_full[u % INFO])) : "memory");
-            }
-            // Every tile's stage is waited for here, in tile order: a parity wait is only
-            // unambiguous one phase behind the barrier, so the gather warpgroup (which
-            // skips the TMA tiles) is handed its stages through k_go / v_go, whose
-            // phases count gathered tiles only.
-            const int s = u & 1;
-            const uint32_t par = ((u >> 1) + 1) & 1;
+            const int64_t slot_row = gath ? -2 : st.window_slot_row(p, b, t);
             // an unmapped slot is read out of range: TMA fills zeros
             const int wy = slot_row >= 0 ? (int)slot_row : (int)p.n_rows_pool;
-            if (!warp_wait(sm, &sm.k_empty[s], par, p.status)) break;
-            if (lane == 0) {
-                if (gath) {
-                    mbar_arrive_local(&sm.k_go[gi & 1]);
-                } else {
-                    const uint32_t full = map_to_rank(&sm.k_full[s], 0);
-                    mbar_arrive_expect_tx_cluster(full, K_BYTES);
-                    tma_load_3d(sm.k[s][0], &k_map, 0, wy + 32 * (int)rank, 0, full);
+            const int s = u & 1;
+            const uint32_t par = ((u >> 1) + 1) & 1;
+            if (kprod) {
+                const int64_t g0 = n0, g1 = n1;
+                if (u + 1 < n_tiles && st.gathered(t + ustride)) {
+                    n0 = st.row(p, b, t + ustride, lane);
+                    n1 = st.row(p, b, t + ustride, lane + 32);
                 }
-            }
-            if (!warp_wait(sm, &sm.v_empty[s], par, p.status)) break;
-            if (lane == 0) {
-                if (gath) {
-                    mbar_arrive_local(&sm.v_go[gi & 1]);
+                unsigned long long mask;
+                if (!gath) {
+                    if (slot_row == -2) flag(p.status, LSA_DEV_TABLE);
+                    mask = slot_row < 0 ? 0ull : ~0ull;
                 } else {
-                    const uint32_t full = map_to_rank(&sm.v_full[s], 0);
-                    mbar_arrive_expect_tx_cluster(full, V_BYTES);
-                    tma_load_4d(sm.v[s][0][0], &v_map, 0, wy, 2 * (int)rank, 0, full);
+                    if ((g0 == -2 || g1 == -2)) flag(p.status, LSA_DEV_TABLE);
+                    const unsigned lo = __ballot_sync(0xffffffffu, g0 >= 0), hi = __ballot_sync(0xffffffffu, g1 >= 0);
+                    mask = (unsigned long long)lo | ((unsigned long long)hi << 32);
+                }
+                if (!warp_wait(sm, &sm.info_empty[u % INFO], ((u / INFO) + 1) & 1, p.status)) break;
+                if (lane == 0) {
+                    sm.info_mask[u % INFO] = mask;
+                    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];\n" ::"r"(smem_addr(&sm.info_full[u % INFO])) : "memory");
+                }
+                if (!warp_wait(sm, &sm.k_empty[s], par, p.status)) break;
+                if (lane == 0) {
+                    if (gath) {
+                        mbar_arrive_local(&sm.k_go[gi & 1]);
+                    } else {
+                        const uint32_t full = map_to_rank(&sm.k_full[s], 0);
+                        mbar_arrive_expect_tx_cluster(full, K_BYTES);
+                        tma_load_3d(sm.k[s][0], &k_map, 0, wy + 32 * (int)rank, 0, full);
+                    }
+                }
+            } else {
+                if (!warp_wait(sm, &sm.v_empty[s], par, p.status)) break;
+                if (lane == 0) {
+                    if (gath) {
+                        mbar_arrive_local(&sm.v_go[gi & 1]);
+                    } else {
+                        const uint32_t full = map_to_rank(&sm.v_full[s], 0);
+                        mbar_arrive_expect_tx_cluster(full, V_BYTES);
+                        tma_load_4d(sm.v[s][0][0], &v_map, 0, wy, 2 * (int)rank, 0, full);
+                    }
                 }
             }
             gi += gath ? 1 : 0;
