@@ -3,17 +3,19 @@
 // (arXiv 2606.09079: the Lightning Indexer's fine top-k inside the kept set,
 // gist.science explainer 2.1 "Gestufte Selektion", cjcn.com.cn article section 2.)
 //
-// One CTA of 1024 threads per sequence.  A 4-pass, 8-bit radix select over
+// One cluster of 16 CTAs per sequence.  A 4-pass, 8-bit radix select over
 // order-preserving uint32 keys finds the k-th largest key T and how many of
-// the keys equal to T are taken; an order-preserving block scan then emits
-// every candidate with key > T and the first `need` candidates with key == T,
-// in candidate order, which is ascending position.
+// the keys equal to T are taken; an order-preserving scan over the cluster then
+// emits every candidate with key > T and the first `need` candidates with
+// key == T, in candidate order, which is ascending position.
 #include "block_scan.cuh"
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace lsa {
 
-constexpr int kTopkThreads = 1024;
+constexpr int kTopkThreads = 512;   // threads per CTA
+constexpr int kTopkCtas = 16;       // CTAs per sequence: one thread-block cluster
 
 int launch_li_scores(const uint16_t *, const uint16_t *, const uint16_t *, int64_t, const int32_t *, int,
                      const int32_t *, const int32_t *, int, const int32_t *, const int32_t *, int, int, int, float *,
@@ -60,87 +62,120 @@ __device__ __forceinline__ void warp_hist_add(int *hist, uint32_t bin, bool acti
     if ((threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(&hist[bin], __popc(same));
 }
 
-// Scores of one sequence: from shared memory when they were staged there, else global.
+__device__ __forceinline__ int ld_cluster_s32(const void *p, uint32_t rank) {
+    int v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];\n" : "=r"(v) : "r"(sm100::map_to_rank(p, rank)) : "memory");
+    return v;
+}
+
+struct TopkShared {
+    int hist[2][256];                     // digit counts of this CTA's slice, double-buffered by pass
+    int warp_tot[kTopkThreads / 32 + 1];
+    int cnt[2];                           // this CTA's counts of keys > T and == T
+    int base, eq_lower;                   // output offset of this CTA, keys == T in lower CTAs
+    uint32_t prefix;
+    int remaining;
+};
+
+// Top-k of the n scores of one sequence by the kTopkCtas CTAs of a cluster.
+// CTA c takes the contiguous slice [c seg, (c + 1) seg) and stages its keys in
+// shared memory when they fit (stage_cap keys).  Each 8-bit radix pass counts
+// digits locally; after a cluster barrier every CTA sums the kTopkCtas
+// histograms through distributed shared memory and picks the same digit, so
+// no result has to be broadcast.  The emission is ordered: a CTA's output
+// offset is the number of selected keys in the lower slices, and ties at the
+// threshold go to the lowest candidate indices.
 template <class PosFn>
-__device__ void topk_block(const float *__restrict__ s_glob, const float *s, int n, int k, PosFn pos,
-                           int32_t *__restrict__ out, int32_t *__restrict__ out_count) {
-    __shared__ int hist[256];
-    __shared__ int warp_tot[kTopkThreads / 32 + 1];
-    __shared__ uint32_t sh_prefix;
-    __shared__ int sh_remaining;
+__device__ void topk_cluster(const float *__restrict__ s, int n, int k, PosFn pos, int32_t *__restrict__ out,
+                             int32_t *__restrict__ out_count, int stage_cap) {
+    __shared__ TopkShared sh;
+    extern __shared__ uint32_t keys[];
     const int t = threadIdx.x;
-    (void)s_glob;
+    const int c = (int)sm100::cluster_rank();
 
     if (n <= k) {  // everything is selected, already in ascending order
-        for (int j = t; j < k; j += kTopkThreads) out[j] = j < n ? pos(j) : -1;
-        if (t == 0) *out_count = n;
+        for (int j = c * kTopkThreads + t; j < k; j += kTopkCtas * kTopkThreads) out[j] = j < n ? pos(j) : -1;
+        if (c == 0 && t == 0) *out_count = n;
         return;
     }
+    const int seg = (n + kTopkCtas - 1) / kTopkCtas;
+    const int j0 = min(n, c * seg), len = min(n, j0 + seg) - j0;
+    const bool staged = len <= stage_cap;
+    if (staged)
+        for (int i = t; i < len; i += kTopkThreads) keys[i] = ordered_key(s[j0 + i]);
+    auto key = [&](int i) { return staged ? keys[i] : ordered_key(s[j0 + i]); };
+    __syncthreads();
 
     uint32_t prefix = 0, pmask = 0;
     int remaining = k;
-    const int n_round = (n + kTopkThreads - 1) / kTopkThreads * kTopkThreads;   // warp-uniform trip count
+    const int len_round = (len + kTopkThreads - 1) / kTopkThreads * kTopkThreads;   // warp-uniform trip count
 #pragma unroll 1
-    for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        // hist[pass & 1] was last read by the other CTAs before the previous pass's
+        // cluster barrier, which this CTA has passed.
+        int *hist = sh.hist[pass & 1];
         if (t < 256) hist[t] = 0;
         __syncthreads();
-        for (int j = t; j < n_round; j += kTopkThreads) {
-            const uint32_t u = j < n ? ordered_key(s[j]) : 0u;
-            warp_hist_add(hist, (u >> shift) & 255u, j < n && (u & pmask) == prefix);
+        for (int i = t; i < len_round; i += kTopkThreads) {
+            const uint32_t u = i < len ? key(i) : 0u;
+            warp_hist_add(hist, (u >> shift) & 255u, i < len && (u & pmask) == prefix);
         }
-        __syncthreads();
-        // suffix counts over digits, highest digit first
-        int v = t < 256 ? hist[255 - t] : 0;
+        sm100::cluster_sync();   // every CTA's histogram of this pass is complete
+        int v = 0;               // suffix counts over digits, highest digit first
+        if (t < 256)
+            for (int r = 0; r < kTopkCtas; ++r) v += ld_cluster_s32(&hist[255 - t], (uint32_t)r);
         int total;
-        int excl = block_exclusive_scan<kTopkThreads>(v, warp_tot, &total);
-        if (t < 256) {
-            int incl = excl + v;
-            if (incl >= remaining && excl < remaining) {
-                sh_prefix = prefix | (uint32_t(255 - t) << shift);
-                sh_remaining = remaining - excl;
-            }
+        const int excl = block_exclusive_scan<kTopkThreads>(v, sh.warp_tot, &total);
+        if (t < 256 && excl < remaining && excl + v >= remaining) {
+            sh.prefix = prefix | (uint32_t(255 - t) << shift);
+            sh.remaining = remaining - excl;
         }
         __syncthreads();
-        prefix = sh_prefix;
-        remaining = sh_remaining;
+        prefix = sh.prefix;
+        remaining = sh.remaining;
         pmask |= 255u << shift;
         __syncthreads();
     }
     const uint32_t T = prefix;
     const int need_eq = remaining;  // keys equal to T that are taken, >= 1
 
-    const int seg = (n + kTopkThreads - 1) / kTopkThreads;
-    const int j0 = min(n, t * seg), j1 = min(n, j0 + seg);
+    const int sub = (len + kTopkThreads - 1) / kTopkThreads;
+    const int i0 = min(len, t * sub), i1 = min(len, i0 + sub);
     int gt = 0, eq = 0;
-    for (int j = j0; j < j1; ++j) {
-        uint32_t u = ordered_key(s[j]);
+    for (int i = i0; i < i1; ++i) {
+        const uint32_t u = key(i);
         gt += u > T;
         eq += u == T;
     }
+    int gt_tot, eq_tot;
+    const int eq_before = block_exclusive_scan<kTopkThreads>(eq, sh.warp_tot, &eq_tot);
+    (void)block_exclusive_scan<kTopkThreads>(gt, sh.warp_tot, &gt_tot);
+    if (t == 0) { sh.cnt[0] = gt_tot; sh.cnt[1] = eq_tot; }
+    sm100::cluster_sync();   // every CTA's counts are published
+    if (t == 0) {
+        int base = 0, eq_lower = 0;
+        for (int r = 0; r < c; ++r) {
+            const int g_r = ld_cluster_s32(&sh.cnt[0], (uint32_t)r), e_r = ld_cluster_s32(&sh.cnt[1], (uint32_t)r);
+            base += g_r + min(e_r, max(0, need_eq - eq_lower));
+            eq_lower += e_r;
+        }
+        sh.base = base;
+        sh.eq_lower = eq_lower;
+    }
+    __syncthreads();
+    int take_eq = min(eq, max(0, need_eq - (sh.eq_lower + eq_before)));
     int dummy;
-    int eq_before = block_exclusive_scan<kTopkThreads>(eq, warp_tot, &dummy);
-    int take_eq = min(eq, max(0, need_eq - eq_before));
-    int o = block_exclusive_scan<kTopkThreads>(gt + take_eq, warp_tot, &dummy);
-    for (int j = j0; j < j1; ++j) {
-        uint32_t u = ordered_key(s[j]);
+    int o = sh.base + block_exclusive_scan<kTopkThreads>(gt + take_eq, sh.warp_tot, &dummy);
+    for (int i = i0; i < i1; ++i) {
+        const uint32_t u = key(i);
         if (u > T || (u == T && take_eq > 0)) {
             if (u == T) --take_eq;
-            out[o++] = pos(j);
+            out[o++] = pos(j0 + i);
         }
     }
-    if (t == 0) *out_count = k;
-}
-
-// Copies n scores into dynamic shared memory when they fit; returns the array to read.
-__device__ __forceinline__ const float *stage_scores(const float *__restrict__ g, int n, int cap) {
-    extern __shared__ float stage[];
-    if (n > cap) return g;
-    const int n4 = (reinterpret_cast<uintptr_t>(g) & 15) == 0 ? n / 4 : 0;
-    for (int i = threadIdx.x; i < n4; i += kTopkThreads)
-        reinterpret_cast<float4 *>(stage)[i] = reinterpret_cast<const float4 *>(g)[i];
-    for (int i = 4 * n4 + threadIdx.x; i < n; i += kTopkThreads) stage[i] = g[i];
-    __syncthreads();
-    return stage;
+    if (c == 0 && t == 0) *out_count = k;
+    sm100::cluster_sync();   // no CTA leaves while another may still read its counts
 }
 
 __global__ void __launch_bounds__(kTopkThreads) topk_kept_kernel(const float *__restrict__ scores, int kept_cap,
@@ -148,27 +183,48 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kept_kernel(const float *__
                                                                  const int32_t *__restrict__ cold, int k,
                                                                  int32_t *__restrict__ topk_idx,
                                                                  int32_t *__restrict__ topk_count, int stage_cap) {
-    const int b = blockIdx.x;
+    const int b = blockIdx.y;
     const int32_t *kept = kept_idx + (size_t)b * kept_cap;
-    const int n = cold[b] * LSA_CHUNK;
-    const float *g = scores + (size_t)b * kept_cap * LSA_CHUNK;
-    const float *s = n > k ? stage_scores(g, n, stage_cap) : g;
-    topk_block(g, s, n, k, CandFromKept{kept}, topk_idx + (size_t)b * k, topk_count + b);
+    const int n = min(max(cold[b], 0), kept_cap) * LSA_CHUNK;
+    topk_cluster(scores + (size_t)b * kept_cap * LSA_CHUNK, n, k, CandFromKept{kept}, topk_idx + (size_t)b * k,
+                 topk_count + b, stage_cap);
 }
 
 __global__ void __launch_bounds__(kTopkThreads) topk_scores_kernel(const float *__restrict__ scores,
                                                                    const int64_t *__restrict__ off, int max_cand,
                                                                    int k, int32_t *__restrict__ topk_idx,
                                                                    int32_t *__restrict__ topk_count, int stage_cap) {
-    const int b = blockIdx.x;
+    const int b = blockIdx.y;
     const int64_t a = off[b];
     const int n = (int)max((int64_t)0, min(off[b + 1] - a, (int64_t)max_cand));
-    const float *s = n > k ? stage_scores(scores + a, n, stage_cap) : scores + a;
-    topk_block(scores + a, s, n, k, CandIdentity{}, topk_idx + (size_t)b * k, topk_count + b);
+    topk_cluster(scores + a, n, k, CandIdentity{}, topk_idx + (size_t)b * k, topk_count + b, stage_cap);
 }
 
-// Scores staged in shared memory: up to 200 KB (51,200 candidates), never more than needed.
-static int stage_capacity(int max_n) { return max(0, min(max_n, 51200)); }
+// Keys staged per CTA: a slice of at most ceil(max_n / 16), never more than 24,576 (96 KB).
+static int stage_capacity(int max_n) { return max(0, min((max_n + kTopkCtas - 1) / kTopkCtas, 24576)); }
+
+// One cluster of kTopkCtas CTAs per sequence.
+template <class... Args>
+static int launch_topk(void (*kernel)(Args...), int B, int stage_cap, cudaStream_t stream, const char *what,
+                       Args... args) {
+    const size_t smem = (size_t)stage_cap * sizeof(uint32_t);
+    LSA_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    LSA_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kTopkCtas, B, 1);
+    cfg.blockDim = dim3(kTopkThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kTopkCtas;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    LSA_CUDA(cudaLaunchKernelEx(&cfg, kernel, args...));
+    return check_launch(what);
+}
 
 }  // namespace lsa
 
@@ -210,11 +266,8 @@ extern "C" int lsa_topk(const lsa_bf16 *q_li, const lsa_bf16 *w_li, const lsa_bf
                           window_start, cold, B, Hl, dl, buf, dev_status, stream);
     if (rc) return rc;
     const int cap = stage_capacity(kept_cap * LSA_CHUNK);
-    LSA_CUDA(cudaFuncSetAttribute(topk_kept_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)(cap * sizeof(float))));
-    topk_kept_kernel<<<B, kTopkThreads, cap * sizeof(float), stream>>>(buf, kept_cap, kept_idx, cold, k, topk_idx,
-                                                                       topk_count, cap);
-    return check_launch("topk_kept_kernel");
+    return launch_topk(topk_kept_kernel, B, cap, stream, "topk_kept_kernel", (const float *)buf, kept_cap,
+                       kept_idx, (const int32_t *)cold, k, topk_idx, topk_count, cap);
 }
 
 extern "C" int lsa_topk_from_scores(const float *scores, const int64_t *cand_offset, int B, int max_cand, int k,
@@ -226,9 +279,6 @@ extern "C" int lsa_topk_from_scores(const float *scores, const int64_t *cand_off
     LSA_REQUIRE(max_cand >= 0, LSA_ERR_INVALID_ARG, "lsa_topk_from_scores: max_cand must be >= 0");
     LSA_REQUIRE(k >= 1 && k <= 65536, LSA_ERR_INVALID_ARG, "lsa_topk_from_scores: k=%d outside [1, 65536]", k);
     const int cap = stage_capacity(max_cand);
-    LSA_CUDA(cudaFuncSetAttribute(topk_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)(cap * sizeof(float))));
-    topk_scores_kernel<<<B, kTopkThreads, cap * sizeof(float), stream>>>(scores, cand_offset, max_cand, k, topk_idx,
-                                                                         topk_count, cap);
-    return check_launch("topk_scores_kernel");
+    return launch_topk(topk_scores_kernel, B, cap, stream, "topk_scores_kernel", scores, cand_offset, max_cand, k,
+                       topk_idx, topk_count, cap);
 }
