@@ -273,29 +273,33 @@ sparse_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict_
     }
 }
 
-// grid (Hq, B), DV/4 threads: combines the splits of one head.
+// grid (Hq, B), DV/4 threads: combines the splits of one head.  A split that
+// saw no rows wrote m = -inf, l = 0 and O = 0, so every partial row is read
+// without branching and the loads of all splits are in flight together.
 __global__ void lse_merge_kernel(const float *__restrict__ o_part, const float *__restrict__ m_part,
                                  const float *__restrict__ l_part, int n_splits, int Hq, int DV,
                                  float *__restrict__ out, float *__restrict__ lse) {
     const int h = blockIdx.x, b = blockIdx.y;
+    const size_t row0 = (size_t)b * n_splits * Hq + h;   // partial row of split s: row0 + s * Hq
     float M = -INFINITY;
-    for (int s = 0; s < n_splits; ++s) M = fmaxf(M, m_part[((size_t)b * n_splits + s) * Hq + h]);
+#pragma unroll 8
+    for (int s = 0; s < n_splits; ++s) M = fmaxf(M, __ldg(m_part + row0 + (size_t)s * Hq));
     float L = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     const int c = threadIdx.x * 4;
+    const bool active = c < DV;
+#pragma unroll 8
     for (int s = 0; s < n_splits; ++s) {
-        const size_t idx = ((size_t)b * n_splits + s) * Hq + h;
+        const size_t idx = row0 + (size_t)s * Hq;
         const float ms = m_part[idx];
-        if (ms == -INFINITY) continue;
-        const float wgt = exp2f(ms - M);
+        const float wgt = ms == -INFINITY ? 0.f : exp2f(ms - M);
         L += wgt * l_part[idx];
-        if (c < DV) {
-            float4 v = *reinterpret_cast<const float4 *>(o_part + idx * DV + c);
-            acc.x += wgt * v.x; acc.y += wgt * v.y; acc.z += wgt * v.z; acc.w += wgt * v.w;
-        }
+        const float4 v = active ? __ldcs(reinterpret_cast<const float4 *>(o_part + idx * DV + c))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+        acc.x += wgt * v.x; acc.y += wgt * v.y; acc.z += wgt * v.z; acc.w += wgt * v.w;
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
-    if (c < DV)
+    if (active)
         *reinterpret_cast<float4 *>(out + ((size_t)b * Hq + h) * DV + c) =
             make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
     if (lse && threadIdx.x == 0)
@@ -305,8 +309,7 @@ __global__ void lse_merge_kernel(const float *__restrict__ o_part, const float *
     __syncthreads();
     const int lines = DV * 4 / 128;
     for (int i = threadIdx.x; i < n_splits * lines; i += blockDim.x) {
-        const size_t idx = ((size_t)b * n_splits + i / lines) * Hq + h;
-        const float *line = o_part + idx * DV + (i % lines) * 32;
+        const float *line = o_part + (row0 + (size_t)(i / lines) * Hq) * DV + (i % lines) * 32;
         asm volatile("discard.global.L2 [%0], 128;\n" ::"l"(line) : "memory");
     }
 }
