@@ -43,7 +43,32 @@ def parse():
     p.add_argument("--workload", default=DEFAULT_WORKLOAD)
     p.add_argument("--no-cold", action="store_true", help="skip the 512K cold-pool figure")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--profile-window", action="store_true",
+                   help="no timing: run two eager windows of the workload's kernels on 24K-token contexts "
+                        "(pools of ~230 MB) for a profiler capture, then exit")
     return p.parse_args()
+
+
+def profile_window(args):
+    """Two eager lookahead windows (4 steps each) of the workload's kernels on a reduced
+    context, small enough for an ncu --set full capture.  The attention launch attends
+    the same rows as at full size (top-k plus the 8000-token window); only the number of
+    indexer candidates and the pool size shrink."""
+    import lsa_workloads as W
+    from lsa_workloads.device import host_build, upload
+    from learned_sparse_kv_b200.decode import Shapes, Window
+    wl0 = W.workload(args.workload)
+    wl = W.workload(args.workload, ctx=tuple([24576] * wl0.B), steps=4)
+    host = host_build(wl)
+    shapes, t, max_ch, cap, cold = upload(host, torch.device("cuda:0"))
+    win = Window(Shapes(**shapes), t, max_ch, cap, cold)
+    for _ in range(2):
+        win.run(use_graph=False)
+    torch.cuda.synchronize()
+    status = win.device_status()
+    print(json.dumps({"profile_window": wl.name, "ctx_per_sequence": 24576, "steps": wl.steps, "status": status}))
+    if status != 0:
+        raise SystemExit(1)
 
 
 def peaks():
@@ -165,13 +190,16 @@ def window_bytes(win):
     return att + li + topk + out + sel
 
 
-def sha(path):
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def sha(*paths):
+    h = hashlib.sha256()
+    for path in paths:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel_file):
-    """Per-launch DRAM bytes from the committed ncu summary if it matches the current source."""
+def recorded_traffic(*kernel_files):
+    """Per-launch DRAM bytes from the committed ncu summary if it matches the current sources."""
     path = os.path.join(ROOT, "profiles", "sparse_decode_traffic.txt")
     if not os.path.exists(path):
         return None
@@ -180,7 +208,7 @@ def recorded_traffic(kernel_file):
         if ":" in line and not line.startswith("#"):
             a, b = line.split(":", 1)
             kv[a.strip()] = b.strip()
-    if kv.get("source_sha256_16") != sha(kernel_file):
+    if kv.get("source_sha256_16") != sha(*kernel_files):
         return None
     try:
         return float(kv["dram_bytes_per_launch_full_size"])
@@ -274,7 +302,8 @@ def run_lsa(args, world, rank, local):
     att_bytes, att_rows = attention_bytes(win)
     per_launch = att_bytes / wl.steps
     achieved = per_launch / (att_ms / 1e3) / 1e9
-    traffic = recorded_traffic(os.path.join(ROOT, "learned_sparse_kv_b200", "csrc", "sparse_decode.cu"))
+    csrc = os.path.join(ROOT, "learned_sparse_kv_b200", "csrc")
+    traffic = recorded_traffic(os.path.join(csrc, "sparse_decode.cu"), os.path.join(csrc, "sparse_decode_sm100.cu"))
     wbytes = window_bytes(win)
     window_gbs = wbytes / (ms_local / args.steps / 1e3) / 1e9
 
@@ -451,6 +480,9 @@ def run_reference(args, world, rank):
 
 def main():
     args = parse()
+    if args.profile_window:
+        profile_window(args)
+        return
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":

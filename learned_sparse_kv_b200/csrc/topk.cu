@@ -3,7 +3,7 @@
 // (arXiv 2606.09079: the Lightning Indexer's fine top-k inside the kept set,
 // gist.science explainer 2.1 "Gestufte Selektion", cjcn.com.cn article section 2.)
 //
-// One cluster of 16 CTAs per sequence.  A 4-pass, 8-bit radix select over
+// One cluster of 8 CTAs per sequence.  A 4-pass, 8-bit radix select over
 // order-preserving uint32 keys finds the k-th largest key T and how many of
 // the keys equal to T are taken; an order-preserving scan over the cluster then
 // emits every candidate with key > T and the first `need` candidates with
@@ -15,7 +15,7 @@
 namespace lsa {
 
 constexpr int kTopkThreads = 512;   // threads per CTA
-constexpr int kTopkCtas = 16;       // CTAs per sequence: one thread-block cluster
+constexpr int kTopkCtas = 8;        // CTAs per sequence: one thread-block cluster (8 measured fastest of 1..16)
 
 int launch_li_scores(const uint16_t *, const uint16_t *, const uint16_t *, int64_t, const int32_t *, int,
                      const int32_t *, const int32_t *, int, const int32_t *, const int32_t *, int, int, int, float *,
@@ -54,12 +54,10 @@ __global__ void __launch_bounds__(256) cold_count_kernel(const int32_t *__restri
     }
 }
 
-// Adds 1 to hist[bin] for every lane with `active`, one shared atomic per distinct bin.
+// Adds 1 to hist[bin] for every lane with `active`.  Plain shared atomics:
+// aggregating equal bins across the warp first (match.any) measured slower.
 __device__ __forceinline__ void warp_hist_add(int *hist, uint32_t bin, bool active) {
-    const unsigned act = __ballot_sync(0xffffffffu, active);
-    if (!active) return;
-    const unsigned same = __match_any_sync(act, bin);
-    if ((threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(&hist[bin], __popc(same));
+    if (active) atomicAdd(&hist[bin], 1);
 }
 
 __device__ __forceinline__ int ld_cluster_s32(const void *p, uint32_t rank) {
@@ -200,7 +198,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_scores_kernel(const float *
     topk_cluster(scores + a, n, k, CandIdentity{}, topk_idx + (size_t)b * k, topk_count + b, stage_cap);
 }
 
-// Keys staged per CTA: a slice of at most ceil(max_n / 16), never more than 24,576 (96 KB).
+// Keys staged per CTA: a slice of at most ceil(max_n / 8), never more than 24,576 (96 KB).
 static int stage_capacity(int max_n) { return max(0, min((max_n + kTopkCtas - 1) / kTopkCtas, 24576)); }
 
 // One cluster of kTopkCtas CTAs per sequence.
