@@ -35,6 +35,7 @@ struct __align__(1024) Smem {
     uint64_t q_full[2], q_empty[2];
     uint64_t acc_full[2], acc_empty[2];
     uint64_t mma_done;
+    float w[MAX_H];                                 // head weights of the epilogue's current sequence
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -143,7 +144,32 @@ li_score_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_consta
         int kslot = 0;
         uint32_t kpar = 0;
         int cur_b = -1, qbuf = 1, qswitch = 0;
+        // Pool slots of the chunks of 16 tiles are looked up at once, lane i holding
+        // chunk i & 1 of tile base + i / 2 (the slot count means "zero fill"), and the
+        // next 16 are in flight meanwhile, so the two dependent lookups per chunk
+        // (kept list, then chunk table) stay off the path from one tile to the next.
+        auto lookup = [&](int base) {
+            const int tt = base + (lane >> 1), i = lane & 1;
+            int slot = (int)p.n_slots;
+            if (tt < t1) {
+                const int bb = tile_seq(wk, p.B, tt);
+                const int j = 2 * (tt - wk.tile_off[bb]) + i;
+                if (j < wk.cold[bb]) {
+                    const int chunk = p.kept_idx[(size_t)bb * p.kept_cap + j];
+                    const int sl = (chunk >= 0 && chunk < p.table_stride) ? p.table[(size_t)bb * p.table_stride + chunk] : -1;
+                    if (sl >= 0 && sl < p.n_slots) slot = sl;
+                }
+            }
+            return slot;
+        };
+        int batch = t0, slots = lookup(t0), slots_next = lookup(t0 + 16);
         for (int t = t0; t < t1; ++t) {
+            if (t - batch == 16) {
+                batch += 16;
+                slots = slots_next;
+                slots_next = lookup(batch + 16);
+            }
+            const int s0 = __shfl_sync(0xffffffffu, slots, 2 * (t - batch)), s1 = __shfl_sync(0xffffffffu, slots, 2 * (t - batch) + 1);
             const int b = tile_seq(wk, p.B, t);
             if (b != cur_b) {                              // query heads and weights of a new sequence
                 cur_b = b;
@@ -159,13 +185,10 @@ li_score_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_consta
             if (!bounded(sm, &sm.k_empty[kslot], kpar ^ 1u, p.status)) break;
             if (lane == 0) {
                 const int j0 = 2 * (t - wk.tile_off[b]);
-                const int32_t *kept = p.kept_idx + (size_t)b * p.kept_cap;
                 const int nck = min(2, wk.cold[b] - j0);
                 expect_tx(&sm.k_full[kslot], (uint32_t)(nck * atoms * 64 * 128));
                 for (int i = 0; i < nck; ++i) {
-                    const int chunk = kept[j0 + i];
-                    int slot = (chunk >= 0 && chunk < p.table_stride) ? p.table[(size_t)b * p.table_stride + chunk] : -1;
-                    if (slot < 0 || slot >= p.n_slots) slot = (int)p.n_slots;   // out of range: zero fill
+                    const int slot = i ? s1 : s0;   // out of range (no slot): zero fill
                     for (int a = 0; a < atoms; ++a)
                         tma_load_2d_local(sm.keys[kslot][a] + i * 64 * 128, &key_map, 64 * a, slot * LSA_CHUNK,
                                           &sm.k_full[kslot]);
@@ -221,9 +244,23 @@ li_score_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_consta
         const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
         const int row = 32 * (warp & 3) + lane;               // TMEM lane = token row of the tile
         bool ok = true;
+        int w_b = -1;
         for (int t = t0, u = 0; t < t1; ++t, ++u) {
             const int b = tile_seq(wk, p.B, t);
-            const uint16_t *wb = p.w_li + (size_t)b * p.H;
+            if (b != w_b) {   // head weights of a new sequence into shared memory
+                named_barrier(1, 128);   // the previous weights are no longer read
+                for (int h = L; h < p.H; h += 128) sm.w[h] = bf16_to_f32(p.w_li[(size_t)b * p.H + h]);
+                named_barrier(1, 128);
+                w_b = b;
+            }
+            // the row's chunk and slot are looked up while the MMA runs
+            const int j0 = 2 * (t - wk.tile_off[b]);
+            const int jj = j0 + (row >> 6);
+            int slot = -1;
+            if (jj < wk.cold[b]) {
+                const int chunk = p.kept_idx[(size_t)b * p.kept_cap + jj];
+                slot = (chunk >= 0 && chunk < p.table_stride) ? p.table[(size_t)b * p.table_stride + chunk] : -1;
+            }
             const int ab = u & 1;
             if (ok) ok = bounded(sm, &sm.acc_full[ab], (u >> 1) & 1, p.status);
             tc_fence_after();
@@ -234,17 +271,13 @@ li_score_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_consta
                 tmem_ld32(base + c0, v);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) acc += bf16_to_f32(wb[c0 + i]) * fmaxf(__uint_as_float(v[i]), 0.f);
+                for (int i = 0; i < 32; ++i) acc += sm.w[c0 + i] * fmaxf(__uint_as_float(v[i]), 0.f);
             }
             tc_fence_before();
             named_barrier(1, 128);
             if (L == 0) arrive(&sm.acc_empty[ab]);
             // write the score of this row if it belongs to a kept cold chunk of the sequence
-            const int j0 = 2 * (t - wk.tile_off[b]);
-            const int jj = j0 + (row >> 6);
             if (ok && jj < wk.cold[b]) {
-                const int chunk = p.kept_idx[(size_t)b * p.kept_cap + jj];
-                const int slot = (chunk >= 0 && chunk < p.table_stride) ? p.table[(size_t)b * p.table_stride + chunk] : -1;
                 const bool valid = slot >= 0 && slot < p.n_slots;
                 if (!valid && (row & 63) == 0) flag(p.status, LSA_DEV_TABLE);
                 p.scores[((size_t)b * p.kept_cap + jj) * LSA_CHUNK + (row & 63)] = valid ? acc : -INFINITY;
