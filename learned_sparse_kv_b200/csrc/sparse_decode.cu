@@ -273,45 +273,74 @@ sparse_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict_
     }
 }
 
-// grid (Hq, B), DV/4 threads: combines the splits of one head.  A split that
-// saw no rows wrote m = -inf, l = 0 and O = 0, so every partial row is read
-// without branching and the loads of all splits are in flight together.
-__global__ void lse_merge_kernel(const float *__restrict__ o_part, const float *__restrict__ m_part,
-                                 const float *__restrict__ l_part, int n_splits, int Hq, int DV,
-                                 float *__restrict__ out, float *__restrict__ lse) {
-    const int h = blockIdx.x, b = blockIdx.y;
+// Combines the split-K partials of each head (the log-sum-exp merge).  DV / 8
+// threads per head, two float4 columns each, 128 threads per CTA: grid
+// (Hq / heads per CTA, B).  A split that saw no rows wrote m = -inf, l = 0 and
+// O = 0, so every partial row is read without branching.  The loads of up to
+// MERGE_GROUP splits are issued together before any arithmetic; a longer split
+// list is taken group by group, rescaling the running sums to the new maximum.
+constexpr int MERGE_GROUP = 10;
+
+template <int DV>
+__global__ void __launch_bounds__(128, 4) lse_merge_kernel(const float *__restrict__ o_part,
+                                                        const float *__restrict__ m_part,
+                                                        const float *__restrict__ l_part, int n_splits, int Hq,
+                                                        float *__restrict__ out, float *__restrict__ lse) {
+    constexpr int TPH = DV / 8, HPB = 128 / TPH;
+    const int t = threadIdx.x % TPH, h = blockIdx.x * HPB + threadIdx.x / TPH, b = blockIdx.y;
+    if (h >= Hq) return;
     const size_t row0 = (size_t)b * n_splits * Hq + h;   // partial row of split s: row0 + s * Hq
-    float M = -INFINITY;
-#pragma unroll 8
-    for (int s = 0; s < n_splits; ++s) M = fmaxf(M, __ldg(m_part + row0 + (size_t)s * Hq));
-    float L = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    const int c = threadIdx.x * 4;
-    const bool active = c < DV;
-#pragma unroll 8
-    for (int s = 0; s < n_splits; ++s) {
-        const size_t idx = row0 + (size_t)s * Hq;
-        const float ms = m_part[idx];
-        const float wgt = ms == -INFINITY ? 0.f : exp2f(ms - M);
-        L += wgt * l_part[idx];
-        const float4 v = active ? __ldcs(reinterpret_cast<const float4 *>(o_part + idx * DV + c))
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-        acc.x += wgt * v.x; acc.y += wgt * v.y; acc.z += wgt * v.z; acc.w += wgt * v.w;
+    float M = -INFINITY, L = 0.f;
+    float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+    for (int s0 = 0; s0 < n_splits; s0 += MERGE_GROUP) {
+        float4 v0[MERGE_GROUP], v1[MERGE_GROUP];
+        float ms[MERGE_GROUP], ls[MERGE_GROUP];
+#pragma unroll
+        for (int j = 0; j < MERGE_GROUP; ++j) {
+            if (s0 + j < n_splits) {
+                const size_t idx = row0 + (size_t)(s0 + j) * Hq;
+                const float4 *src = reinterpret_cast<const float4 *>(o_part + idx * DV);
+                v0[j] = __ldcs(src + t);
+                v1[j] = __ldcs(src + TPH + t);
+                ms[j] = __ldg(m_part + idx);
+                ls[j] = __ldg(l_part + idx);
+            } else {
+                v0[j] = v1[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+                ms[j] = -INFINITY;
+                ls[j] = 0.f;
+            }
+        }
+        float Mn = M;
+#pragma unroll
+        for (int j = 0; j < MERGE_GROUP; ++j) Mn = fmaxf(Mn, ms[j]);
+        const float r = M == -INFINITY ? 0.f : exp2f(M - Mn);   // the sums so far are 0 while M = -inf
+        L *= r;
+        a0.x *= r; a0.y *= r; a0.z *= r; a0.w *= r;
+        a1.x *= r; a1.y *= r; a1.z *= r; a1.w *= r;
+#pragma unroll
+        for (int j = 0; j < MERGE_GROUP; ++j) {
+            const float w = ms[j] == -INFINITY ? 0.f : exp2f(ms[j] - Mn);
+            L += w * ls[j];
+            a0.x += w * v0[j].x; a0.y += w * v0[j].y; a0.z += w * v0[j].z; a0.w += w * v0[j].w;
+            a1.x += w * v1[j].x; a1.y += w * v1[j].y; a1.z += w * v1[j].z; a1.w += w * v1[j].w;
+        }
+        M = Mn;
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
-    if (active)
-        *reinterpret_cast<float4 *>(out + ((size_t)b * Hq + h) * DV + c) =
-            make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-    if (lse && threadIdx.x == 0)
+    float4 *dst = reinterpret_cast<float4 *>(out + ((size_t)b * Hq + h) * DV);
+    dst[t] = make_float4(a0.x * inv, a0.y * inv, a0.z * inv, a0.w * inv);
+    dst[TPH + t] = make_float4(a1.x * inv, a1.y * inv, a1.z * inv, a1.w * inv);
+    if (lse && t == 0)
         lse[(size_t)b * Hq + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
-    // The partial rows of this head are dead now: drop their L2 lines without
-    // writing them back, so split-K scratch costs no DRAM write bandwidth.
-    __syncthreads();
-    const int lines = DV * 4 / 128;
-    for (int i = threadIdx.x; i < n_splits * lines; i += blockDim.x) {
-        const float *line = o_part + (row0 + (size_t)(i / lines) * Hq) * DV + (i % lines) * 32;
-        asm volatile("discard.global.L2 [%0], 128;\n" ::"l"(line) : "memory");
-    }
+}
+
+template <int DV>
+static int launch_merge(const float *o_part, const float *m_part, const float *l_part, int n_splits, int Hq, int B,
+                        float *out, float *lse, cudaStream_t stream) {
+    constexpr int HPB = 128 / (DV / 8);
+    lse_merge_kernel<DV><<<dim3((Hq + HPB - 1) / HPB, B), 128, 0, stream>>>(o_part, m_part, l_part, n_splits, Hq,
+                                                                           out, lse);
+    return check_launch("lse_merge_kernel");
 }
 
 using CfgSep16 = DecodeCfg<16, 128, 128, 4, false>;
@@ -437,6 +466,6 @@ extern "C" int lsa_sparse_decode(const lsa_bf16 *q, const lsa_bf16 *k_pool, int6
                                     topk_idx, topk_count, k, window_start, window_len, B, Hq, scale, ns, o_part, m_part,
                                     l_part, dev_status, stream);
     if (rc) return rc;
-    lse_merge_kernel<<<dim3(Hq, B), dv / 4, 0, stream>>>(o_part, m_part, l_part, ns, Hq, dv, out, lse);
-    return check_launch("lse_merge_kernel");
+    return dv == 512 ? launch_merge<512>(o_part, m_part, l_part, ns, Hq, B, out, lse, stream)
+                     : launch_merge<128>(o_part, m_part, l_part, ns, Hq, B, out, lse, stream);
 }
