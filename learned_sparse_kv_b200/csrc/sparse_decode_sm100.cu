@@ -22,14 +22,15 @@
 // fetches a CTA's K rows (36 KB) and a 4D box {64, 64 rows, 2, 2} its value
 // columns (32 KB), both straight into the 128-byte-swizzled operand layout.
 // Gathered tiles (top-k rows, and window tiles that are not a whole aligned
-// chunk) are copied by a warpgroup with 16-byte cp.async into the same layout;
+// chunk) are copied by two warpgroups with 16-byte cp.async into the same layout;
 // missing rows are zero-filled.  Two stages of each operand are in flight.
 // Warp roles:
 //   0      K producer (TMA), tile-validity masks
 //   1      S = Q K^T issuer (even CTA)        2   O += P V issuer (even CTA)
 //   3      TMEM allocator, V producer (TMA)
 //   4..7   softmax, O rescale, epilogue (one thread per TMEM lane)
-//   8..11  row gather for gathered tiles
+//   8..15  row gather for gathered tiles (256 threads: the copy rate of one
+//          multiprocessor grows with the number of copying warps)
 // The online softmax is evaluated in the log2 domain; the reference maximum
 // is only moved when a row maximum grows by more than 2^8, which keeps P <= 256
 // in bf16 and makes O rescales rare.  Every mbarrier wait is bounded: on
@@ -51,8 +52,8 @@ constexpr int NTILE = 64;         // kv rows per tile
 constexpr int KCH = DQK / 64;     // 9 column chunks of 64
 constexpr int STAGES = 2;         // tiles in flight per operand
 constexpr int INFO = 4;           // tile-validity ring
-constexpr int THREADS = 384;
-constexpr int GATHER_THREADS = 128;
+constexpr int THREADS = 512;
+constexpr int GATHER_THREADS = 256;
 constexpr uint32_t Q_BYTES = KCH * HPC * 128;          // per CTA
 constexpr uint32_t K_BYTES = KCH * 32 * 128;           // per CTA and tile
 constexpr uint32_t V_BYTES = 2 * 2 * NTILE * 128;      // per CTA and tile
@@ -361,7 +362,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         __syncwarp();
     } else if (warp >= 8 && n_tiles > 0) {
         // ------------------------------------------------ row gather (cp.async)
-        // Thread g copies 16-byte pieces: K pieces q = g + 128 i of the CTA's 32
+        // Thread g copies 16-byte pieces: K pieces q = g + 256 i of the CTA's 32
         // rows x 72 pieces, V pieces of 64 rows x 4 value atoms x 8 pieces.  A
         // tile is signalled once its copies (and those of the tile before) have
         // landed: after the next tile's K copies are issued when the next
@@ -394,8 +395,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             if (!ok) break;
             const int32_t *gr = sm.grow[s];
             const uint32_t kb = smem_addr(sm.k[s][0]);
-#pragma unroll 6
-            for (int i = 0; i < 18; ++i) {
+#pragma unroll
+            for (int i = 0; i < 32 * 72 / GATHER_THREADS; ++i) {
                 const int q = g + GATHER_THREADS * i;   // < 32 x 72
                 const int row = q / 72, w = q - row * 72;
                 const int32_t pr = gr[32 * (int)rank + row];
@@ -418,8 +419,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             ok = group_wait(sm, &sm.v_go[gi & 1], (gi >> 1) & 1, p.status, g);
             if (!ok) break;
             const uint32_t vb = smem_addr(sm.v[s][0][0]);
-#pragma unroll 4
-            for (int i = 0; i < 16; ++i) {
+#pragma unroll
+            for (int i = 0; i < 64 * 32 / GATHER_THREADS; ++i) {
                 const int q = g + GATHER_THREADS * i;   // < 64 x 32
                 const int row = q >> 5, w = q & 31, a = w >> 3, pp = w & 7;   // a = 2 j + atom
                 const int32_t pr = gr[row];
