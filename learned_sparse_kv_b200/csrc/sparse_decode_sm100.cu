@@ -225,6 +225,15 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
     // chunk-aligned window tiles) are thereby spread evenly over the splits.
     const int n_tiles = split < st.total ? (st.total - 1 - split) / p.n_splits + 1 : 0;
     const int u0 = split, ustride = p.n_splits;
+    // The split's gathered top-k tiles come first in its share; the first window
+    // tile is moved ahead of them, so the tensor pipe starts on a TMA-loaded tile
+    // while the gathered rows are being copied.
+    const int n_gath = min(n_tiles, split < st.t_topk ? (st.t_topk - 1 - split) / ustride + 1 : 0);
+    const bool lead = n_gath > 0 && n_gath < n_tiles;
+    auto tile_of = [&](int u) {
+        const int k = !lead ? u : (u == 0 ? n_gath : (u <= n_gath ? u - 1 : u));
+        return u0 + k * ustride;
+    };
 
     // Every tile's stage is waited for by its producer in tile order: a parity wait is
     // only unambiguous one phase behind the barrier, so the gather warpgroup (which
@@ -241,10 +250,10 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         }
         // row indices of the next gathered tile are loaded while the current tile is issued
         int64_t n0 = -1, n1 = -1;
-        if (kprod && st.gathered(u0)) { n0 = st.row(p, b, u0, lane); n1 = st.row(p, b, u0, lane + 32); }
+        if (kprod && st.gathered(tile_of(0))) { n0 = st.row(p, b, tile_of(0), lane); n1 = st.row(p, b, tile_of(0), lane + 32); }
         int gi = 0;   // gathered tiles handed to the gather warpgroup so far
         for (int u = 0; u < n_tiles; ++u) {
-            const int t = u0 + u * ustride;
+            const int t = tile_of(u);
             const bool gath = st.gathered(t);
             const int64_t slot_row = gath ? -2 : st.window_slot_row(p, b, t);
             // an unmapped slot is read out of range: TMA fills zeros
@@ -253,9 +262,9 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             const uint32_t par = ((u >> 1) + 1) & 1;
             if (kprod) {
                 const int64_t g0 = n0, g1 = n1;
-                if (u + 1 < n_tiles && st.gathered(t + ustride)) {
-                    n0 = st.row(p, b, t + ustride, lane);
-                    n1 = st.row(p, b, t + ustride, lane + 32);
+                if (u + 1 < n_tiles && st.gathered(tile_of(u + 1))) {
+                    n0 = st.row(p, b, tile_of(u + 1), lane);
+                    n1 = st.row(p, b, tile_of(u + 1), lane + 32);
                 }
                 unsigned long long mask;
                 if (!gath) {
@@ -370,7 +379,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         const int g = threadIdx.x - 256;
         auto next_gathered = [&](int u) {
             for (; u < n_tiles; ++u)
-                if (st.gathered(u0 + u * ustride)) return u;
+                if (st.gathered(tile_of(u))) return u;
             return n_tiles;
         };
         auto signal = [&](int s) {
@@ -383,14 +392,14 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             }
         };
         int u = next_gathered(0);
-        int32_t nxt = (u < n_tiles && g < NTILE) ? gather_row(st, p, b, u0 + u * ustride, g) : -1;
+        int32_t nxt = (u < n_tiles && g < NTILE) ? gather_row(st, p, b, tile_of(u), g) : -1;
         int pending = -1, gi = 0;
         bool ok = true;
         while (u < n_tiles) {
             const int s = u & 1;
             if (g < NTILE) sm.grow[s][g] = nxt;   // unmapped rows are flagged by the producer warp
             const int un = next_gathered(u + 1);
-            if (un < n_tiles && g < NTILE) nxt = gather_row(st, p, b, u0 + un * ustride, g);
+            if (un < n_tiles && g < NTILE) nxt = gather_row(st, p, b, tile_of(un), g);
             ok = group_wait(sm, &sm.k_go[gi & 1], (gi >> 1) & 1, p.status, g);   // also publishes grow[s]
             if (!ok) break;
             const int32_t *gr = sm.grow[s];
