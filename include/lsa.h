@@ -128,6 +128,11 @@ int lsa_topk(const lsa_bf16 *q_li, const lsa_bf16 *w_li, const lsa_bf16 *li_pool
              int32_t *topk_idx, int32_t *topk_count, float *scores, int32_t *dev_status,
              void *ws, size_t ws_bytes, lsa_stream_t stream);
 size_t lsa_topk_workspace_size(int B, int kept_cap);
+/* Kernels one lsa_topk call launches for these sizes: 2 where the tcgen05
+ * indexer kernel serves the shape (Hl in {32, 64, 128}, dl in {64, 128},
+ * B <= 64) and counts the kept cold chunks in its own prologue, else 3 (a
+ * counting kernel first); 0 for sizes that lsa_topk rejects.  Host only. */
+int lsa_topk_kernel_count(int B, int Hl, int dl);
 
 /*
  * a3 alone, on given fp32 scores (exact unit entry point).

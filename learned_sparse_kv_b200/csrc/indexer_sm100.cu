@@ -44,7 +44,9 @@ struct Params {
     const uint16_t *w_li;
     const int32_t *table;
     const int32_t *kept_idx;
-    const int32_t *cold;          // kept chunks before the window, per sequence
+    const int32_t *kept_count;
+    const int32_t *window_start;
+    int32_t *cold;                // out: kept chunks before the window, per sequence (written by CTA 0)
     float *scores;
     int32_t *status;
     int64_t n_slots;
@@ -83,12 +85,30 @@ struct Work {
     int first, last;    // tile range of this CTA
 };
 
+// Every CTA counts, per sequence, the kept chunks that lie before the recent
+// window (they hold the indexer's candidates): warp w takes sequences w, w + 6, ...
+// CTA 0 also writes the counts out for the top-k pass that follows.
+__device__ void count_cold(const Params &p, Work &wk, int warp, int lane) {
+    for (int b = warp; b < p.B; b += THREADS / 32) {
+        const int cnt = min(max(p.kept_count[b], 0), p.kept_cap);
+        const int fw = p.window_start[b] / LSA_CHUNK;
+        const int32_t *kept = p.kept_idx + (size_t)b * p.kept_cap;
+        int c = 0;
+#pragma unroll 8
+        for (int i = lane; i < cnt; i += 32) c += kept[i] < fw;
+        c = __reduce_add_sync(0xffffffffu, c);
+        if (lane == 0) {
+            wk.cold[b] = c;
+            if (blockIdx.x == 0) p.cold[b] = c;
+        }
+    }
+}
+
 __device__ void build_work(const Params &p, Work &wk) {
     if (threadIdx.x == 0) {
         int acc = 0;
         for (int b = 0; b < p.B; ++b) {
             wk.tile_off[b] = acc;
-            wk.cold[b] = p.cold[b];
             acc += (wk.cold[b] + 1) >> 1;
         }
         wk.tile_off[p.B] = acc;
@@ -130,12 +150,14 @@ li_score_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_consta
         sm.abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
-    build_work(p, wk);
+    count_cold(p, wk, warp, lane);
     if (warp == 1) asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
                                     smem_addr(&sm.tmem_base)), "r"(256));
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    build_work(p, wk);
+    __syncthreads();
     const uint32_t tmem = sm.tmem_base;
     const int t0 = wk.first, t1 = wk.last;
 
@@ -321,15 +343,16 @@ bool shape_ok(int H, int D, int B) { return (H == 32 || H == 64 || H == 128) && 
 
 int launch(const uint16_t *q_li, const uint16_t *w_li, const uint16_t *li_pool, int64_t n_slots, const int32_t *table,
            int table_stride, const int32_t *kept_idx, const int32_t *kept_count, int kept_cap,
-           const int32_t *cold, int B, int H, int D, float *scores, int32_t *status, cudaStream_t stream) {
+           const int32_t *window_start, int32_t *cold, int B, int H, int D, float *scores, int32_t *status,
+           cudaStream_t stream) {
     CUtensorMap key_map, q_map;
     if (!make_map(&key_map, li_pool, D, (uint64_t)n_slots * LSA_CHUNK, LSA_CHUNK))
         return fail(LSA_ERR_CUDA, "lsa_topk: cuTensorMapEncodeTiled failed for the indexer key pool");
     if (!make_map(&q_map, q_li, D, (uint64_t)B * H, H))
         return fail(LSA_ERR_CUDA, "lsa_topk: cuTensorMapEncodeTiled failed for the indexer queries");
     Params prm;
-    (void)kept_count;
-    prm.w_li = w_li; prm.table = table; prm.kept_idx = kept_idx; prm.cold = cold; prm.scores = scores; prm.status = status; prm.n_slots = n_slots;
+    prm.w_li = w_li; prm.table = table; prm.kept_idx = kept_idx; prm.kept_count = kept_count;
+    prm.window_start = window_start; prm.cold = cold; prm.scores = scores; prm.status = status; prm.n_slots = n_slots;
     prm.B = B; prm.H = H; prm.D = D; prm.table_stride = table_stride; prm.kept_cap = kept_cap;
     const size_t smem = sizeof(Smem) + 1024;
     LSA_CUDA(cudaFuncSetAttribute(li_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));

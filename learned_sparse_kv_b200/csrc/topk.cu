@@ -18,9 +18,10 @@ constexpr int kTopkThreads = 512;   // threads per CTA
 constexpr int kTopkCtas = 8;        // CTAs per sequence: one thread-block cluster (8 measured fastest of 1..16)
 
 int launch_li_scores(const uint16_t *, const uint16_t *, const uint16_t *, int64_t, const int32_t *, int,
-                     const int32_t *, const int32_t *, int, const int32_t *, const int32_t *, int, int, int, float *,
+                     const int32_t *, const int32_t *, int, const int32_t *, int32_t *, int, int, int, float *,
                      int32_t *, cudaStream_t);
 bool indexer_shape_ok(int H, int D);
+bool indexer_counts_cold(int H, int D, int B);
 
 struct CandFromKept {   // candidate j -> token position kept[j / 64] * 64 + j % 64
     const int32_t *kept;
@@ -257,15 +258,23 @@ extern "C" int lsa_topk(const lsa_bf16 *q_li, const lsa_bf16 *w_li, const lsa_bf
     int32_t *cold = c.take<int32_t>((size_t)B);
     float *buf = c.take<float>((size_t)B * kept_cap * LSA_CHUNK);
     if (scores) buf = scores;
-    cold_count_kernel<<<B, 256, 0, stream>>>(kept_idx, kept_count, kept_cap, window_start, cold);
-    int rc = check_launch("cold_count_kernel");
-    if (rc) return rc;
+    int rc = LSA_OK;
+    if (!indexer_counts_cold(Hl, dl, B)) {
+        cold_count_kernel<<<B, 256, 0, stream>>>(kept_idx, kept_count, kept_cap, window_start, cold);
+        rc = check_launch("cold_count_kernel");
+        if (rc) return rc;
+    }
     rc = launch_li_scores(q_li, w_li, li_pool, n_slots, chunk_table, table_stride, kept_idx, kept_count, kept_cap,
                           window_start, cold, B, Hl, dl, buf, dev_status, stream);
     if (rc) return rc;
     const int cap = stage_capacity(kept_cap * LSA_CHUNK);
     return launch_topk(topk_kept_kernel, B, cap, stream, "topk_kept_kernel", (const float *)buf, kept_cap,
                        kept_idx, (const int32_t *)cold, k, topk_idx, topk_count, cap);
+}
+
+extern "C" int lsa_topk_kernel_count(int B, int Hl, int dl) {
+    if (B <= 0 || !indexer_shape_ok(Hl, dl)) return 0;
+    return indexer_counts_cold(Hl, dl, B) ? 2 : 3;
 }
 
 extern "C" int lsa_topk_from_scores(const float *scores, const int64_t *cand_offset, int B, int max_cand, int k,

@@ -160,8 +160,11 @@ class Window:
             self.steps()
 
     def launches_per_window(self) -> int:
-        """Kernels this library launches per window (select: 2; per step: append 1, top-k 3, decode 2)."""
-        return 2 + self.s.steps * 6
+        """Kernels this library launches per window (select: 2; per step: append 1, top-k 2 or 3, decode 2).
+
+        The top-k call counts the kept cold chunks inside the tcgen05 indexer kernel when
+        that kernel serves the indexer shape, else in a kernel of its own."""
+        return 2 + self.s.steps * (1 + lsa.topk_kernel_count(self.s.B, self.s.Hl, self.s.dl) + 2)
 
     def device_status(self) -> int:
         return int(self.status.item())

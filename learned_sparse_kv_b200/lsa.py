@@ -36,6 +36,7 @@ def _load():
         "lsa_nmi_select_workspace_size": ([I, I], SZ),
         "lsa_topk": ([P, P, P, I64, P, I, P, P, I, P, I, I, I, I, P, P, P, P, P, SZ, P], I),
         "lsa_topk_workspace_size": ([I, I], SZ),
+        "lsa_topk_kernel_count": ([I, I, I], I),
         "lsa_topk_from_scores": ([P, P, I, I, I, P, P, P, SZ, P], I),
         "lsa_sparse_decode": ([P, P, I64, P, I64, I64, P, I, P, P, I, P, P, I, I, I, I, I, F, P, P, P, P, SZ, P], I),
         "lsa_sparse_decode_workspace_size": ([I, I, I, I, I, I], SZ),
@@ -120,6 +121,10 @@ def nmi_select(q, w, khat, seq_chunk_offset, max_chunks_per_seq, kept_cap, *, lo
 
 def topk_workspace_size(B, kept_cap):
     return _lib.lsa_topk_workspace_size(B, kept_cap)
+
+
+def topk_kernel_count(B, Hl, dl):
+    return _lib.lsa_topk_kernel_count(B, Hl, dl)
 
 
 def topk(q_li, w_li, li_pool, chunk_table, kept_idx, kept_count, window_start, k, *, scores=None, status=None,
