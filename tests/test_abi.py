@@ -97,3 +97,18 @@ def test_workspace_queries_are_host_only(lib):
     assert lib.lsa_label_vote_workspace_size(32, 64, 2048) == 64 * 2048 * 4
     assert lib.lsa_topk_workspace_size(8, 2048) >= 8 * 2048 * 64 * 4 + 8 * 4
     assert lib.lsa_nmi_select_workspace_size(8, 2048) >= 8 * 32 * 8
+
+
+def test_topk_kernel_count_follows_the_indexer_shape(lib):
+    # The tcgen05 indexer (Hl in {32, 64, 128}, dl in {64, 128}, B <= 64) counts the kept cold
+    # chunks itself: 2 kernels per lsa_topk call; other accepted shapes add a counting kernel.
+    assert lib.lsa_topk_kernel_count(8, 64, 128) == 2
+    assert lib.lsa_topk_kernel_count(1, 32, 64) == 2
+    assert lib.lsa_topk_kernel_count(64, 128, 128) == 2
+    assert lib.lsa_topk_kernel_count(65, 64, 128) == 3
+    assert lib.lsa_topk_kernel_count(1, 8, 64) == 3
+    assert lib.lsa_topk_kernel_count(8, 48, 128) == 3
+    # shapes lsa_topk rejects
+    assert lib.lsa_topk_kernel_count(8, 7, 128) == 0
+    assert lib.lsa_topk_kernel_count(8, 64, 96) == 0
+    assert lib.lsa_topk_kernel_count(0, 64, 128) == 0
