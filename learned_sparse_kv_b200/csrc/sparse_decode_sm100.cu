@@ -173,7 +173,7 @@ __device__ __forceinline__ bool warp_wait_cluster(Smem &sm, const uint64_t *bar,
     return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
-// Gather-warpgroup-uniform bounded wait: one thread polls, the group agrees by barrier reduction.
+// Gather-group-uniform bounded wait: one thread polls, the group agrees by barrier reduction.
 __device__ __forceinline__ bool group_wait(Smem &sm, const uint64_t *bar, uint32_t parity, int32_t *status, int g) {
     bool ok = true;
     if (g == 0) {
@@ -236,7 +236,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
     };
 
     // Every tile's stage is waited for by its producer in tile order: a parity wait is
-    // only unambiguous one phase behind the barrier, so the gather warpgroup (which
+    // only unambiguous one phase behind the barrier, so the gather group (which
     // skips the TMA tiles) is handed its stages through k_go / v_go, whose phases count
     // gathered tiles only.  K (warp 0) and V (warp 3) have a producer each, so K of a
     // later tile never waits behind the P.V that frees a V stage.
@@ -251,7 +251,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         // row indices of the next gathered tile are loaded while the current tile is issued
         int64_t n0 = -1, n1 = -1;
         if (kprod && st.gathered(tile_of(0))) { n0 = st.row(p, b, tile_of(0), lane); n1 = st.row(p, b, tile_of(0), lane + 32); }
-        int gi = 0;   // gathered tiles handed to the gather warpgroup so far
+        int gi = 0;   // gathered tiles handed to the gather group so far
         for (int u = 0; u < n_tiles; ++u) {
             const int t = tile_of(u);
             const bool gath = st.gathered(t);
