@@ -103,6 +103,10 @@ __device__ void topk_cluster(const float *__restrict__ s, int n, int k, PosFn po
     if (staged)
         for (int i = t; i < len; i += kTopkThreads) keys[i] = ordered_key(s[j0 + i]);
     auto key = [&](int i) { return staged ? keys[i] : ordered_key(s[j0 + i]); };
+    if (t < 256) {
+        sh.hist[0][t] = 0;
+        sh.hist[1][t] = 0;
+    }
     __syncthreads();
 
     uint32_t prefix = 0, pmask = 0;
@@ -111,19 +115,20 @@ __device__ void topk_cluster(const float *__restrict__ s, int n, int k, PosFn po
 #pragma unroll 1
     for (int pass = 0; pass < 4; ++pass) {
         const int shift = 24 - 8 * pass;
-        // hist[pass & 1] was last read by the other CTAs before the previous pass's
-        // cluster barrier, which this CTA has passed.
-        int *hist = sh.hist[pass & 1];
-        if (t < 256) hist[t] = 0;
-        __syncthreads();
+        int *hist = sh.hist[pass & 1];   // zeroed, and ordered before these adds by a block barrier
         for (int i = t; i < len_round; i += kTopkThreads) {
             const uint32_t u = i < len ? key(i) : 0u;
             warp_hist_add(hist, (u >> shift) & 255u, i < len && (u & pmask) == prefix);
         }
         sm100::cluster_sync();   // every CTA's histogram of this pass is complete
         int v = 0;               // suffix counts over digits, highest digit first
-        if (t < 256)
+        if (t < 256) {
             for (int r = 0; r < kTopkCtas; ++r) v += ld_cluster_s32(&hist[255 - t], (uint32_t)r);
+            // The other buffer serves the next pass: every CTA finished reading it
+            // (in the previous pass) before the cluster barrier above.  Pass 1 finds
+            // it zero from the start.
+            if (pass >= 1 && pass < 3) sh.hist[(pass + 1) & 1][t] = 0;
+        }
         int total;
         const int excl = block_exclusive_scan<kTopkThreads>(v, sh.warp_tot, &total);
         if (t < 256 && excl < remaining && excl + v >= remaining) {
@@ -131,10 +136,9 @@ __device__ void topk_cluster(const float *__restrict__ s, int n, int k, PosFn po
             sh.remaining = remaining - excl;
         }
         __syncthreads();
-        prefix = sh.prefix;
+        prefix = sh.prefix;   // rewritten only after the next pass's barriers
         remaining = sh.remaining;
         pmask |= 255u << shift;
-        __syncthreads();
     }
     const uint32_t T = prefix;
     const int need_eq = remaining;  // keys equal to T that are taken, >= 1
@@ -152,15 +156,28 @@ __device__ void topk_cluster(const float *__restrict__ s, int n, int k, PosFn po
     (void)block_exclusive_scan<kTopkThreads>(gt, sh.warp_tot, &gt_tot);
     if (t == 0) { sh.cnt[0] = gt_tot; sh.cnt[1] = eq_tot; }
     sm100::cluster_sync();   // every CTA's counts are published
-    if (t == 0) {
-        int base = 0, eq_lower = 0;
-        for (int r = 0; r < c; ++r) {
-            const int g_r = ld_cluster_s32(&sh.cnt[0], (uint32_t)r), e_r = ld_cluster_s32(&sh.cnt[1], (uint32_t)r);
-            base += g_r + min(e_r, max(0, need_eq - eq_lower));
-            eq_lower += e_r;
+    if (t < 32) {
+        // Lane r < c reads CTA r's counts (all remote loads in flight at once); CTA r
+        // contributes its keys above T and its share of the keys equal to T, which go
+        // to the lowest CTAs first (eq_before_r = keys equal to T in CTAs below r).
+        int g_r = 0, e_r = 0;
+        if (t < c) {
+            g_r = ld_cluster_s32(&sh.cnt[0], (uint32_t)t);
+            e_r = ld_cluster_s32(&sh.cnt[1], (uint32_t)t);
         }
-        sh.base = base;
-        sh.eq_lower = eq_lower;
+        int e_incl = e_r;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, e_incl, o);
+            if (t >= o) e_incl += y;
+        }
+        const int eq_before_r = e_incl - e_r;
+        const int base = __reduce_add_sync(0xffffffffu, g_r + min(e_r, max(0, need_eq - eq_before_r)));
+        const int eq_lower = __reduce_add_sync(0xffffffffu, e_r);
+        if (t == 0) {
+            sh.base = base;
+            sh.eq_lower = eq_lower;
+        }
     }
     __syncthreads();
     int take_eq = min(eq, max(0, need_eq - (sh.eq_lower + eq_before)));
