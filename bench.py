@@ -303,7 +303,7 @@ def run_lsa(args, world, rank, local):
     per_launch = att_bytes / wl.steps
     achieved = per_launch / (att_ms / 1e3) / 1e9
     csrc = os.path.join(ROOT, "learned_sparse_kv_b200", "csrc")
-    traffic = recorded_traffic(os.path.join(csrc, "sparse_decode.cu"), os.path.join(csrc, "sparse_decode_sm100.cu"))
+    traffic = recorded_traffic(*(os.path.join(csrc, f) for f in ("sparse_decode_sm100.cu", "sm100.cuh", "common.cuh")))
     wbytes = window_bytes(win)
     window_gbs = wbytes / (ms_local / args.steps / 1e3) / 1e9
 

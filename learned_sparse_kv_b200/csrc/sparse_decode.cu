@@ -279,6 +279,8 @@ sparse_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict_
 // O = 0, so every partial row is read without branching.  The loads of up to
 // MERGE_GROUP splits are issued together before any arithmetic; a longer split
 // list is taken group by group, rescaling the running sums to the new maximum.
+// A group of 10 keeps the kernel within 128 registers (four CTAs per
+// multiprocessor), so the 512 CTAs of an 8-sequence, 128-head merge are one wave.
 constexpr int MERGE_GROUP = 10;
 
 template <int DV>
