@@ -14,6 +14,8 @@
 // columns, 128-byte swizzle) into a 3-stage ring; the per-sequence query heads
 // live in two buffers so a CTA can cross a sequence boundary without a stall.
 // Warp roles: 0 TMA producer, 1 MMA issuer (also allocates TMEM), 2..5 epilogue.
+// In the prologue every warp counts the kept cold chunks of some sequences (the
+// tile list is built from those counts; CTA 0 also writes them for the top-k).
 #include <cuda.h>
 
 #include "common.cuh"
