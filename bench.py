@@ -336,14 +336,19 @@ def run_lsa(args, world, rank, local):
 
 def run_e2e(win, wl, args, world):
     """Same metric through the public API with host buffers: per decode step the step's
-    inputs go host->device from pinned memory and the attention output comes back."""
+    inputs go host->device from pinned memory and the attention output comes back.
+
+    The copies run on a side stream and overlap the steps, as a serving loop would run
+    them: step s + 1's inputs land in the second of two input buffers while step s
+    computes, and step s's output is copied back while step s + 1 computes.  A window
+    ends when its last output is on the host."""
     from learned_sparse_kv_b200 import lsa
     t, sh = win.t, win.s
     S = wl.steps
     keys = ["q_li", "w_li", "q", "new_li"] + (["new_kv"] if sh.latent else ["new_k", "new_v"])
     host_in = {k: t[k].cpu().pin_memory() for k in keys}
     host_sel = {k: t[k].cpu().pin_memory() for k in ("q_nmi", "w_nmi")}
-    dev_in = {k: torch.empty_like(t[k][0]) for k in keys}
+    dev_in = [{k: torch.empty_like(t[k][0]) for k in keys} for _ in range(2)]
     host_out = torch.empty(S, *win.out.shape[1:], dtype=torch.float32).pin_memory()
     h2d = sum(host_in[k][0].numel() * host_in[k].element_size() for k in keys) * S + \
         sum(v.numel() * v.element_size() for v in host_sel.values())
@@ -352,18 +357,30 @@ def run_e2e(win, wl, args, world):
     graphs = []
     torch.cuda.synchronize()
     for s in range(S):
+        d = dev_in[s % 2]
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            lsa.append_token(dev_in["new_kv"] if sh.latent else dev_in["new_k"], None if sh.latent else dev_in["new_v"],
-                             dev_in["new_li"], win.k_pool, win.v_pool, t["li"], t["chunk_table"], t["window_start"],
+            lsa.append_token(d["new_kv"] if sh.latent else d["new_k"], None if sh.latent else d["new_v"],
+                             d["new_li"], win.k_pool, win.v_pool, t["li"], t["chunk_table"], t["window_start"],
                              win.window_len, status=win.status)
-            lsa.topk(dev_in["q_li"], dev_in["w_li"], t["li"], t["chunk_table"], win.kept_idx, win.kept_count,
+            lsa.topk(d["q_li"], d["w_li"], t["li"], t["chunk_table"], win.kept_idx, win.kept_count,
                      t["window_start"], sh.k, scores=win.scores, status=win.status, topk_idx=win.topk_idx[s],
                      topk_count=win.topk_count[s], ws=win.ws_topk)
-            lsa.sparse_decode(dev_in["q"], win.k_pool, win.v_pool, t["chunk_table"], win.topk_idx[s],
+            lsa.sparse_decode(d["q"], win.k_pool, win.v_pool, t["chunk_table"], win.topk_idx[s],
                               win.topk_count[s], t["window_start"], win.window_len, win.max_window_len, sh.dv,
                               sh.scale, out=win.out[s], lse=win.lse[s], status=win.status, ws=win.ws_decode)
         graphs.append(g)
+
+    compute = torch.cuda.current_stream()
+    copy = torch.cuda.Stream()
+    inputs_ready = [torch.cuda.Event() for _ in range(S)]
+    step_done = [torch.cuda.Event() for _ in range(S)]
+
+    def h2d_step(s):
+        with torch.cuda.stream(copy):
+            for k in keys:
+                dev_in[s % 2][k].copy_(host_in[k][s], non_blocking=True)
+            inputs_ready[s].record(copy)
 
     def one_window():
         t["q_nmi"].copy_(host_sel["q_nmi"], non_blocking=True)
@@ -371,15 +388,26 @@ def run_e2e(win, wl, args, world):
         win.reset()
         if win.cold is None:
             win.select()
+        copy.wait_stream(compute)   # the previous window's steps are done with both input buffers
+        h2d_step(0)
         for s in range(S):
-            for k in keys:
-                dev_in[k].copy_(host_in[k][s], non_blocking=True)
+            if s + 1 < S:
+                if s >= 1:
+                    copy.wait_event(step_done[s - 1])   # buffer (s + 1) % 2 was read by step s - 1
+                h2d_step(s + 1)
+            compute.wait_event(inputs_ready[s])
             graphs[s].replay()
-            host_out[s].copy_(win.out[s], non_blocking=True)
+            step_done[s].record(compute)
+            with torch.cuda.stream(copy):
+                copy.wait_event(step_done[s])
+                host_out[s].copy_(win.out[s], non_blocking=True)
+        compute.wait_stream(copy)
 
     for _ in range(args.warmup):
         one_window()
     torch.cuda.synchronize()
+    if args.warmup > 0 and not torch.equal(host_out, win.out.cpu()):
+        raise RuntimeError("end-to-end run: the outputs copied to the host differ from the device outputs")
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
