@@ -262,6 +262,9 @@ size_t lsa_label_vote_workspace_size(int n_layers, int n_steps, int n_chunks);
  *     before voting.
  *   - The first call on a device looks up the array's device address with
  *     that device current; make that first call before any stream capture.
+ *     The address is kept for the life of the process: after a
+ *     cudaDeviceReset of that device it is stale, so do not call this entry
+ *     point on that device again in the same process.
  *   - Every call shares the one array: calls whose GPU work overlaps (on
  *     different streams, or from different threads) race and must be ordered
  *     by the caller.

@@ -220,6 +220,9 @@ static uint32_t *g_vote_scratch_dev[64];   // device address of g_vote_scratch, 
 
 // Host code may not use g_vote_scratch itself (it names a host-side stand-in);
 // the device address is looked up once per device, with that device current.
+// The cached address belongs to the device's context at that time: after a
+// cudaDeviceReset of the device it is stale, and this entry point must not be
+// called on that device again in the same process.
 static int vote_scratch(uint32_t **out) {
     int dev = 0;
     LSA_CUDA(cudaGetDevice(&dev));

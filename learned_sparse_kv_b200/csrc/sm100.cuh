@@ -1,6 +1,6 @@
 // sm100.cuh -- thin inline-PTX wrappers for the Blackwell (sm_100a) pieces used by
 // the attention kernel: mbarriers with bounded waits, cluster addressing, TMA
-// tensor loads (tile and gather4), tcgen05 TMEM allocation / MMA / commit /
+// tensor loads (tile mode), tcgen05 TMEM allocation / MMA / commit /
 // loads and stores, and the shared-memory matrix descriptors for UMMA.
 #pragma once
 
@@ -153,17 +153,8 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32
 
 // ---------------------------------------------------------------- TMA -----
 
-// 2D tile load of box at (x, y) into this CTA's shared memory; completion is
+// 3D / 4D tile loads of a box into this CTA's shared memory; completion is
 // counted on an mbarrier that may live in the peer CTA (cta_group::2).
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint32_t mbar_cluster) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.cta_group::2"
-        " [%0], [%1, {%2, %3}], [%4];\n" ::"r"(smem_addr(dst)),
-        "l"(map), "r"(x), "r"(y), "r"(mbar_cluster)
-        : "memory");
-}
-
-// 3D / 4D boxes, same completion rule.
 __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int x, int y, int z, uint32_t mbar_cluster) {
     asm volatile(
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.cta_group::2"
@@ -178,21 +169,6 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, i
         " [%0], [%1, {%2, %3, %4, %5}], [%6];\n" ::"r"(smem_addr(dst)),
         "l"(map), "r"(x), "r"(y), "r"(z), "r"(w), "r"(mbar_cluster)
         : "memory");
-}
-
-// Four rows y0..y3 of width box-x at column x; the map's box is one row high.
-__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, int x, int y0, int y1, int y2, int y3,
-                                            uint32_t mbar_cluster) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes.cta_group::2"
-        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];\n" ::"r"(smem_addr(dst)),
-        "l"(map), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(mbar_cluster)
-        : "memory");
-}
-
-// Fetches `bytes` (a multiple of 16) at a 16-byte aligned global address into L2.
-__device__ __forceinline__ void l2_prefetch(const void *src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(src), "r"(bytes) : "memory");
 }
 
 // ------------------------------------------------------------- tcgen05 ----

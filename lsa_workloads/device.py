@@ -4,10 +4,15 @@ Two phases so that a test can adjust inputs between them:
   host = host_build(wl)          numpy bf16 bits, one array per pool in device-slot layout
   dev = upload(host, device)     torch tensors for learned_sparse_kv_b200.decode.Window
 
-The host pools already hold the rows of the tokens appended during the window
-(positions ctx .. ctx+steps-1); the device append writes the same values again.
-For a cold workload the device pools hold only the window chunks, and
-host["oracle_pools"] / host["oracle_table"] give the fully resident view.
+host["pools"] is what goes to the device.  Its rows for the tokens appended
+during the window (positions ctx .. ctx+steps-1) hold bf16 NaN: only the
+device append can give them their values, so an append that writes nothing or
+writes the wrong row shows up in every later step that attends the row.
+host["oracle_pools"] / host["oracle_table"] are the oracle's view: every chunk
+resident, the appended rows already in place (for a resident workload the
+appended chunk of sequence b sits in an extra trailing slot n_slots + b that is
+never uploaded).  For a cold workload the device pools hold only the window
+chunks and the oracle view is the whole host pool.
 """
 import numpy as np
 import torch
@@ -47,8 +52,23 @@ def _write_new_rows(wl, pools, table, st, steps):
             pools["li"][slot, row] = st["new_li"][s, b]
 
 
+BF16_NAN = np.uint16(0x7FC0)
+
+
+def _poison_new_rows(wl, pools, table, steps):
+    """bf16 NaN in the device rows of the tokens appended during the window."""
+    for s in range(steps):
+        for b in range(wl.B):
+            pos = wl.ctx[b] + s
+            slot, row = table[b, pos // CHUNK], pos % CHUNK
+            for k in pools:
+                pools[k][slot, row] = BF16_NAN
+
+
 def host_build(wl: Workload, steps: int = None, nmi=None, structural: bool = True, fetch_fraction: float = 0.25):
     steps = wl.steps if steps is None else steps
+    assert all(L % CHUNK == 0 and L >= wl.window for L in wl.ctx), "contexts are whole chunks, at least the window"
+    assert steps <= CHUNK, "one lookahead window appends at most one chunk"
     nm = nmi if nmi is not None else nmi_inputs(wl, structural=structural)
     st = stacked_steps(wl, steps)
     host = dict(wl=wl, steps=steps, nmi=nm, step=st, max_chunks=max(wl.n_ch), kept_cap=max(wl.n_ch))
@@ -62,13 +82,19 @@ def host_build(wl: Workload, steps: int = None, nmi=None, structural: bool = Tru
         otab = np.arange(wl.n_ch[0] + 1, dtype=np.int32)[None, :]
         opools = {k: np.concatenate([hp[k], np.zeros((1,) + hp[k].shape[1:], np.uint16)]) for k in _kinds(wl)}
         _write_new_rows(wl, opools, otab, st, steps)
-        _write_new_rows(wl, host["pools"], lay["chunk_table"], st, steps)
+        _poison_new_rows(wl, host["pools"], lay["chunk_table"], steps)
         host.update(oracle_pools=opools, oracle_table=otab, first_window_chunk=fw, first_free_slot=lay["fetch_base"])
     else:
         lay = resident_layout(wl)
-        host["pools"] = kv_pools(wl, lay)
-        _write_new_rows(wl, host["pools"], lay["chunk_table"], st, steps)
-        host.update(oracle_pools=host["pools"], oracle_table=lay["chunk_table"])
+        n = lay["n_slots"]
+        full = kv_pools(wl, lay, extra_slots=wl.B)
+        host["pools"] = {k: v[:n] for k, v in full.items()}      # views: the device part
+        otab = lay["chunk_table"].copy()
+        for b in range(wl.B):
+            otab[b, wl.n_ch[b]] = n + b                            # appended chunk, oracle view only
+        _write_new_rows(wl, full, otab, st, steps)
+        _poison_new_rows(wl, host["pools"], lay["chunk_table"], steps)
+        host.update(oracle_pools=full, oracle_table=otab)
     host["chunk_table"] = lay["chunk_table"]
     host["window_start"] = np.asarray(lay["window_start"], np.int32)
     return host

@@ -218,18 +218,19 @@ def chunk_rows(wl: Workload, b: int, c0: int, c1: int, kind: str) -> np.ndarray:
     return out
 
 
-def kv_pools(wl: Workload, layout, chunks_of=None):
+def kv_pools(wl: Workload, layout, chunks_of=None, extra_slots: int = 0):
     """Fills device-pool arrays for a layout from chunk_rows().
 
-    Returns dict(kv or k+v, li) uint16 arrays [n_slots, 64, width].  Slots that
-    hold no chunk stay zero.  `chunks_of(b)` may restrict the chunks written.
+    Returns dict(kv or k+v, li) uint16 arrays [n_slots + extra_slots, 64, width].
+    Slots that hold no chunk stay zero.  `chunks_of(b)` may restrict the chunks
+    written.
     """
     kinds = ["kv", "li"] if wl.latent else ["k", "v", "li"]
     pools = {}
     table = layout["chunk_table"]
     for kind in kinds:
         width = {"kv": wl.dqk, "k": wl.dqk, "v": wl.dv, "li": wl.dl}[kind]
-        pool = np.zeros((layout["n_slots"], CHUNK, width), np.uint16)
+        pool = np.zeros((layout["n_slots"] + extra_slots, CHUNK, width), np.uint16)
         for b in range(wl.B):
             n_ch = wl.n_ch[b]
             chunks = np.arange(n_ch) if chunks_of is None else np.asarray(chunks_of(b))

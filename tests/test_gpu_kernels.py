@@ -180,8 +180,10 @@ def _decode_case(L, wl, kept, host, s, topk_override=None, table_override=None):
         sel = r["topk"][:r["topk_count"]] if topk_override is None else topk_override[b]
         tk[b, :len(sel)] = sel
         tc[b] = len(sel)
-    pools = host["pools"]
-    table = host["chunk_table"] if table_override is None else table_override
+    # the oracle's view of the pools: it holds the rows of the tokens appended during the
+    # window, which these direct attention calls attend without running the append
+    pools = host["oracle_pools"]
+    table = host["oracle_table"] if table_override is None else table_override
     wlen = np.full(B, wl.window + s + 1, np.int32)
     status = torch.zeros(1, dtype=torch.int32, device=d)
     out, lse = L.sparse_decode(bf16(st["q"][s], d), bf16(pools["kv"] if wl.latent else pools["k"], d),
@@ -231,7 +233,7 @@ def test_sparse_decode_skips_rows_without_slot_and_flags(L):
     sel = [H.oracle_step(host, kept[b], b, 0) for b in range(wl.B)]
     sel = [r["topk"][:r["topk_count"]] for r in sel]
     gone = int(sel[0][0]) // CH                       # this chunk loses its slot
-    table = host["chunk_table"].copy()
+    table = host["oracle_table"].copy()
     table[0, gone] = -1
     out, _, _, st = _decode_case(L, wl, kept, host, 0, topk_override=sel, table_override=table)
     assert st & L.DEV_TABLE
@@ -355,6 +357,54 @@ def test_append_writes_rows_and_advances_window(L):
     for b, pos in enumerate([127, 64, 133]):
         slot = int(table[b, pos // CH])
         assert torch.equal(kv[slot, pos % CH], nk[b]) and torch.equal(li[slot, pos % CH], nl[b])
+
+
+def test_append_cold_layout_fills_appended_chunk_across_the_boundary(L):
+    """Cold layout (window chunks in slots 0..7, the appended chunk in slot 8, fetch area
+    after it): 65 appends starting at the last row of the last window chunk write row 63 of
+    slot 7, then rows 0..63 of slot 8, and nothing else."""
+    d = dev()
+    wl = W.workload("decode_512k_b1_mla_cold", ctx=(40 * CH,), window=8 * CH, steps=1)
+    lay = W.cold_layout(wl, kept_cap=4)
+    assert lay["fetch_base"] == 9 and lay["chunk_table"][0, wl.n_ch[0]] == 8
+    n_slots = lay["n_slots"]
+    kv = torch.full((n_slots, CH, 576), float("nan"), dtype=torch.bfloat16, device=d)
+    li = torch.full((n_slots, CH, 128), float("nan"), dtype=torch.bfloat16, device=d)
+    table = i32(lay["chunk_table"], d)
+    wstart = i32(lay["window_start"], d)
+    wlen = torch.tensor([wl.window - 1], dtype=torch.int32, device=d)
+    g = torch.Generator(device="cpu").manual_seed(3)
+    nk = torch.randn(65, 1, 576, generator=g).to(torch.bfloat16).to(d)
+    nl = torch.randn(65, 1, 128, generator=g).to(torch.bfloat16).to(d)
+    status = torch.zeros(1, dtype=torch.int32, device=d)
+    for i in range(65):
+        L.append_token(nk[i], None, nl[i], kv, None, li, table, wstart, wlen, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0 and wlen.item() == wl.window + 64
+    assert torch.equal(kv[7, 63], nk[0, 0]) and torch.equal(li[7, 63], nl[0, 0])
+    assert torch.equal(kv[8], nk[1:, 0]) and torch.equal(li[8], nl[1:, 0])
+    untouched = torch.ones(n_slots, CH, dtype=torch.bool)
+    untouched[7, 63] = False
+    untouched[8] = False
+    assert bool(torch.isnan(kv.float().cpu()[untouched]).all()) and bool(torch.isnan(li.float().cpu()[untouched]).all())
+
+
+def test_append_past_the_last_slot_flags_and_writes_nothing(L):
+    """A position whose chunk has no slot (-1 in the table) sets LSA_DEV_TABLE, leaves the
+    pools unchanged and does not advance the window."""
+    d = dev()
+    kv = torch.zeros(2, CH, 576, dtype=torch.bfloat16, device=d)
+    li = torch.zeros(2, CH, 128, dtype=torch.bfloat16, device=d)
+    table = torch.tensor([[0, 1, -1]], dtype=torch.int32, device=d)
+    wstart = torch.tensor([0], dtype=torch.int32, device=d)
+    wlen = torch.tensor([128], dtype=torch.int32, device=d)
+    status = torch.zeros(1, dtype=torch.int32, device=d)
+    L.append_token(torch.ones(1, 576, dtype=torch.bfloat16, device=d), None,
+                   torch.ones(1, 128, dtype=torch.bfloat16, device=d), kv, None, li, table, wstart, wlen,
+                   status=status)
+    torch.cuda.synchronize()
+    assert status.item() & L.DEV_TABLE
+    assert wlen.item() == 128 and not bool(kv.any()) and not bool(li.any())
 
 
 def test_gather_copies_kept_cold_chunks(L):

@@ -7,9 +7,12 @@ offers lsa_label_vote_noalloc, which keeps its vote masks in a fixed array built
 into the library instead of a caller workspace.
 
 These tests call it through the C ABI and compare it with lsa_label_vote (which
-takes a caller workspace) on two consecutive calls with different inputs, so a
-mask left over from the first call would show up in the second.  Labels and
-vote counts are integers and must match exactly.
+takes a caller workspace) and with the oracle, on two consecutive calls with
+different inputs, so a mask left over from the first call would show up in the
+second.  The inputs get the same nucleus-margin repair as the other vote tests
+(no cumulative sum within 2e-5 of top_p), so the fp32 GPU path and the fp64
+oracle take every nucleus cut the same way.  Labels and vote counts are
+integers and must match exactly.
 """
 import ctypes
 
@@ -18,6 +21,8 @@ import pytest
 import torch
 
 import lsa_workloads as W
+import oracle
+from tests import helpers as H
 
 pytestmark = pytest.mark.gpu
 
@@ -48,13 +53,17 @@ def test_noalloc_vote_matches_workspace_vote_on_two_calls():
              (p["seed"] + 1, 1, 20, 40, 1500)]                        # a different, smaller problem next
     for seed, mode, L, T, N in cases:
         d = W.label_vote_scores(L, T, N, min(p["planted"], N // 4), seed)
+        H.repair_vote_margin(d, p["top_p"])
         scores = torch.from_numpy(d["scores"]).cuda()
+        oracle_labels, oracle_votes = oracle.label_vote(d["scores"], p["top_p"], p["min_layers"], mode)
         ref_labels, ref_votes = lsa.label_vote(scores, p["top_p"], p["min_layers"], mode)
         rc, labels, votes = _call(fn, scores, p["top_p"], p["min_layers"], mode)
         torch.cuda.synchronize()
         assert rc == 0, lsa._lib.lsa_last_error().decode()
         assert torch.equal(votes, ref_votes)
         assert torch.equal(labels, ref_labels)
+        np.testing.assert_array_equal(votes.cpu().numpy(), oracle_votes)
+        np.testing.assert_array_equal(labels.cpu().numpy(), oracle_labels)
         assert 0 < int(ref_labels.sum()) < N
 
 
