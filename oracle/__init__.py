@@ -34,6 +34,8 @@ def _load():
         c_int, c_double, c_i64 = ctypes.c_int, ctypes.c_double, ctypes.c_int64
         lib.lsao_nmi_select.argtypes = [_u16p, _u16p, _u16p, _i64p, c_int, c_int, c_int,
                                         _i32p, _i32p, c_int, _f64p, _f64p]
+        lib.lsao_nmi_select_union.argtypes = [c_int, ctypes.POINTER(_u16p), ctypes.POINTER(_u16p),
+                                              ctypes.POINTER(_u16p), _i64p, c_int, c_int, c_int, _i32p, _i32p, c_int]
         lib.lsao_li_scores.argtypes = [_u16p, _u16p, _u16p, c_int, c_int, c_int, _f64p]
         lib.lsao_topk_select.argtypes = [_f64p, c_int, c_int, _i32p, _i32p]
         lib.lsao_topk_select_f32.argtypes = [_f32p, c_int, c_int, _i32p, _i32p]
@@ -46,7 +48,7 @@ def _load():
                                          _i32p, _i32p, _f64p, _i32p, _f64p, _f64p]
         lib.lsao_nucleus.argtypes = [_f32p, c_int, c_double, _u8p]
         lib.lsao_label_vote.argtypes = [_f32p, c_int, c_int, c_int, c_double, c_int, c_int, _u8p, _i32p]
-        for name in ("lsao_nmi_select", "lsao_li_scores", "lsao_topk_select", "lsao_topk_select_f32",
+        for name in ("lsao_nmi_select", "lsao_nmi_select_union", "lsao_li_scores", "lsao_topk_select", "lsao_topk_select_f32",
                      "lsao_attention_dense", "lsao_decode_step", "lsao_nucleus", "lsao_label_vote"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
@@ -85,6 +87,26 @@ def nmi_select(q, w, khat, seq_chunk_offset, kept_cap=None):
                                  _p(kept, _i32p), _p(cnt, _i32p), kept_cap, _p(logits, _f64p), _p(probs, _f64p))
     lists = [kept[b, :min(int(cnt[b]), kept_cap)].copy() for b in range(B)]
     return lists, logits[:total], probs[:total], rc, cnt
+
+
+def nmi_select_union(qs, ws, khats, seq_chunk_offset, kept_cap=None):
+    """OR-mode union of independent indexers: lists of q [B,Hn,dn], w [B,Hn], khat [sum n_ch, dn].
+
+    Returns (kept list per sequence, status, counts)."""
+    qs, ws, khats = [_u16(a) for a in qs], [_u16(a) for a in ws], [_u16(a) for a in khats]
+    n = len(qs)
+    assert n == len(ws) == len(khats) and n >= 1
+    off = np.ascontiguousarray(seq_chunk_offset, dtype=np.int64)
+    B, Hn, dn = qs[0].shape
+    if kept_cap is None:
+        kept_cap = int(np.max(np.diff(off))) if B else 0
+    kept = np.full((B, max(kept_cap, 1)), -1, np.int32)
+    cnt = np.zeros(B, np.int32)
+    arr = lambda xs: (_u16p * n)(*[_p(x, _u16p) for x in xs])
+    rc = _load().lsao_nmi_select_union(n, arr(qs), arr(ws), arr(khats), _p(off, _i64p), B, Hn, dn,
+                                       _p(kept, _i32p), _p(cnt, _i32p), kept_cap)
+    lists = [kept[b, :min(int(cnt[b]), kept_cap)].copy() for b in range(B)]
+    return lists, rc, cnt
 
 
 def li_scores(q_li, w_li, keys):

@@ -17,11 +17,16 @@
  *               (periodic trigger tau=64, lookahead index score I_{t,s},
  *               sigmoid gating, fetch of every entry with I >= 0.5, staged
  *               Lightning-Indexer top-k inside the fetched set)
+ *   [gist 2.4]  same page, section 2.4 (three independent indexers at layers
+ *               10, 12 and 20, their predictions combined by a union, OR mode)
  *   [gist 2.2]  same page, section 2.2 (softmax -> top-p 0.6 -> at least
  *               theta = 3 layers vote)
  *   [cjcn 2]    cjcn.com.cn article, section 2 (trigger every 64 steps, ReLU
  *               replaced by Sigmoid, threshold 0.5, second-stage top-k, the
  *               most recent 8000 tokens always resident on the GPU)
+ *   [cjcn 4]    same article, section 4 (one independent memory indexer at
+ *               each of layers 10, 12 and 20; a chunk is recalled when any of
+ *               the three scores it at 0.5 or more: "OR-mode routing")
  *   [cjcn 3]    same article, section 3 (cross-layer majority vote labelling:
  *               softmax, nucleus top-p 0.6, selected by at least 3 layers,
  *               golden blocks of all steps in the window merged)
@@ -110,6 +115,50 @@ int lsao_nmi_select(const uint16_t *q, const uint16_t *w, const uint16_t *khat,
             if (logits) logits[first + s] = logit;
             if (probs) probs[first + s] = prob;
             if (prob >= 0.5) {
+                if (count < kept_cap)
+                    kept_idx[(size_t)b * kept_cap + count] = (int32_t)s;
+                else
+                    status = LSAO_ERR_CAPACITY;
+                ++count;
+            }
+        }
+        kept_count[b] = count;
+    }
+    return status;
+}
+
+/*
+ * OR-mode routing over several independent indexers  [cjcn 4] [gist 2.4]:
+ * the deployed configuration places one indexer at each of three layers; each
+ * has its own queries, head weights and compressed keys and scores every chunk
+ * exactly as lsao_nmi_select does, and a chunk is fetched when ANY of them
+ * gives it a score of at least 0.5.  Kept chunk indices are written in
+ * ascending order; capacity is handled as in lsao_nmi_select.
+ *   q[i] [B, Hn, dn], w[i] [B, Hn], khat[i] [total_chunks, dn] for indexer i.
+ */
+int lsao_nmi_select_union(int n_idx, const uint16_t *const *q, const uint16_t *const *w,
+                          const uint16_t *const *khat, const int64_t *seq_chunk_offset, int B,
+                          int Hn, int dn, int32_t *kept_idx, int32_t *kept_count, int kept_cap)
+{
+    int status = LSAO_OK;
+    if (n_idx <= 0 || B < 0 || Hn <= 0 || dn <= 0 || kept_cap < 0)
+        return LSAO_ERR_ARG;
+    for (int b = 0; b < B; ++b) {
+        int64_t first = seq_chunk_offset[b];
+        int64_t n_ch = seq_chunk_offset[b + 1] - first;
+        int count = 0;
+        for (int j = 0; j < kept_cap; ++j)
+            kept_idx[(size_t)b * kept_cap + j] = -1;
+        for (int64_t s = 0; s < n_ch; ++s) {
+            int fetched = 0;
+            for (int i = 0; i < n_idx; ++i) {
+                double logit = nmi_logit(q[i] + (size_t)b * Hn * dn, w[i] + (size_t)b * Hn,
+                                         khat[i] + (size_t)(first + s) * dn, Hn, dn);
+                double prob = 1.0 / (1.0 + exp(-logit));
+                if (prob >= 0.5)
+                    fetched = 1;
+            }
+            if (fetched > 0) {
                 if (count < kept_cap)
                     kept_idx[(size_t)b * kept_cap + count] = (int32_t)s;
                 else

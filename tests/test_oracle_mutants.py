@@ -30,6 +30,10 @@ MUTANTS = {
     "V read with K stride": ("vo[j] = row * (v_pool ? v_row_stride : k_row_stride);", "vo[j] = ko[j];"),
     "nucleus drops crossing element": ("        sel[ord[i].idx] = 1;\n        ++taken;\n        if (cum >= top_p) break;",
                                        "        if (cum >= top_p) break;\n        sel[ord[i].idx] = 1;\n        ++taken;"),
+    "union takes only the first indexer": ("for (int i = 0; i < n_idx; ++i) {", "for (int i = 0; i < 1; ++i) {"),
+    "union becomes intersection": ("                if (prob >= 0.5)\n                    fetched = 1;",
+                                   "                if (prob < 0.5)\n                    fetched = -1;\n"
+                                   "                else if (fetched == 0)\n                    fetched = 1;"),
     "vote threshold strict": ("labels[c] = (uint8_t)(best >= min_layers);", "labels[c] = (uint8_t)(best > min_layers);"),
     "vote counts any step": ("if (count[(size_t)t * n_chunks + c] > best) best = count[(size_t)t * n_chunks + c];",
                              "best += count[(size_t)t * n_chunks + c];"),
@@ -41,6 +45,8 @@ PINS = [
     lambda o: TS.test_nmi_structural_plant_is_recovered_exactly(o),
     lambda o: TS.test_nmi_special_cases(o),
     lambda o: TS.test_nmi_sequences_use_their_own_queries(o),
+    lambda o: TS.test_nmi_union_keeps_exactly_the_union_of_the_plants(o),
+    lambda o: TS.test_nmi_union_each_indexer_alone_keeps_a_different_chunk(o),
     lambda o: TS.test_li_score_odd_part_is_linear(o),
     lambda o: TS.test_li_score_special_cases(o),
     lambda o: TS.test_topk_equals_full_library_sort_with_ties(o, 200, 64),
@@ -73,7 +79,7 @@ def test_pins_catch_planted_mistake(tmp_path, name):
     libpath = _compile_mutant(tmp_path, name, old, new)
     real = oracle._load()
     mutant = ctypes.CDLL(libpath)
-    for fn in ("lsao_nmi_select", "lsao_li_scores", "lsao_topk_select", "lsao_topk_select_f32",
+    for fn in ("lsao_nmi_select", "lsao_nmi_select_union", "lsao_li_scores", "lsao_topk_select", "lsao_topk_select_f32",
                "lsao_attention_dense", "lsao_decode_step", "lsao_nucleus", "lsao_label_vote"):
         getattr(mutant, fn).argtypes = getattr(real, fn).argtypes
         getattr(mutant, fn).restype = ctypes.c_int

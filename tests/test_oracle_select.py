@@ -51,6 +51,71 @@ def test_nmi_probability_is_library_sigmoid_and_gate_is_logit_sign(oracle_mod):
         assert cnt[b] == ref.size
 
 
+# ------------------------------------------- OR-mode union of three indexers --
+
+def _three_indexers(seed=21, B=2, ctx=(16384, 8192), rates=(0.125, 0.2)):
+    wl = W.workload("decode_16k_b1_h16", B=B, ctx=ctx, pass_rate=rates, seed=seed)
+    return wl, [W.nmi_inputs(wl, seed_offset=i) for i in range(3)]
+
+
+def test_nmi_union_keeps_exactly_the_union_of_the_plants(oracle_mod):
+    """Each indexer keeps exactly its planted chunks (by construction of the inputs); the
+    OR-mode union must keep the set union of the three plants, and no other chunk."""
+    _, ns = _three_indexers()
+    kept, rc, cnt = oracle_mod.nmi_select_union([n["q"] for n in ns], [n["w"] for n in ns],
+                                                [n["khat"] for n in ns], ns[0]["seq_chunk_offset"])
+    assert rc == 0
+    for b in range(2):
+        ref = np.union1d(np.union1d(ns[0]["planted"][b], ns[1]["planted"][b]), ns[2]["planted"][b])
+        np.testing.assert_array_equal(kept[b], ref)
+        assert cnt[b] == ref.size
+        assert ref.size > max(n["planted"][b].size for n in ns)     # the plants really differ
+
+
+def test_nmi_union_each_indexer_alone_keeps_a_different_chunk(oracle_mod):
+    """Hand-built: four chunks, one head, width 2; indexer i's keys point along its query only
+    for chunk i, so chunk i is kept by indexer i alone and chunk 3 by none."""
+    one, minus = int(bits(np.float32(1.0))[0]), int(bits(np.float32(-1.0))[0])
+    q = np.array([[[one, 0]]], np.uint16)
+    w = np.array([[one]], np.uint16)
+    off = np.array([0, 4], np.int64)
+    khats = []
+    for i in range(3):
+        k = np.full((4, 2), minus, np.uint16)
+        k[i, 0] = one
+        khats.append(k)
+    kept, rc, cnt = oracle_mod.nmi_select_union([q] * 3, [w] * 3, khats, off)
+    assert rc == 0 and cnt[0] == 3
+    np.testing.assert_array_equal(kept[0], [0, 1, 2])
+    for i in range(3):
+        alone, _, _, _, _ = oracle_mod.nmi_select(q, w, khats[i], off)
+        np.testing.assert_array_equal(alone[0], [i])
+
+
+def test_nmi_union_of_one_indexer_or_identical_indexers_is_the_single_gate(oracle_mod):
+    rng = np.random.default_rng(23)
+    q, w, khat, off = _ragged_nmi(rng)
+    single, _, _, _, _ = oracle_mod.nmi_select(q, w, khat, off)
+    for n in (1, 3):
+        kept, rc, _ = oracle_mod.nmi_select_union([q] * n, [w] * n, [khat] * n, off)
+        for b in range(q.shape[0]):
+            np.testing.assert_array_equal(kept[b], single[b])
+
+
+def test_nmi_union_equals_set_union_of_independent_gates(oracle_mod):
+    """Random, independent indexers on a ragged batch: the union list equals the sorted
+    set union of the three single-indexer lists."""
+    rng = np.random.default_rng(24)
+    sets = [_ragged_nmi(rng) for _ in range(3)]
+    off = sets[0][3]
+    kept, rc, cnt = oracle_mod.nmi_select_union([s[0] for s in sets], [s[1] for s in sets],
+                                                [s[2] for s in sets], off)
+    singles = [oracle_mod.nmi_select(s[0], s[1], s[2], off)[0] for s in sets]
+    for b in range(3):
+        ref = np.union1d(np.union1d(singles[0][b], singles[1][b]), singles[2][b])
+        np.testing.assert_array_equal(kept[b], ref)
+
+
 def test_nmi_structural_plant_is_recovered_exactly(oracle_mod):
     wl = W.workload("decode_16k_b1_h16")
     nm = W.nmi_inputs(wl)
