@@ -101,6 +101,32 @@ int lsa_nmi_select(const lsa_bf16 *q, const lsa_bf16 *w, const lsa_bf16 *khat,
 size_t lsa_nmi_select_workspace_size(int B, int max_chunks_per_seq);
 
 /*
+ * a1, OR mode -- several independent memory indexers gated together.
+ * Passage: cjcn.com.cn article section 4 (one independent indexer at each of
+ * layers 10, 12 and 20; a chunk is recalled when any of the three scores it at
+ * 0.5 or more, "OR-mode routing"); gist.science explainer 2.4 (a union of the
+ * three layers' predictions).
+ *
+ * Indexer i (0 <= i < n_idx) has its own queries q[i] [B, Hn, dn], head
+ * weights w[i] [B, Hn] and compressed keys khat[i] [total_chunks, dn] (all
+ * bf16, device); the ARRAYS q, w, khat of n_idx device pointers are host
+ * memory.  Every indexer scores every chunk as lsa_nmi_select does; chunk s of
+ * sequence b is kept iff at least one indexer's logit is >= 0.  The kept list
+ * is the ascending union; kept_idx, kept_count, kept_cap, dev_status and the
+ * capacity rule are those of lsa_nmi_select.
+ *   logits  [n_idx, total_chunks] fp32 (device, out, optional): each indexer's logits
+ * Supported: 1 <= n_idx <= 4, shapes as lsa_nmi_select (common to all indexers).
+ * n_idx = 1 is exactly lsa_nmi_select.
+ */
+int lsa_nmi_select_union(int n_idx, const lsa_bf16 *const *q, const lsa_bf16 *const *w,
+                         const lsa_bf16 *const *khat, const int64_t *seq_chunk_offset, int B, int Hn, int dn,
+                         int64_t total_chunks, int max_chunks_per_seq,
+                         int32_t *kept_idx, int32_t *kept_count, int kept_cap,
+                         float *logits, int32_t *dev_status,
+                         void *ws, size_t ws_bytes, lsa_stream_t stream);
+size_t lsa_nmi_select_union_workspace_size(int n_idx, int B, int max_chunks_per_seq);
+
+/*
  * a2 + a3 -- Lightning-Indexer scoring and fine top-k inside the kept chunks.
  * Passage: gist.science explainer 2.1 ("Gestufte Selektion"); cjcn.com.cn
  * article section 2 (the native indexer takes a top-k inside the reduced set).

@@ -101,15 +101,29 @@ __device__ void score_tile(IdxSmem &sm, int H) {
 
 // ------------------------------------------------------------------- a1 ----
 
-// grid (tiles of 64 chunks, B).  Writes logits and one 64-bit gate mask per tile.
+// Up to four independent indexers gated together (OR mode): indexer i has its
+// own queries, head weights and compressed keys, and optional logits output.
+constexpr int kMaxIndexers = 4;
+struct NmiSet {
+    const uint16_t *q[kMaxIndexers];
+    const uint16_t *w[kMaxIndexers];
+    const uint16_t *khat[kMaxIndexers];
+    float *logits[kMaxIndexers];
+};
+
+// grid (tiles of 64 chunks, B, indexers).  Writes logits and one 64-bit gate
+// mask per tile; indexer i's masks start at masks + i * B * tiles_per_seq.
 template <int D>
-__global__ void __launch_bounds__(128) nmi_score_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ w,
-                                                        const uint16_t *__restrict__ khat,
-                                                        const int64_t *__restrict__ off, int H, int tiles_per_seq,
-                                                        float *__restrict__ logits, unsigned long long *__restrict__ masks) {
+__global__ void __launch_bounds__(128) nmi_score_kernel(const NmiSet set, const int64_t *__restrict__ off, int H,
+                                                        int tiles_per_seq, unsigned long long *__restrict__ masks) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     IdxSmem &sm = *reinterpret_cast<IdxSmem *>(smem_raw);
-    const int b = blockIdx.y, tile = blockIdx.x;
+    const int b = blockIdx.y, tile = blockIdx.x, ix = blockIdx.z;
+    const uint16_t *__restrict__ q = set.q[ix];
+    const uint16_t *__restrict__ w = set.w[ix];
+    const uint16_t *__restrict__ khat = set.khat[ix];
+    float *__restrict__ logits = set.logits[ix];
+    masks += (size_t)ix * gridDim.y * tiles_per_seq;
     const int64_t first = off[b];
     const int64_t n_ch = off[b + 1] - first;
     const int64_t s0 = (int64_t)tile * kRows;
@@ -141,7 +155,8 @@ __global__ void __launch_bounds__(128) nmi_score_kernel(const uint16_t *__restri
 }
 
 // grid B, 256 threads: gate masks -> ascending kept list, count, capacity flag.
-__global__ void __launch_bounds__(256) nmi_compact_kernel(const unsigned long long *__restrict__ masks,
+// With several indexers a chunk is kept when any of their masks has its bit.
+__global__ void __launch_bounds__(256) nmi_compact_kernel(const unsigned long long *__restrict__ masks, int n_idx,
                                                           const int64_t *__restrict__ off, int tiles_per_seq,
                                                           int32_t *__restrict__ kept_idx, int32_t *__restrict__ kept_count,
                                                           int kept_cap, int32_t *status) {
@@ -156,13 +171,19 @@ __global__ void __launch_bounds__(256) nmi_compact_kernel(const unsigned long lo
     const int per = (n_words + 255) / 256;
     const int w0 = min(n_words, (int)threadIdx.x * per), w1 = min(n_words, w0 + per);
     const unsigned long long *m = masks + (size_t)b * tiles_per_seq;
+    const size_t idx_stride = (size_t)gridDim.x * tiles_per_seq;
+    auto word = [&](int i) {
+        unsigned long long x = m[i];
+        for (int j = 1; j < n_idx; ++j) x |= m[j * idx_stride + i];
+        return x;
+    };
     int mine = 0;
-    for (int i = w0; i < w1; ++i) mine += __popcll(m[i]);
+    for (int i = w0; i < w1; ++i) mine += __popcll(word(i));
     int total;
     int pos = block_exclusive_scan<256>(mine, warp_tot, &total);
     int32_t *out = kept_idx + (size_t)b * kept_cap;
     for (int i = w0; i < w1; ++i) {
-        unsigned long long bits = m[i];
+        unsigned long long bits = word(i);
         while (bits) {
             int bit = __ffsll((long long)bits) - 1;
             bits &= bits - 1;
@@ -258,44 +279,82 @@ bool indexer_shape_ok(int H, int D) { return heads_ok(H) && (D == 64 || D == 128
 
 using namespace lsa;
 
-extern "C" size_t lsa_nmi_select_workspace_size(int B, int max_chunks_per_seq) {
-    if (B <= 0 || max_chunks_per_seq < 0) return 0;
+extern "C" size_t lsa_nmi_select_union_workspace_size(int n_idx, int B, int max_chunks_per_seq) {
+    if (n_idx < 1 || n_idx > kMaxIndexers || B <= 0 || max_chunks_per_seq < 0) return 0;
     Carver c(nullptr);
     int tiles = (max_chunks_per_seq + kRows - 1) / kRows;
-    c.take<unsigned long long>((size_t)B * (tiles > 0 ? tiles : 1));
+    c.take<unsigned long long>((size_t)n_idx * B * (tiles > 0 ? tiles : 1));
     return align_up(c.used, 256);
 }
+
+extern "C" size_t lsa_nmi_select_workspace_size(int B, int max_chunks_per_seq) {
+    return lsa_nmi_select_union_workspace_size(1, B, max_chunks_per_seq);
+}
+
+namespace lsa {
+
+static int nmi_select_impl(const char *who, int n_idx, const NmiSet &set, const int64_t *seq_chunk_offset, int B,
+                           int Hn, int dn, int64_t total_chunks, int max_chunks_per_seq, int32_t *kept_idx,
+                           int32_t *kept_count, int kept_cap, int32_t *dev_status, void *ws, size_t ws_bytes,
+                           cudaStream_t stream) {
+    LSA_REQUIRE(B > 0, LSA_ERR_INVALID_ARG, "%s: B must be positive (got %d)", who, B);
+    for (int i = 0; i < n_idx; ++i)
+        LSA_REQUIRE(set.q[i] && set.w[i] && set.khat[i], LSA_ERR_INVALID_ARG, "%s: null input pointer of indexer %d",
+                    who, i);
+    LSA_REQUIRE(seq_chunk_offset && kept_idx && kept_count, LSA_ERR_INVALID_ARG, "%s: null input or output pointer",
+                who);
+    LSA_REQUIRE(indexer_shape_ok(Hn, dn), LSA_ERR_SHAPE,
+                "%s: unsupported Hn=%d dn=%d (dn in {64,128}, Hn multiple of 8 up to 128)", who, Hn, dn);
+    LSA_REQUIRE(max_chunks_per_seq >= 0 && total_chunks >= 0 && kept_cap >= 1, LSA_ERR_INVALID_ARG,
+                "%s: bad sizes (max_chunks_per_seq=%d total_chunks=%lld kept_cap=%d)", who, max_chunks_per_seq,
+                (long long)total_chunks, kept_cap);
+    const size_t need = lsa_nmi_select_union_workspace_size(n_idx, B, max_chunks_per_seq);
+    LSA_REQUIRE(ws_bytes >= need && ws, LSA_ERR_WORKSPACE, "%s: workspace of %zu bytes, %zu needed", who, ws_bytes,
+                need);
+    const int tiles = max(1, (max_chunks_per_seq + kRows - 1) / kRows);
+    Carver c(ws);
+    auto *masks = c.take<unsigned long long>((size_t)n_idx * B * tiles);
+    const size_t smem = sizeof(IdxSmem);
+    dim3 grid(tiles, B, n_idx);
+    if (dn == 128) {
+        LSA_CUDA(cudaFuncSetAttribute(nmi_score_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+        nmi_score_kernel<128><<<grid, 128, smem, stream>>>(set, seq_chunk_offset, Hn, tiles, masks);
+    } else {
+        LSA_CUDA(cudaFuncSetAttribute(nmi_score_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+        nmi_score_kernel<64><<<grid, 128, smem, stream>>>(set, seq_chunk_offset, Hn, tiles, masks);
+    }
+    int rc = check_launch("nmi_score_kernel");
+    if (rc) return rc;
+    nmi_compact_kernel<<<B, 256, 0, stream>>>(masks, n_idx, seq_chunk_offset, tiles, kept_idx, kept_count, kept_cap,
+                                              dev_status);
+    return check_launch("nmi_compact_kernel");
+}
+
+}  // namespace lsa
 
 extern "C" int lsa_nmi_select(const lsa_bf16 *q, const lsa_bf16 *w, const lsa_bf16 *khat,
                               const int64_t *seq_chunk_offset, int B, int Hn, int dn, int64_t total_chunks,
                               int max_chunks_per_seq, int32_t *kept_idx, int32_t *kept_count, int kept_cap,
                               float *logits, int32_t *dev_status, void *ws, size_t ws_bytes, lsa_stream_t stream) {
-    LSA_REQUIRE(B > 0, LSA_ERR_INVALID_ARG, "lsa_nmi_select: B must be positive (got %d)", B);
-    LSA_REQUIRE(q && w && khat && seq_chunk_offset && kept_idx && kept_count, LSA_ERR_INVALID_ARG,
-                "lsa_nmi_select: null input or output pointer");
-    LSA_REQUIRE(indexer_shape_ok(Hn, dn), LSA_ERR_SHAPE,
-                "lsa_nmi_select: unsupported Hn=%d dn=%d (dn in {64,128}, Hn multiple of 8 up to 128)", Hn, dn);
-    LSA_REQUIRE(max_chunks_per_seq >= 0 && total_chunks >= 0 && kept_cap >= 1, LSA_ERR_INVALID_ARG,
-                "lsa_nmi_select: bad sizes (max_chunks_per_seq=%d total_chunks=%lld kept_cap=%d)",
-                max_chunks_per_seq, (long long)total_chunks, kept_cap);
-    LSA_REQUIRE(ws_bytes >= lsa_nmi_select_workspace_size(B, max_chunks_per_seq) && ws, LSA_ERR_WORKSPACE,
-                "lsa_nmi_select: workspace of %zu bytes, %zu needed", ws_bytes,
-                lsa_nmi_select_workspace_size(B, max_chunks_per_seq));
-    const int tiles = max(1, (max_chunks_per_seq + kRows - 1) / kRows);
-    Carver c(ws);
-    auto *masks = c.take<unsigned long long>((size_t)B * tiles);
-    const size_t smem = sizeof(IdxSmem);
-    dim3 grid(tiles, B);
-    if (dn == 128) {
-        LSA_CUDA(cudaFuncSetAttribute(nmi_score_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-        nmi_score_kernel<128><<<grid, 128, smem, stream>>>(q, w, khat, seq_chunk_offset, Hn, tiles, logits, masks);
-    } else {
-        LSA_CUDA(cudaFuncSetAttribute(nmi_score_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-        nmi_score_kernel<64><<<grid, 128, smem, stream>>>(q, w, khat, seq_chunk_offset, Hn, tiles, logits, masks);
+    NmiSet set = {};
+    set.q[0] = q; set.w[0] = w; set.khat[0] = khat; set.logits[0] = logits;
+    return nmi_select_impl("lsa_nmi_select", 1, set, seq_chunk_offset, B, Hn, dn, total_chunks, max_chunks_per_seq,
+                           kept_idx, kept_count, kept_cap, dev_status, ws, ws_bytes, stream);
+}
+
+extern "C" int lsa_nmi_select_union(int n_idx, const lsa_bf16 *const *q, const lsa_bf16 *const *w,
+                                    const lsa_bf16 *const *khat, const int64_t *seq_chunk_offset, int B, int Hn, int dn,
+                                    int64_t total_chunks, int max_chunks_per_seq, int32_t *kept_idx,
+                                    int32_t *kept_count, int kept_cap, float *logits, int32_t *dev_status, void *ws,
+                                    size_t ws_bytes, lsa_stream_t stream) {
+    LSA_REQUIRE(n_idx >= 1 && n_idx <= kMaxIndexers, LSA_ERR_INVALID_ARG,
+                "lsa_nmi_select_union: n_idx must be 1..%d (got %d)", kMaxIndexers, n_idx);
+    LSA_REQUIRE(q && w && khat, LSA_ERR_INVALID_ARG, "lsa_nmi_select_union: null pointer array");
+    NmiSet set = {};
+    for (int i = 0; i < n_idx; ++i) {
+        set.q[i] = q[i]; set.w[i] = w[i]; set.khat[i] = khat[i];
+        set.logits[i] = logits ? logits + (size_t)i * total_chunks : nullptr;
     }
-    int rc = check_launch("nmi_score_kernel");
-    if (rc) return rc;
-    nmi_compact_kernel<<<B, 256, 0, stream>>>(masks, seq_chunk_offset, tiles, kept_idx, kept_count, kept_cap,
-                                              dev_status);
-    return check_launch("nmi_compact_kernel");
+    return nmi_select_impl("lsa_nmi_select_union", n_idx, set, seq_chunk_offset, B, Hn, dn, total_chunks,
+                           max_chunks_per_seq, kept_idx, kept_count, kept_cap, dev_status, ws, ws_bytes, stream);
 }

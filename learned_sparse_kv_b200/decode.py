@@ -45,6 +45,7 @@ class Window:
 
     tensors (all on one CUDA device unless noted):
       q_nmi [B,Hn,dn], w_nmi [B,Hn], khat [sum n_ch, dn] bf16; seq_chunk_offset [B+1] int64
+      nmi_union (optional): list of (q, w, khat) of several indexers gated in OR mode
       kv or k+v pools [slots,64,w] bf16, li pool [slots,64,dl] bf16
       chunk_table [B, stride] int32; window_start [B] int32
       per-step inputs stacked on dim 0: q_li [S,B,Hl,dl], w_li [S,B,Hl], q [S,B,Hq,dqk],
@@ -73,7 +74,8 @@ class Window:
         self.window_len = torch.full((B,), shapes.window, dtype=torch.int32, device=d)
         self.status = torch.zeros(1, dtype=torch.int32, device=d)
         self.max_window_len = shapes.window + S
-        self.ws_select = torch.empty(max(lsa.nmi_select_workspace_size(B, max_chunks_per_seq), 256),
+        n_idx = len(t["nmi_union"]) if "nmi_union" in t else 1
+        self.ws_select = torch.empty(max(lsa.nmi_select_union_workspace_size(n_idx, B, max_chunks_per_seq), 256),
                                      dtype=torch.uint8, device=d)
         self.scores = torch.empty(B, kept_cap * CHUNK, dtype=torch.float32, device=d)
         self.ws_topk = torch.empty(max(lsa.topk_workspace_size(B, kept_cap), 256), dtype=torch.uint8, device=d)
@@ -95,6 +97,12 @@ class Window:
 
     def select(self):
         t = self.t
+        if "nmi_union" in t:
+            u = t["nmi_union"]
+            lsa.nmi_select_union([x[0] for x in u], [x[1] for x in u], [x[2] for x in u], t["seq_chunk_offset"],
+                                 self.max_chunks, self.kept_cap, status=self.status, kept_idx=self.kept_idx,
+                                 kept_count=self.kept_count, ws=self.ws_select)
+            return
         lsa.nmi_select(t["q_nmi"], t["w_nmi"], t["khat"], t["seq_chunk_offset"], self.max_chunks, self.kept_cap,
                        logits=self.logits, status=self.status, kept_idx=self.kept_idx, kept_count=self.kept_count,
                        ws=self.ws_select)

@@ -34,6 +34,8 @@ def _load():
     sig = {
         "lsa_nmi_select": ([P, P, P, P, I, I, I, I64, I, P, P, I, P, P, P, SZ, P], I),
         "lsa_nmi_select_workspace_size": ([I, I], SZ),
+        "lsa_nmi_select_union": ([I, P, P, P, P, I, I, I, I64, I, P, P, I, P, P, P, SZ, P], I),
+        "lsa_nmi_select_union_workspace_size": ([I, I, I], SZ),
         "lsa_topk": ([P, P, P, I64, P, I, P, P, I, P, I, I, I, I, P, P, P, P, P, SZ, P], I),
         "lsa_topk_workspace_size": ([I, I], SZ),
         "lsa_topk_kernel_count": ([I, I, I], I),
@@ -114,6 +116,36 @@ def nmi_select(q, w, khat, seq_chunk_offset, max_chunks_per_seq, kept_cap, *, lo
     _check(_lib.lsa_nmi_select(_ptr(q), _ptr(w), _ptr(khat), _ptr(seq_chunk_offset), B, Hn, dn, khat.shape[0],
                                max_chunks_per_seq, _ptr(kept_idx), _ptr(kept_count), kept_cap, _ptr(logits),
                                _ptr(status), _ptr(ws), ws.numel(), _stream(stream)))
+    return kept_idx, kept_count
+
+
+def nmi_select_union_workspace_size(n_idx, B, max_chunks_per_seq):
+    return _lib.lsa_nmi_select_union_workspace_size(n_idx, B, max_chunks_per_seq)
+
+
+def nmi_select_union(qs, ws_, khats, seq_chunk_offset, max_chunks_per_seq, kept_cap, *, logits=None, status=None,
+                     kept_idx=None, kept_count=None, ws=None, stream=None):
+    """OR-mode gate of several indexers (lists of q [B,Hn,dn], w [B,Hn], khat [sum n_ch, dn]).
+
+    Returns (kept_idx [B, kept_cap] int32, kept_count [B] int32)."""
+    n = len(qs)
+    if not (n == len(ws_) == len(khats)):
+        raise LSAError(1, "qs, ws and khats must have the same length")
+    for i in range(n):
+        _dev(qs[i], torch.bfloat16, f"qs[{i}]"); _dev(ws_[i], torch.bfloat16, f"ws[{i}]")
+        _dev(khats[i], torch.bfloat16, f"khats[{i}]")
+    _dev(seq_chunk_offset, torch.int64, "seq_chunk_offset")
+    B, Hn, dn = qs[0].shape
+    dev = qs[0].device
+    if kept_idx is None:
+        kept_idx = torch.empty(B, kept_cap, dtype=torch.int32, device=dev)
+    if kept_count is None:
+        kept_count = torch.empty(B, dtype=torch.int32, device=dev)
+    ws = _ws(nmi_select_union_workspace_size(n, B, max_chunks_per_seq), dev, ws)
+    arr = lambda ts: (ctypes.c_void_p * n)(*[t.data_ptr() for t in ts])
+    _check(_lib.lsa_nmi_select_union(n, arr(qs), arr(ws_), arr(khats), _ptr(seq_chunk_offset), B, Hn, dn,
+                                     khats[0].shape[0], max_chunks_per_seq, _ptr(kept_idx), _ptr(kept_count),
+                                     kept_cap, _ptr(logits), _ptr(status), _ptr(ws), ws.numel(), _stream(stream)))
     return kept_idx, kept_count
 
 

@@ -65,13 +65,20 @@ def _poison_new_rows(wl, pools, table, steps):
                 pools[k][slot, row] = BF16_NAN
 
 
-def host_build(wl: Workload, steps: int = None, nmi=None, structural: bool = True, fetch_fraction: float = 0.25):
+def host_build(wl: Workload, steps: int = None, nmi=None, structural: bool = True, fetch_fraction: float = 0.25,
+               n_indexers: int = 1):
+    """Host-side arrays of one window.  With n_indexers > 1 the gate is the OR-mode union of
+    that many independent indexers (host["nmi_union"]: one nmi_inputs() draw each, the
+    first being host["nmi"])."""
     steps = wl.steps if steps is None else steps
     assert all(L % CHUNK == 0 and L >= wl.window for L in wl.ctx), "contexts are whole chunks, at least the window"
     assert steps <= CHUNK, "one lookahead window appends at most one chunk"
     nm = nmi if nmi is not None else nmi_inputs(wl, structural=structural)
     st = stacked_steps(wl, steps)
     host = dict(wl=wl, steps=steps, nmi=nm, step=st, max_chunks=max(wl.n_ch), kept_cap=max(wl.n_ch))
+    if n_indexers > 1:
+        host["nmi_union"] = [nm] + [nmi_inputs(wl, structural=structural, seed_offset=101 * i)
+                                    for i in range(1, n_indexers)]
     if wl.cold:
         lay = cold_layout(wl, kept_cap=int(np.ceil(fetch_fraction * wl.n_ch[0])))
         fw = lay["first_window_chunk"]
@@ -105,6 +112,9 @@ def upload(host, device):
     wl, nm, st = host["wl"], host["nmi"], host["step"]
     t = {"q_nmi": bf16(nm["q"], device), "w_nmi": bf16(nm["w"], device), "khat": bf16(nm["khat"], device),
          "seq_chunk_offset": torch.from_numpy(nm["seq_chunk_offset"]).to(device)}
+    if "nmi_union" in host:
+        t["nmi_union"] = [(bf16(n["q"], device), bf16(n["w"], device), bf16(n["khat"], device))
+                          for n in host["nmi_union"]]
     for key, v in st.items():
         t[key] = bf16(v, device)
     for k, v in host["pools"].items():

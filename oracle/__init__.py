@@ -36,6 +36,8 @@ def _load():
                                         _i32p, _i32p, c_int, _f64p, _f64p]
         lib.lsao_nmi_select_union.argtypes = [c_int, ctypes.POINTER(_u16p), ctypes.POINTER(_u16p),
                                               ctypes.POINTER(_u16p), _i64p, c_int, c_int, c_int, _i32p, _i32p, c_int]
+        lib.lsao_select_baseline.argtypes = [c_int, _i32p, c_int, ctypes.c_uint64, c_int, c_int, _i32p, _i32p,
+                                             c_int]
         lib.lsao_li_scores.argtypes = [_u16p, _u16p, _u16p, c_int, c_int, c_int, _f64p]
         lib.lsao_topk_select.argtypes = [_f64p, c_int, c_int, _i32p, _i32p]
         lib.lsao_topk_select_f32.argtypes = [_f32p, c_int, c_int, _i32p, _i32p]
@@ -48,7 +50,7 @@ def _load():
                                          _i32p, _i32p, _f64p, _i32p, _f64p, _f64p]
         lib.lsao_nucleus.argtypes = [_f32p, c_int, c_double, _u8p]
         lib.lsao_label_vote.argtypes = [_f32p, c_int, c_int, c_int, c_double, c_int, c_int, _u8p, _i32p]
-        for name in ("lsao_nmi_select", "lsao_nmi_select_union", "lsao_li_scores", "lsao_topk_select", "lsao_topk_select_f32",
+        for name in ("lsao_nmi_select", "lsao_nmi_select_union", "lsao_select_baseline", "lsao_li_scores", "lsao_topk_select", "lsao_topk_select_f32",
                      "lsao_attention_dense", "lsao_decode_step", "lsao_nucleus", "lsao_label_vote"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
@@ -105,6 +107,24 @@ def nmi_select_union(qs, ws, khats, seq_chunk_offset, kept_cap=None):
     arr = lambda xs: (_u16p * n)(*[_p(x, _u16p) for x in xs])
     rc = _load().lsao_nmi_select_union(n, arr(qs), arr(ws), arr(khats), _p(off, _i64p), B, Hn, dn,
                                        _p(kept, _i32p), _p(cnt, _i32p), kept_cap)
+    lists = [kept[b, :min(int(cnt[b]), kept_cap)].copy() for b in range(B)]
+    return lists, rc, cnt
+
+
+RECENT, RANDOM = 0, 1
+
+
+def select_baseline(mode, window_start, seed=0, keep_num=1, keep_den=10, kept_cap=None):
+    """Baseline selectors: mode RECENT (no older chunk) or RANDOM (a random keep_num/keep_den
+    of the chunks before each sequence's window).  Returns (kept lists, status, counts)."""
+    ws = np.ascontiguousarray(window_start, dtype=np.int32)
+    B = ws.shape[0]
+    if kept_cap is None:
+        kept_cap = max(1, int(ws.max()) // CHUNK) if B else 1
+    kept = np.full((B, max(kept_cap, 1)), -1, np.int32)
+    cnt = np.zeros(B, np.int32)
+    rc = _load().lsao_select_baseline(int(mode), _p(ws, _i32p), B, ctypes.c_uint64(seed), int(keep_num),
+                                      int(keep_den), _p(kept, _i32p), _p(cnt, _i32p), kept_cap)
     lists = [kept[b, :min(int(cnt[b]), kept_cap)].copy() for b in range(B)]
     return lists, rc, cnt
 

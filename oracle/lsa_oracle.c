@@ -27,6 +27,10 @@
  *   [cjcn 4]    same article, section 4 (one independent memory indexer at
  *               each of layers 10, 12 and 20; a chunk is recalled when any of
  *               the three scores it at 0.5 or more: "OR-mode routing")
+ *   [cjcn 5]    same article, section 5 (results: the baselines are a pure
+ *               sliding window keeping the recent 8K, and random retention of
+ *               10 % of the history chunks; all schemes keep the recent window)
+ *   [gist 4]    same page, section 4 ("Recency Only" and "Random 10%" baselines)
  *   [cjcn 3]    same article, section 3 (cross-layer majority vote labelling:
  *               softmax, nucleus top-p 0.6, selected by at least 3 layers,
  *               golden blocks of all steps in the window merged)
@@ -243,6 +247,72 @@ int lsao_topk_select_f32(const float *scores, int n, int k, int32_t *out, int32_
     int rc = lsao_topk_select(wide, n, k, out, out_count);
     free(wide);
     return rc;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Baseline selectors  [cjcn 5] [gist 4]                                      */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * Output number c (counting from 0) of a SplitMix64 stream started at `seed`
+ * (Steele, Lea and Flood, "Fast splittable pseudorandom number generators",
+ * OOPSLA 2014): the state advances by the golden-ratio increment before each
+ * output, and each output is the state passed through the generator's mixing
+ * function.
+ */
+static uint64_t splitmix64_output(uint64_t seed, uint64_t c)
+{
+    uint64_t z = seed + (c + 1) * 0x9E3779B97F4A7C15ull;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+
+/*
+ * The two baselines the pages compare LSA with.  Every scheme keeps the recent
+ * window; they differ only in the older history, the n_old = window_start / 64
+ * chunks before it.
+ *   mode 0, recency only: no older chunk is kept.
+ *   mode 1, random fraction: exactly m = floor((n_old * keep_num + keep_den / 2)
+ *     / keep_den) older chunks are kept (keep_num / keep_den = 1 / 10 for the
+ *     pages' "random 10 %"), chosen uniformly at random: chunk s of sequence b
+ *     draws u = (output number b * 2^32 + s of SplitMix64(seed)) >> 40, and the
+ *     m chunks with the smallest draws are kept, ties to the lower index.
+ * Kept lists are ascending; capacity as in lsao_nmi_select.
+ */
+int lsao_select_baseline(int mode, const int32_t *window_start, int B, uint64_t seed, int keep_num,
+                         int keep_den, int32_t *kept_idx, int32_t *kept_count, int kept_cap)
+{
+    if ((mode != 0 && mode != 1) || B < 0 || kept_cap < 0 || keep_num < 0 || keep_den <= 0)
+        return LSAO_ERR_ARG;
+    int status = LSAO_OK;
+    for (int b = 0; b < B; ++b) {
+        int32_t *out = kept_idx + (size_t)b * kept_cap;
+        for (int j = 0; j < kept_cap; ++j)
+            out[j] = -1;
+        int n_old = window_start[b] > 0 ? window_start[b] / LSAO_CHUNK : 0;
+        int64_t m = mode == 0 ? 0 : ((int64_t)n_old * keep_num + keep_den / 2) / keep_den;
+        if (m > n_old) m = n_old;
+        if (m == 0) { kept_count[b] = 0; continue; }
+        /* smallest draws first = largest negated draws first, ties to the lower index */
+        double *neg = (double *)malloc(sizeof(double) * (size_t)n_old);
+        int32_t *sel = (int32_t *)malloc(sizeof(int32_t) * (size_t)n_old);
+        int32_t cnt = 0;
+        if (!neg || !sel) { free(neg); free(sel); return LSAO_ERR_ARG; }
+        for (int c = 0; c < n_old; ++c) {
+            uint64_t u = splitmix64_output(seed, ((uint64_t)b << 32) + (uint64_t)c) >> 40;
+            neg[c] = -(double)u;
+        }
+        lsao_topk_select(neg, n_old, (int)m, sel, &cnt);
+        for (int j = 0; j < cnt; ++j) {
+            if (j < kept_cap) out[j] = sel[j];
+            else status = LSAO_ERR_CAPACITY;
+        }
+        kept_count[b] = cnt;
+        free(neg);
+        free(sel);
+    }
+    return status;
 }
 
 /* ------------------------------------------------------------------------- */

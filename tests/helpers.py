@@ -15,6 +15,11 @@ CH = W.CHUNK
 
 
 def kept_lists(host):
+    if "nmi_union" in host:
+        u = host["nmi_union"]
+        lists, rc, cnt = oracle.nmi_select_union([n["q"] for n in u], [n["w"] for n in u], [n["khat"] for n in u],
+                                                 u[0]["seq_chunk_offset"], kept_cap=host["kept_cap"])
+        return lists, None, rc, cnt
     nm = host["nmi"]
     lists, logits, _, rc, cnt = oracle.nmi_select(nm["q"], nm["w"], nm["khat"], nm["seq_chunk_offset"],
                                                   kept_cap=host["kept_cap"])

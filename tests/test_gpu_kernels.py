@@ -111,6 +111,59 @@ def test_nmi_select_capacity_overflow_truncates_and_flags(L):
     np.testing.assert_array_equal(kept[0], nm["planted"][0][:10])
 
 
+@pytest.mark.parametrize("name", ["decode_128k_b8_mla", "decode_512k_b1_mla_cold", "decode_ragged_b32_mla"])
+def test_nmi_select_union_of_three_indexers_exact(L, name):
+    """OR mode of three independent indexers (structural plants with different seeds): the
+    kept list is the oracle's union, which is the union of the three plants."""
+    wl = W.workload(name)
+    sets = [W.nmi_inputs(wl, seed_offset=101 * i) for i in range(3)]
+    cap = max(wl.n_ch)
+    d = dev()
+    status = torch.zeros(1, dtype=torch.int32, device=d)
+    off = torch.from_numpy(sets[0]["seq_chunk_offset"]).to(d)
+    logits = torch.empty(3, sets[0]["khat"].shape[0], dtype=torch.float32, device=d)
+    kept, cnt = L.nmi_select_union([bf16(n["q"], d) for n in sets], [bf16(n["w"], d) for n in sets],
+                                   [bf16(n["khat"], d) for n in sets], off, cap, cap, logits=logits, status=status)
+    kept, cnt = kept.cpu().numpy(), cnt.cpu().numpy()
+    ref, rc, rcnt = oracle.nmi_select_union([n["q"] for n in sets], [n["w"] for n in sets],
+                                            [n["khat"] for n in sets], sets[0]["seq_chunk_offset"], cap)
+    assert status.item() == 0 and rc == 0
+    for b in range(wl.B):
+        np.testing.assert_array_equal(kept[b, :cnt[b]], ref[b])
+        planted = np.union1d(np.union1d(sets[0]["planted"][b], sets[1]["planted"][b]), sets[2]["planted"][b])
+        np.testing.assert_array_equal(ref[b], planted)
+        assert np.all(kept[b, cnt[b]:] == -1)
+    for i in range(3):   # each indexer's logits are those of the single gate
+        _, ref_logits, _, _, _ = oracle.nmi_select(sets[i]["q"], sets[i]["w"], sets[i]["khat"],
+                                                   sets[i]["seq_chunk_offset"], cap)
+        np.testing.assert_allclose(logits[i].cpu().numpy(), ref_logits, rtol=1e-4, atol=1e-3)
+
+
+def test_nmi_select_union_random_inputs_and_single_indexer(L):
+    """Independent random indexers with margin-repaired keys, ragged batch; and n_idx = 1
+    gives exactly lsa_nmi_select."""
+    n_ch = (300, 1, 64, 129)
+    wl = W.workload("decode_128k_b8_mla", B=len(n_ch), ctx=tuple(c * CH for c in n_ch), pass_rate=(0.5,) * 4)
+    sets = []
+    for i in range(3):
+        nm = W.nmi_inputs(wl, structural=False, seed_offset=7 * i + 1)
+        H.repair_nmi_margin(dict(nmi=nm, kept_cap=max(n_ch)), seed=50 + i)
+        sets.append(nm)
+    d = dev()
+    off = torch.from_numpy(sets[0]["seq_chunk_offset"]).to(d)
+    kept, cnt = L.nmi_select_union([bf16(n["q"], d) for n in sets], [bf16(n["w"], d) for n in sets],
+                                   [bf16(n["khat"], d) for n in sets], off, max(n_ch), max(n_ch))
+    ref, _, _ = oracle.nmi_select_union([n["q"] for n in sets], [n["w"] for n in sets], [n["khat"] for n in sets],
+                                        sets[0]["seq_chunk_offset"], max(n_ch))
+    kept, cnt = kept.cpu().numpy(), cnt.cpu().numpy()
+    for b in range(wl.B):
+        np.testing.assert_array_equal(kept[b, :cnt[b]], ref[b])
+    one, one_cnt = L.nmi_select_union([bf16(sets[1]["q"], d)], [bf16(sets[1]["w"], d)], [bf16(sets[1]["khat"], d)],
+                                      off, max(n_ch), max(n_ch))
+    single, single_cnt, _, _ = _nmi_gpu(L, sets[1], max(n_ch), max(n_ch))
+    assert np.array_equal(one.cpu().numpy(), single) and np.array_equal(one_cnt.cpu().numpy(), single_cnt)
+
+
 # -------------------------------------------------------------- a2 + a3 ---
 
 def _small_mla(**kw):

@@ -119,6 +119,30 @@ def test_window_512k_cold_pool():
     _check_window(host, win, pairs)
 
 
+def test_window_128k_b8_union_of_three_indexers():
+    """The pages' deployed gate: three independent indexers in OR mode select the chunks once,
+    then 64 steps of append, top-k and attention run over the larger kept set."""
+    wl = W.workload("decode_128k_b8_mla")
+    host = host_build(wl, n_indexers=3)
+    kept, _, _, _ = H.kept_lists(host)
+    assert min(k.size for k in kept) > 0.3 * wl.n_ch[0]          # union of three 13.5 % plants
+    pairs = [(1, 0), (6, 40), (4, 63)]
+    H.open_topk_gap(host, kept, pairs)
+    win = _window(host)
+    _check_window(host, win, pairs)
+
+
+def test_window_512k_cold_pool_union_of_three_indexers():
+    wl = W.workload("decode_512k_b1_mla_cold")
+    host = host_build(wl, n_indexers=3, fetch_fraction=0.4)
+    kept, _, _, _ = H.kept_lists(host)
+    pairs = [(0, 0), (0, 37)]
+    H.open_topk_gap(host, kept, pairs)
+    win = _window(host)
+    assert win.n_fetched == sum(1 for c in kept[0] if c < host["first_window_chunk"])
+    _check_window(host, win, pairs)
+
+
 def test_window_context_is_window_plus_one_chunk():
     wl = W.workload("decode_128k_b8_mla", B=2, ctx=(8064, 8128), pass_rate=(1.0, 0.5), steps=4)
     host = host_build(wl)

@@ -13,6 +13,7 @@ import pytest
 import oracle
 from oracle import build as obuild
 from tests import test_oracle_attention as TA
+from tests import test_oracle_baselines as TB
 from tests import test_oracle_label_vote as TL
 from tests import test_oracle_select as TS
 
@@ -34,6 +35,10 @@ MUTANTS = {
     "union becomes intersection": ("                if (prob >= 0.5)\n                    fetched = 1;",
                                    "                if (prob < 0.5)\n                    fetched = -1;\n"
                                    "                else if (fetched == 0)\n                    fetched = 1;"),
+    "random keeps the largest draws": ("neg[c] = -(double)u;", "neg[c] = (double)u;"),
+    "random count rounds down": ("((int64_t)n_old * keep_num + keep_den / 2) / keep_den",
+                                 "((int64_t)n_old * keep_num) / keep_den"),
+    "random draws ignore the sequence": ("((uint64_t)b << 32) + (uint64_t)c", "(uint64_t)c"),
     "vote threshold strict": ("labels[c] = (uint8_t)(best >= min_layers);", "labels[c] = (uint8_t)(best > min_layers);"),
     "vote counts any step": ("if (count[(size_t)t * n_chunks + c] > best) best = count[(size_t)t * n_chunks + c];",
                              "best += count[(size_t)t * n_chunks + c];"),
@@ -47,6 +52,10 @@ PINS = [
     lambda o: TS.test_nmi_sequences_use_their_own_queries(o),
     lambda o: TS.test_nmi_union_keeps_exactly_the_union_of_the_plants(o),
     lambda o: TS.test_nmi_union_each_indexer_alone_keeps_a_different_chunk(o),
+    lambda o: TB.test_recency_only_keeps_no_older_chunk(o),
+    lambda o: TB.test_random_selection_is_the_smallest_sequential_splitmix_draws(o),
+    lambda o: TB.test_random_count_rounds_half_up_and_respects_the_fraction(o),
+    lambda o: TB.test_random_sequences_draw_from_their_own_counters(o),
     lambda o: TS.test_li_score_odd_part_is_linear(o),
     lambda o: TS.test_li_score_special_cases(o),
     lambda o: TS.test_topk_equals_full_library_sort_with_ties(o, 200, 64),
@@ -79,7 +88,7 @@ def test_pins_catch_planted_mistake(tmp_path, name):
     libpath = _compile_mutant(tmp_path, name, old, new)
     real = oracle._load()
     mutant = ctypes.CDLL(libpath)
-    for fn in ("lsao_nmi_select", "lsao_nmi_select_union", "lsao_li_scores", "lsao_topk_select", "lsao_topk_select_f32",
+    for fn in ("lsao_nmi_select", "lsao_nmi_select_union", "lsao_select_baseline", "lsao_li_scores", "lsao_topk_select", "lsao_topk_select_f32",
                "lsao_attention_dense", "lsao_decode_step", "lsao_nucleus", "lsao_label_vote"):
         getattr(mutant, fn).argtypes = getattr(real, fn).argtypes
         getattr(mutant, fn).restype = ctypes.c_int
