@@ -127,6 +127,36 @@ int lsa_nmi_select_union(int n_idx, const lsa_bf16 *const *q, const lsa_bf16 *co
 size_t lsa_nmi_select_union_workspace_size(int n_idx, int B, int max_chunks_per_seq);
 
 /*
+ * Baseline selectors: the two schemes the pages compare LSA with, producing a
+ * kept list in the same form as lsa_nmi_select so that the same top-k,
+ * attention and fetch calls run after them.
+ * Passage: cjcn.com.cn article section 5 (a pure sliding window keeping the
+ * recent 8K tokens, and random retention of 10 % of the history chunks; every
+ * scheme keeps the recent window); gist.science explainer section 4 ("Recency
+ * Only" and "Random 10%").
+ *
+ * n_old = window_start[b] / 64 chunks lie before sequence b's window.
+ *   LSA_SELECT_RECENT: no older chunk is kept (kept_count 0, kept_idx all -1);
+ *     window_start may be NULL.
+ *   LSA_SELECT_RANDOM: m = floor((n_old * keep_num + keep_den / 2) / keep_den)
+ *     older chunks are kept, uniformly at random: chunk s draws
+ *     u = (output number b * 2^32 + s of a SplitMix64 stream started at seed) >> 40
+ *     and the m chunks with the smallest u are kept, ties to the lower index.
+ *     (SplitMix64: Steele, Lea and Flood, OOPSLA 2014; output c is
+ *     mix(seed + (c + 1) * 0x9E3779B97F4A7C15).)
+ *   window_start [B] int32 (device); max_old_chunks: host bound of n_old (larger
+ *     n_old is cut to it and sets LSA_DEV_INDEX)
+ *   kept_idx [B, kept_cap], kept_count [B] int32 (device, out): ascending, -1 after
+ * Returns LSA_ERR_CAPACITY if round(max_old_chunks * keep_num / keep_den) > kept_cap.
+ */
+#define LSA_SELECT_RECENT 0
+#define LSA_SELECT_RANDOM 1
+int lsa_select_baseline(int mode, const int32_t *window_start, int B, int max_old_chunks, uint64_t seed,
+                        int keep_num, int keep_den, int32_t *kept_idx, int32_t *kept_count, int kept_cap,
+                        int32_t *dev_status, void *ws, size_t ws_bytes, lsa_stream_t stream);
+size_t lsa_select_baseline_workspace_size(int B, int max_old_chunks);
+
+/*
  * a2 + a3 -- Lightning-Indexer scoring and fine top-k inside the kept chunks.
  * Passage: gist.science explainer 2.1 ("Gestufte Selektion"); cjcn.com.cn
  * article section 2 (the native indexer takes a top-k inside the reduced set).

@@ -216,6 +216,63 @@ __global__ void __launch_bounds__(kTopkThreads) topk_scores_kernel(const float *
     topk_cluster(scores + a, n, k, CandIdentity{}, topk_idx + (size_t)b * k, topk_count + b, stage_cap);
 }
 
+// ------------------------------------------------------- baseline selectors --
+// The pages compare LSA with a recency-only window and with random retention of
+// a fraction of the older chunks (cjcn.com.cn article section 5, gist.science
+// explainer section 4).  The random selector keeps, of the n_old chunks before
+// the window, the m with the smallest SplitMix64 draws; as scores for the
+// cluster top-k above they are 2^24 - 1 - draw, exact in fp32, so the m largest
+// scores are the m smallest draws and ties go to the lower chunk index.
+
+// Output number c of a SplitMix64 stream started at `seed` (Steele, Lea and
+// Flood, OOPSLA 2014): state = seed + (c + 1) * golden-ratio increment, mixed.
+__device__ __forceinline__ uint64_t splitmix64_output(uint64_t seed, uint64_t c) {
+    uint64_t z = seed + (c + 1) * 0x9E3779B97F4A7C15ull;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+
+__device__ __forceinline__ int older_chunks(const int32_t *window_start, int b, int max_old, int32_t *status) {
+    const int n = max(window_start[b], 0) / LSA_CHUNK;
+    if (n > max_old) {
+        if (status && threadIdx.x == 0 && blockIdx.x == 0) flag(status, LSA_DEV_INDEX);
+        return max_old;
+    }
+    return n;
+}
+
+// grid (ceil(max_old / 256), B): scores[b, s] for the older chunks s of sequence b.
+__global__ void __launch_bounds__(256) random_score_kernel(const int32_t *__restrict__ window_start, int max_old,
+                                                           uint64_t seed, float *__restrict__ scores) {
+    const int b = blockIdx.y, s = blockIdx.x * 256 + threadIdx.x;
+    const int n_old = min(max(window_start[b], 0) / LSA_CHUNK, max_old);
+    if (s >= n_old) return;
+    const uint32_t draw = (uint32_t)(splitmix64_output(seed, ((uint64_t)b << 32) + (uint64_t)s) >> 40);
+    scores[(size_t)b * max_old + s] = (float)(0xFFFFFFu - draw);
+}
+
+// One cluster per sequence: the m = round(n_old * num / den) chunks with the largest
+// scores, ascending, then -1 up to kept_cap.
+__global__ void __launch_bounds__(kTopkThreads) random_select_kernel(const float *__restrict__ scores,
+                                                                     const int32_t *__restrict__ window_start,
+                                                                     int max_old, int num, int den,
+                                                                     int32_t *__restrict__ kept_idx,
+                                                                     int32_t *__restrict__ kept_count, int kept_cap,
+                                                                     int32_t *status, int stage_cap) {
+    const int b = blockIdx.y;
+    const int n_old = older_chunks(window_start, b, max_old, status);
+    const int m = (int)min(((int64_t)n_old * num + den / 2) / den, (int64_t)n_old);   // <= kept_cap (host check)
+    int32_t *out = kept_idx + (size_t)b * kept_cap;
+    const int c = (int)sm100::cluster_rank();
+    for (int j = m + c * kTopkThreads + (int)threadIdx.x; j < kept_cap; j += kTopkCtas * kTopkThreads) out[j] = -1;
+    if (m == 0) {
+        if (c == 0 && threadIdx.x == 0) kept_count[b] = 0;
+        return;
+    }
+    topk_cluster(scores + (size_t)b * max_old, n_old, m, CandIdentity{}, out, kept_count + b, stage_cap);
+}
+
 // Keys staged per CTA: a slice of at most ceil(max_n / 8), never more than 24,576 (96 KB).
 static int stage_capacity(int max_n) { return max(0, min((max_n + kTopkCtas - 1) / kTopkCtas, 24576)); }
 
@@ -305,4 +362,47 @@ extern "C" int lsa_topk_from_scores(const float *scores, const int64_t *cand_off
     const int cap = stage_capacity(max_cand);
     return launch_topk(topk_scores_kernel, B, cap, stream, "topk_scores_kernel", scores, cand_offset, max_cand, k,
                        topk_idx, topk_count, cap);
+}
+
+extern "C" size_t lsa_select_baseline_workspace_size(int B, int max_old_chunks) {
+    if (B <= 0 || max_old_chunks < 0) return 0;
+    Carver c(nullptr);
+    c.take<float>((size_t)B * (max_old_chunks > 0 ? max_old_chunks : 1));   // draws as top-k scores
+    return align_up(c.used, 256);
+}
+
+extern "C" int lsa_select_baseline(int mode, const int32_t *window_start, int B, int max_old_chunks, uint64_t seed,
+                                   int keep_num, int keep_den, int32_t *kept_idx, int32_t *kept_count, int kept_cap,
+                                   int32_t *dev_status, void *ws, size_t ws_bytes, lsa_stream_t stream) {
+    LSA_REQUIRE(mode == LSA_SELECT_RECENT || mode == LSA_SELECT_RANDOM, LSA_ERR_INVALID_ARG,
+                "lsa_select_baseline: mode must be LSA_SELECT_RECENT or LSA_SELECT_RANDOM (got %d)", mode);
+    LSA_REQUIRE(B > 0 && kept_cap >= 1 && max_old_chunks >= 0, LSA_ERR_INVALID_ARG,
+                "lsa_select_baseline: bad sizes (B=%d kept_cap=%d max_old_chunks=%d)", B, kept_cap, max_old_chunks);
+    LSA_REQUIRE(kept_idx && kept_count, LSA_ERR_INVALID_ARG, "lsa_select_baseline: null output pointer");
+    if (mode == LSA_SELECT_RECENT) {
+        LSA_CUDA(cudaMemsetAsync(kept_idx, 0xFF, sizeof(int32_t) * (size_t)B * kept_cap, stream));   // -1
+        LSA_CUDA(cudaMemsetAsync(kept_count, 0, sizeof(int32_t) * (size_t)B, stream));
+        return LSA_OK;
+    }
+    LSA_REQUIRE(window_start, LSA_ERR_INVALID_ARG, "lsa_select_baseline: null window_start");
+    LSA_REQUIRE(keep_num >= 0 && keep_den >= 1 && keep_num <= keep_den, LSA_ERR_INVALID_ARG,
+                "lsa_select_baseline: keep fraction %d/%d outside [0, 1]", keep_num, keep_den);
+    const int64_t m_max = ((int64_t)max_old_chunks * keep_num + keep_den / 2) / keep_den;
+    LSA_REQUIRE(m_max <= kept_cap, LSA_ERR_CAPACITY,
+                "lsa_select_baseline: up to %lld chunks are kept, kept_cap is %d", (long long)m_max, kept_cap);
+    const size_t need = lsa_select_baseline_workspace_size(B, max_old_chunks);
+    LSA_REQUIRE(ws && ws_bytes >= need, LSA_ERR_WORKSPACE, "lsa_select_baseline: workspace of %zu bytes, %zu needed",
+                ws_bytes, need);
+    Carver c(ws);
+    float *scores = c.take<float>((size_t)B * (max_old_chunks > 0 ? max_old_chunks : 1));
+    if (max_old_chunks > 0) {
+        random_score_kernel<<<dim3((max_old_chunks + 255) / 256, B), 256, 0, stream>>>(window_start, max_old_chunks,
+                                                                                      seed, scores);
+        int rc = check_launch("random_score_kernel");
+        if (rc) return rc;
+    }
+    const int cap = stage_capacity(max_old_chunks);
+    return launch_topk(random_select_kernel, B, cap, stream, "random_select_kernel", (const float *)scores,
+                       window_start, max_old_chunks, keep_num, keep_den, kept_idx, kept_count, kept_cap, dev_status,
+                       cap);
 }

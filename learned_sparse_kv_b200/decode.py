@@ -55,8 +55,12 @@ class Window:
     """
 
     def __init__(self, shapes: Shapes, t: Dict[str, torch.Tensor], max_chunks_per_seq: int, kept_cap: int,
-                 cold: Optional[dict] = None):
+                 cold: Optional[dict] = None, selector: Optional[dict] = None):
+        """selector: None for the memory-indexer gate (OR mode when t has "nmi_union"), or a
+        baseline: dict(mode=lsa.SELECT_RECENT) or dict(mode=lsa.SELECT_RANDOM, seed=.., keep_num=1,
+        keep_den=10)."""
         self.s = shapes
+        self.selector = selector
         self.t = t
         self.dev = t["q"].device
         self.max_chunks = max_chunks_per_seq
@@ -75,7 +79,8 @@ class Window:
         self.status = torch.zeros(1, dtype=torch.int32, device=d)
         self.max_window_len = shapes.window + S
         n_idx = len(t["nmi_union"]) if "nmi_union" in t else 1
-        self.ws_select = torch.empty(max(lsa.nmi_select_union_workspace_size(n_idx, B, max_chunks_per_seq), 256),
+        self.ws_select = torch.empty(max(lsa.nmi_select_union_workspace_size(n_idx, B, max_chunks_per_seq),
+                                         lsa.select_baseline_workspace_size(B, max_chunks_per_seq), 256),
                                      dtype=torch.uint8, device=d)
         self.scores = torch.empty(B, kept_cap * CHUNK, dtype=torch.float32, device=d)
         self.ws_topk = torch.empty(max(lsa.topk_workspace_size(B, kept_cap), 256), dtype=torch.uint8, device=d)
@@ -97,6 +102,13 @@ class Window:
 
     def select(self):
         t = self.t
+        if self.selector is not None:
+            sel = self.selector
+            lsa.select_baseline(sel["mode"], t["window_start"], self.max_chunks, self.kept_cap,
+                                seed=sel.get("seed", 0), keep_num=sel.get("keep_num", 1),
+                                keep_den=sel.get("keep_den", 10), status=self.status, kept_idx=self.kept_idx,
+                                kept_count=self.kept_count, ws=self.ws_select)
+            return
         if "nmi_union" in t:
             u = t["nmi_union"]
             lsa.nmi_select_union([x[0] for x in u], [x[1] for x in u], [x[2] for x in u], t["seq_chunk_offset"],
@@ -168,11 +180,13 @@ class Window:
             self.steps()
 
     def launches_per_window(self) -> int:
-        """Kernels this library launches per window (select: 2; per step: append 1, top-k 2 or 3, decode 2).
+        """Kernels this library launches per window (select: 2, or 0 for the recency baseline, which
+        only fills memory; per step: append 1, top-k 2 or 3, decode 2).
 
         The top-k call counts the kept cold chunks inside the tcgen05 indexer kernel when
         that kernel serves the indexer shape, else in a kernel of its own."""
-        return 2 + self.s.steps * (1 + lsa.topk_kernel_count(self.s.B, self.s.Hl, self.s.dl) + 2)
+        sel = 0 if (self.selector is not None and self.selector["mode"] == lsa.SELECT_RECENT) else 2
+        return sel + self.s.steps * (1 + lsa.topk_kernel_count(self.s.B, self.s.Hl, self.s.dl) + 2)
 
     def device_status(self) -> int:
         return int(self.status.item())

@@ -36,6 +36,8 @@ def _load():
         "lsa_nmi_select_workspace_size": ([I, I], SZ),
         "lsa_nmi_select_union": ([I, P, P, P, P, I, I, I, I64, I, P, P, I, P, P, P, SZ, P], I),
         "lsa_nmi_select_union_workspace_size": ([I, I, I], SZ),
+        "lsa_select_baseline": ([I, P, I, I, ctypes.c_uint64, I, I, P, P, I, P, P, SZ, P], I),
+        "lsa_select_baseline_workspace_size": ([I, I], SZ),
         "lsa_topk": ([P, P, P, I64, P, I, P, P, I, P, I, I, I, I, P, P, P, P, P, SZ, P], I),
         "lsa_topk_workspace_size": ([I, I], SZ),
         "lsa_topk_kernel_count": ([I, I, I], I),
@@ -146,6 +148,32 @@ def nmi_select_union(qs, ws_, khats, seq_chunk_offset, max_chunks_per_seq, kept_
     _check(_lib.lsa_nmi_select_union(n, arr(qs), arr(ws_), arr(khats), _ptr(seq_chunk_offset), B, Hn, dn,
                                      khats[0].shape[0], max_chunks_per_seq, _ptr(kept_idx), _ptr(kept_count),
                                      kept_cap, _ptr(logits), _ptr(status), _ptr(ws), ws.numel(), _stream(stream)))
+    return kept_idx, kept_count
+
+
+SELECT_RECENT, SELECT_RANDOM = 0, 1
+
+
+def select_baseline_workspace_size(B, max_old_chunks):
+    return _lib.lsa_select_baseline_workspace_size(B, max_old_chunks)
+
+
+def select_baseline(mode, window_start, max_old_chunks, kept_cap, *, seed=0, keep_num=1, keep_den=10, status=None,
+                    kept_idx=None, kept_count=None, ws=None, stream=None):
+    """Recency-only (SELECT_RECENT) or random-fraction (SELECT_RANDOM) kept list in the gate's format.
+
+    Returns (kept_idx [B, kept_cap] int32, kept_count [B] int32)."""
+    _dev(window_start, torch.int32, "window_start")
+    B = window_start.shape[0]
+    dev = window_start.device
+    if kept_idx is None:
+        kept_idx = torch.empty(B, kept_cap, dtype=torch.int32, device=dev)
+    if kept_count is None:
+        kept_count = torch.empty(B, dtype=torch.int32, device=dev)
+    ws = _ws(select_baseline_workspace_size(B, max_old_chunks), dev, ws)
+    _check(_lib.lsa_select_baseline(int(mode), _ptr(window_start), B, max_old_chunks, ctypes.c_uint64(seed),
+                                    int(keep_num), int(keep_den), _ptr(kept_idx), _ptr(kept_count), kept_cap,
+                                    _ptr(status), _ptr(ws), ws.numel(), _stream(stream)))
     return kept_idx, kept_count
 
 

@@ -15,6 +15,12 @@ CH = W.CHUNK
 
 
 def kept_lists(host):
+    if "selector" in host:
+        sel = host["selector"]
+        lists, rc, cnt = oracle.select_baseline(sel["mode"], host["window_start"], seed=sel.get("seed", 0),
+                                                keep_num=sel.get("keep_num", 1), keep_den=sel.get("keep_den", 10),
+                                                kept_cap=host["kept_cap"])
+        return lists, None, rc, cnt
     if "nmi_union" in host:
         u = host["nmi_union"]
         lists, rc, cnt = oracle.nmi_select_union([n["q"] for n in u], [n["w"] for n in u], [n["khat"] for n in u],

@@ -164,6 +164,41 @@ def test_nmi_select_union_random_inputs_and_single_indexer(L):
     assert np.array_equal(one.cpu().numpy(), single) and np.array_equal(one_cnt.cpu().numpy(), single_cnt)
 
 
+@pytest.mark.parametrize("seed", [0, 77, 2 ** 63 + 5])
+def test_select_baseline_random_and_recent_exact(L, seed):
+    """Random 10 % of the older chunks (and 3/8, and all) against the oracle, bit for bit, on
+    the window starts of the 128K, 512K and ragged workloads plus edge cases; recency-only
+    gives empty lists."""
+    d = dev()
+    starts = [131072 - 8000 + 8, 524288 - 8000 + 8, 0, 64, 640] + [L_ - 8000 + 8 for L_ in
+                                                                     W.workload("decode_ragged_b32_mla").ctx[:9]]
+    starts = np.array([x - x % 64 for x in starts], np.int32)
+    max_old = int(starts.max()) // CH
+    ws = i32(starts, d)
+    for num, den in ((1, 10), (3, 8), (1, 1)):
+        cap = (max_old * num + den // 2) // den
+        status = torch.zeros(1, dtype=torch.int32, device=d)
+        kept, cnt = L.select_baseline(L.SELECT_RANDOM, ws, max_old, max(cap, 1), seed=seed, keep_num=num,
+                                      keep_den=den, status=status)
+        ref, rc, rcnt = oracle.select_baseline(oracle.RANDOM, starts, seed=seed, keep_num=num, keep_den=den,
+                                               kept_cap=max(cap, 1))
+        kept, cnt = kept.cpu().numpy(), cnt.cpu().numpy()
+        assert status.item() == 0 and rc == 0
+        for b in range(starts.size):
+            assert cnt[b] == rcnt[b]
+            np.testing.assert_array_equal(kept[b, :cnt[b]], ref[b])
+            assert np.all(kept[b, cnt[b]:] == -1)
+    kept, cnt = L.select_baseline(L.SELECT_RECENT, ws, max_old, 16)
+    assert int(cnt.abs().sum()) == 0 and bool((kept == -1).all())
+
+
+def test_select_baseline_rejects_a_too_small_capacity(L):
+    ws = torch.tensor([64 * 1000], dtype=torch.int32, device=dev())
+    with pytest.raises(L.LSAError) as e:
+        L.select_baseline(L.SELECT_RANDOM, ws, 1000, 99)         # 100 chunks are kept
+    assert e.value.code == 4
+
+
 # -------------------------------------------------------------- a2 + a3 ---
 
 def _small_mla(**kw):

@@ -21,7 +21,7 @@ CH = W.CHUNK
 def _window(host, graph=True):
     from learned_sparse_kv_b200.decode import Shapes, Window
     shapes, t, max_ch, kept_cap, cold = upload(host, torch.device("cuda:0"))
-    win = Window(Shapes(**shapes), t, max_ch, kept_cap, cold)
+    win = Window(Shapes(**shapes), t, max_ch, kept_cap, cold, selector=host.get("selector"))
     if graph:
         win.capture()
     win.run(use_graph=graph)
@@ -140,6 +140,33 @@ def test_window_512k_cold_pool_union_of_three_indexers():
     H.open_topk_gap(host, kept, pairs)
     win = _window(host)
     assert win.n_fetched == sum(1 for c in kept[0] if c < host["first_window_chunk"])
+    _check_window(host, win, pairs)
+
+
+def test_window_128k_b8_random_10_percent_baseline():
+    """The random-10 % baseline through the same top-k and attention: 10 % of the older chunks
+    of each sequence, drawn by the counter-based generator, then 64 decode steps."""
+    wl = W.workload("decode_128k_b8_mla")
+    host = host_build(wl)
+    host["selector"] = dict(mode=1, seed=4242, keep_num=1, keep_den=10)      # random
+    kept, _, _, _ = H.kept_lists(host)
+    assert all(k.size == (host["window_start"][b] // CH + 5) // 10 for b, k in enumerate(kept))
+    pairs = [(0, 0), (5, 33), (7, 63)]
+    H.open_topk_gap(host, kept, pairs)
+    win = _window(host)
+    _check_window(host, win, pairs)
+
+
+def test_window_512k_cold_recency_only_baseline():
+    """Recency only on the cold 512K workload: nothing is fetched and every step attends the
+    window alone."""
+    wl = W.workload("decode_512k_b1_mla_cold", steps=8)
+    host = host_build(wl)
+    host["selector"] = dict(mode=0)                                          # recency only
+    kept, _, _, _ = H.kept_lists(host)
+    pairs = [(0, s) for s in range(8)]
+    win = _window(host)
+    assert win.n_fetched == 0 and int(win.kept_count.sum()) == 0
     _check_window(host, win, pairs)
 
 
