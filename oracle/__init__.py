@@ -38,6 +38,8 @@ def _load():
                                               ctypes.POINTER(_u16p), _i64p, c_int, c_int, c_int, _i32p, _i32p, c_int]
         lib.lsao_select_baseline.argtypes = [c_int, _i32p, c_int, ctypes.c_uint64, c_int, c_int, _i32p, _i32p,
                                              c_int]
+        lib.lsao_query_encoder.argtypes = [_u16p, c_int, c_int, _u16p, c_int, _u16p, _u16p, c_int, c_int,
+                                           _f64p, _f64p]
         lib.lsao_li_scores.argtypes = [_u16p, _u16p, _u16p, c_int, c_int, c_int, _f64p]
         lib.lsao_topk_select.argtypes = [_f64p, c_int, c_int, _i32p, _i32p]
         lib.lsao_topk_select_f32.argtypes = [_f32p, c_int, c_int, _i32p, _i32p]
@@ -50,7 +52,8 @@ def _load():
                                          _i32p, _i32p, _f64p, _i32p, _f64p, _f64p]
         lib.lsao_nucleus.argtypes = [_f32p, c_int, c_double, _u8p]
         lib.lsao_label_vote.argtypes = [_f32p, c_int, c_int, c_int, c_double, c_int, c_int, _u8p, _i32p]
-        for name in ("lsao_nmi_select", "lsao_nmi_select_union", "lsao_select_baseline", "lsao_li_scores", "lsao_topk_select", "lsao_topk_select_f32",
+        for name in ("lsao_nmi_select", "lsao_nmi_select_union", "lsao_select_baseline", "lsao_query_encoder",
+                     "lsao_li_scores", "lsao_topk_select", "lsao_topk_select_f32",
                      "lsao_attention_dense", "lsao_decode_step", "lsao_nucleus", "lsao_label_vote"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
@@ -109,6 +112,21 @@ def nmi_select_union(qs, ws, khats, seq_chunk_offset, kept_cap=None):
                                        _p(kept, _i32p), _p(cnt, _i32p), kept_cap)
     lists = [kept[b, :min(int(cnt[b]), kept_cap)].copy() for b in range(B)]
     return lists, rc, cnt
+
+
+def query_encoder(h, w_down, w_up, w_head, Hn, dn):
+    """Indexer query encoder.  h [B, d_model], w_down [rank, d_model], w_up [Hn*dn, rank],
+    w_head [Hn, d_model] (bf16 bits).  Returns (q [B, Hn, dn] fp64, w [B, Hn] fp64)."""
+    h, w_down, w_up, w_head = _u16(h), _u16(w_down), _u16(w_up), _u16(w_head)
+    B, d_model = h.shape
+    rank = w_down.shape[0]
+    assert w_down.shape == (rank, d_model) and w_up.shape == (Hn * dn, rank) and w_head.shape == (Hn, d_model)
+    q = np.zeros((max(B, 1), Hn, dn), np.float64)
+    w = np.zeros((max(B, 1), Hn), np.float64)
+    rc = _load().lsao_query_encoder(_p(h, _u16p), B, d_model, _p(w_down, _u16p), rank, _p(w_up, _u16p),
+                                    _p(w_head, _u16p), Hn, dn, _p(q, _f64p), _p(w, _f64p))
+    assert rc == 0
+    return q[:B], w[:B]
 
 
 RECENT, RANDOM = 0, 1

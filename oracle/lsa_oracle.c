@@ -27,6 +27,8 @@
  *   [cjcn 4]    same article, section 4 (one independent memory indexer at
  *               each of layers 10, 12 and 20; a chunk is recalled when any of
  *               the three scores it at 0.5 or more: "OR-mode routing")
+ *   [gist 2.3]  same page, section 2.3 (frozen compressed keys; only the
+ *               low-rank projection matrices of the query encoder are trained)
  *   [cjcn 5]    same article, section 5 (results: the baselines are a pure
  *               sliding window keeping the recent 8K, and random retention of
  *               10 % of the history chunks; all schemes keep the recent window)
@@ -247,6 +249,55 @@ int lsao_topk_select_f32(const float *scores, int n, int k, int32_t *out, int32_
     int rc = lsao_topk_select(wide, n, k, out, out_count);
     free(wide);
     return rc;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Memory-indexer query encoder  [gist 2.1, 2.3] [cjcn 4]                     */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * The indexer maps the hidden state h_t of the current token to low-rank
+ * indexer queries; only these low-rank projections are trained, and their rank
+ * is 2048 in the pages' configuration.  Reading taken (the pages give no
+ * formula): a down-projection to the rank, then an up-projection to the heads,
+ * and the per-head weights projected from h_t directly, with no normalisation
+ * or nonlinearity in between:
+ *   c = W_down h           (rank entries)
+ *   q = W_up c             (Hn * dn entries, head-major: q[h][d] = entry h * dn + d)
+ *   w = W_head h           (Hn entries)
+ * for each of the B tokens.  Weights are [out, in] row-major, inputs bf16.
+ */
+int lsao_query_encoder(const uint16_t *h, int B, int d_model, const uint16_t *w_down, int rank,
+                       const uint16_t *w_up, const uint16_t *w_head, int Hn, int dn,
+                       double *q_out, double *w_out)
+{
+    if (B < 0 || d_model <= 0 || rank <= 0 || Hn <= 0 || dn <= 0)
+        return LSAO_ERR_ARG;
+    double *c = (double *)malloc(sizeof(double) * (size_t)rank);
+    if (!c) return LSAO_ERR_ARG;
+    for (int b = 0; b < B; ++b) {
+        const uint16_t *hb = h + (size_t)b * d_model;
+        for (int i = 0; i < rank; ++i) {
+            double acc = 0.0;
+            for (int k = 0; k < d_model; ++k)
+                acc += bf16_value(w_down[(size_t)i * d_model + k]) * bf16_value(hb[k]);
+            c[i] = acc;
+        }
+        for (int o = 0; o < Hn * dn; ++o) {
+            double acc = 0.0;
+            for (int i = 0; i < rank; ++i)
+                acc += bf16_value(w_up[(size_t)o * rank + i]) * c[i];
+            q_out[(size_t)b * Hn * dn + o] = acc;
+        }
+        for (int o = 0; o < Hn; ++o) {
+            double acc = 0.0;
+            for (int k = 0; k < d_model; ++k)
+                acc += bf16_value(w_head[(size_t)o * d_model + k]) * bf16_value(hb[k]);
+            w_out[(size_t)b * Hn + o] = acc;
+        }
+    }
+    free(c);
+    return LSAO_OK;
 }
 
 /* ------------------------------------------------------------------------- */

@@ -14,6 +14,7 @@ import oracle
 from oracle import build as obuild
 from tests import test_oracle_attention as TA
 from tests import test_oracle_baselines as TB
+from tests import test_oracle_encoder as TE
 from tests import test_oracle_label_vote as TL
 from tests import test_oracle_select as TS
 
@@ -39,6 +40,9 @@ MUTANTS = {
     "random count rounds down": ("((int64_t)n_old * keep_num + keep_den / 2) / keep_den",
                                  "((int64_t)n_old * keep_num) / keep_den"),
     "random draws ignore the sequence": ("((uint64_t)b << 32) + (uint64_t)c", "(uint64_t)c"),
+    "encoder W_up transposed": ("w_up[(size_t)o * rank + i]", "w_up[(size_t)i * (Hn * dn) + o]"),
+    "encoder head weights from W_down": ("bf16_value(w_head[(size_t)o * d_model + k])",
+                                         "bf16_value(w_down[(size_t)o * d_model + k])"),
     "vote threshold strict": ("labels[c] = (uint8_t)(best >= min_layers);", "labels[c] = (uint8_t)(best > min_layers);"),
     "vote counts any step": ("if (count[(size_t)t * n_chunks + c] > best) best = count[(size_t)t * n_chunks + c];",
                              "best += count[(size_t)t * n_chunks + c];"),
@@ -52,6 +56,8 @@ PINS = [
     lambda o: TS.test_nmi_sequences_use_their_own_queries(o),
     lambda o: TS.test_nmi_union_keeps_exactly_the_union_of_the_plants(o),
     lambda o: TS.test_nmi_union_each_indexer_alone_keeps_a_different_chunk(o),
+    lambda o: TE.test_encoder_equals_library_matrix_products(o),
+    lambda o: TE.test_encoder_queries_span_at_most_rank_dimensions(o),
     lambda o: TB.test_recency_only_keeps_no_older_chunk(o),
     lambda o: TB.test_random_selection_is_the_smallest_sequential_splitmix_draws(o),
     lambda o: TB.test_random_count_rounds_half_up_and_respects_the_fraction(o),
@@ -88,7 +94,8 @@ def test_pins_catch_planted_mistake(tmp_path, name):
     libpath = _compile_mutant(tmp_path, name, old, new)
     real = oracle._load()
     mutant = ctypes.CDLL(libpath)
-    for fn in ("lsao_nmi_select", "lsao_nmi_select_union", "lsao_select_baseline", "lsao_li_scores", "lsao_topk_select", "lsao_topk_select_f32",
+    for fn in ("lsao_nmi_select", "lsao_nmi_select_union", "lsao_select_baseline", "lsao_query_encoder",
+               "lsao_li_scores", "lsao_topk_select", "lsao_topk_select_f32",
                "lsao_attention_dense", "lsao_decode_step", "lsao_nucleus", "lsao_label_vote"):
         getattr(mutant, fn).argtypes = getattr(real, fn).argtypes
         getattr(mutant, fn).restype = ctypes.c_int
