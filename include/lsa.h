@@ -127,6 +127,33 @@ int lsa_nmi_select_union(int n_idx, const lsa_bf16 *const *q, const lsa_bf16 *co
 size_t lsa_nmi_select_union_workspace_size(int n_idx, int B, int max_chunks_per_seq);
 
 /*
+ * Memory-indexer query encoder: the hidden state h_t of each token mapped to
+ * the gate's low-rank queries and head weights (the inputs of lsa_nmi_select).
+ * Passage: gist.science explainer 2.1 ("Memory Indexer": a dual encoder maps
+ * h_t to low-rank indexer queries) and 2.3 (only the query encoder's low-rank
+ * projections are trained); cjcn.com.cn article section 4 (randomly
+ * initialised weights; query projection rank 2048 instead of 1536).
+ *
+ * Reading taken (the pages give no formula): for every token b
+ *   c = W_down h[b]          rank entries
+ *   q[b] = W_up c            Hn * dn entries, head-major (entry h * dn + d)
+ *   w[b] = W_head h[b]       Hn entries
+ * with no normalisation or nonlinearity.  Products accumulate in fp32; c
+ * enters the second product as two bf16 parts (hi = bf16(c), lo = bf16(c - hi)).
+ *
+ *   h       [B, d_model] bf16 (device)
+ *   w_down  [rank, d_model], w_up [Hn * dn, rank], w_head [Hn, d_model] bf16 (device, row-major)
+ *   q_out   [B, Hn, dn] bf16 and w_out [B, Hn] bf16 (device, out): round to nearest even
+ *   q_f32   [B, Hn, dn], w_f32 [B, Hn] fp32 (device, out, optional): before rounding
+ * Supported: 1 <= B <= 32; d_model and rank multiples of 64.
+ */
+int lsa_query_encoder(const lsa_bf16 *h, int B, int d_model, const lsa_bf16 *w_down, int rank,
+                      const lsa_bf16 *w_up, const lsa_bf16 *w_head, int Hn, int dn,
+                      lsa_bf16 *q_out, lsa_bf16 *w_out, float *q_f32, float *w_f32, int32_t *dev_status,
+                      void *ws, size_t ws_bytes, lsa_stream_t stream);
+size_t lsa_query_encoder_workspace_size(int B, int d_model, int rank, int Hn, int dn);
+
+/*
  * Baseline selectors: the two schemes the pages compare LSA with, producing a
  * kept list in the same form as lsa_nmi_select so that the same top-k,
  * attention and fetch calls run after them.

@@ -36,6 +36,8 @@ def _load():
         "lsa_nmi_select_workspace_size": ([I, I], SZ),
         "lsa_nmi_select_union": ([I, P, P, P, P, I, I, I, I64, I, P, P, I, P, P, P, SZ, P], I),
         "lsa_nmi_select_union_workspace_size": ([I, I, I], SZ),
+        "lsa_query_encoder": ([P, I, I, P, I, P, P, I, I, P, P, P, P, P, P, SZ, P], I),
+        "lsa_query_encoder_workspace_size": ([I, I, I, I, I], SZ),
         "lsa_select_baseline": ([I, P, I, I, ctypes.c_uint64, I, I, P, P, I, P, P, SZ, P], I),
         "lsa_select_baseline_workspace_size": ([I, I], SZ),
         "lsa_topk": ([P, P, P, I64, P, I, P, P, I, P, I, I, I, I, P, P, P, P, P, SZ, P], I),
@@ -149,6 +151,32 @@ def nmi_select_union(qs, ws_, khats, seq_chunk_offset, max_chunks_per_seq, kept_
                                      khats[0].shape[0], max_chunks_per_seq, _ptr(kept_idx), _ptr(kept_count),
                                      kept_cap, _ptr(logits), _ptr(status), _ptr(ws), ws.numel(), _stream(stream)))
     return kept_idx, kept_count
+
+
+def query_encoder_workspace_size(B, d_model, rank, Hn, dn):
+    return _lib.lsa_query_encoder_workspace_size(B, d_model, rank, Hn, dn)
+
+
+def query_encoder(h, w_down, w_up, w_head, Hn, dn, *, q_out=None, w_out=None, q_f32=None, w_f32=None, status=None,
+                  ws=None, stream=None):
+    """Indexer queries from hidden states: h [B, d_model] -> (q [B, Hn, dn] bf16, w [B, Hn] bf16)."""
+    for name, t in (("h", h), ("w_down", w_down), ("w_up", w_up), ("w_head", w_head)):
+        _dev(t, torch.bfloat16, name)
+    B, d_model = h.shape
+    rank = w_down.shape[0]
+    if tuple(w_down.shape) != (rank, d_model) or tuple(w_up.shape) != (Hn * dn, rank) or \
+            tuple(w_head.shape) != (Hn, d_model):
+        raise LSAError(1, "query_encoder: weight shapes do not match h, rank, Hn and dn")
+    dev = h.device
+    if q_out is None:
+        q_out = torch.empty(B, Hn, dn, dtype=torch.bfloat16, device=dev)
+    if w_out is None:
+        w_out = torch.empty(B, Hn, dtype=torch.bfloat16, device=dev)
+    ws = _ws(query_encoder_workspace_size(B, d_model, rank, Hn, dn), dev, ws)
+    _check(_lib.lsa_query_encoder(_ptr(h), B, d_model, _ptr(w_down), rank, _ptr(w_up), _ptr(w_head), Hn, dn,
+                                  _ptr(q_out), _ptr(w_out), _ptr(q_f32), _ptr(w_f32), _ptr(status), _ptr(ws),
+                                  ws.numel(), _stream(stream)))
+    return q_out, w_out
 
 
 SELECT_RECENT, SELECT_RANDOM = 0, 1

@@ -29,4 +29,5 @@ from .generate import (  # noqa: F401
     to_bf16_bits, bf16_bits_to_f32, normal_bf16,
     nmi_inputs, resident_layout, cold_layout, chunk_rows, kv_pools, host_pool,
     step_inputs, label_vote_scores, redraw_slice, nudge_bits,
+    encoder_inputs, ENCODER_D_MODEL, ENCODER_RANK,
 )

@@ -10,7 +10,7 @@ WINDOW = 8000   # recent tokens that always stay on the GPU (125 chunks)
 STEPS = 64      # decode steps per lookahead window
 
 # stream ids: one independent random stream per kind of input
-_S_NMI, _S_PLANT, _S_KV, _S_LI, _S_STEP, _S_VOTE, _S_CTX = 1, 2, 3, 4, 5, 6, 7
+_S_NMI, _S_PLANT, _S_KV, _S_LI, _S_STEP, _S_VOTE, _S_CTX, _S_ENC = 1, 2, 3, 4, 5, 6, 7, 8
 _BLOCK_CHUNKS = 256
 
 
@@ -255,6 +255,25 @@ def host_pool(wl: Workload, b: int = 0):
     """Every chunk of sequence b in host layout [n_ch, 64, width] (cold tier)."""
     kinds = ["kv", "li"] if wl.latent else ["k", "v", "li"]
     return {kind: chunk_rows(wl, b, 0, wl.n_ch[b], kind) for kind in kinds}
+
+
+# ------------------------------------------------------- query encoder (f3) --
+
+ENCODER_D_MODEL = 4096   # hidden size of the synthetic backbone (the pages give none)
+ENCODER_RANK = 2048      # low-rank dimension of the indexer's query projection
+
+
+def encoder_inputs(wl: Workload, d_model: int = ENCODER_D_MODEL, rank: int = ENCODER_RANK, seed_offset: int = 0):
+    """Hidden states and randomly initialised encoder weights (bf16 bits).
+
+    h ~ N(0, 1) [B, d_model]; W_down ~ N(0, 1/d_model) [rank, d_model];
+    W_up ~ N(0, 1/rank) [Hn*dn, rank]; W_head ~ N(0, 1/d_model) [Hn, d_model].
+    """
+    r = _rng(wl.seed + seed_offset, _S_ENC)
+    return dict(h=normal_bf16(r, (wl.B, d_model)),
+                w_down=normal_bf16(r, (rank, d_model), math.sqrt(1.0 / d_model)),
+                w_up=normal_bf16(r, (wl.Hn * wl.dn, rank), math.sqrt(1.0 / rank)),
+                w_head=normal_bf16(r, (wl.Hn, d_model), math.sqrt(1.0 / d_model)))
 
 
 # ---------------------------------------------------------- per-step inputs --

@@ -199,6 +199,63 @@ def test_select_baseline_rejects_a_too_small_capacity(L):
     assert e.value.code == 4
 
 
+# ------------------------------------------------------- query encoder (f3) --
+
+def _bf16_rne(x):
+    return W.to_bf16_bits(np.asarray(x, np.float32))
+
+
+@pytest.mark.parametrize("shape", ["decode_128k_b8_mla", "decode_512k_b1_mla_cold", "b32", "small"])
+def test_query_encoder_matches_oracle(L, shape):
+    """fp32 outputs within a bound derived from the arithmetic: fp32 accumulation over K terms
+    and c carried as two bf16 parts (about 2^-16 relative) stay far below
+    1e-4 x (|W_up| |W_down| |h|); the bf16 outputs are the round-to-nearest-even of the fp32
+    ones and within one bf16 step of the rounded oracle."""
+    if shape == "b32":
+        wl = W.workload("decode_128k_b8_mla", B=32, ctx=(16384,) * 32, pass_rate=(0.1,) * 32)
+        kw = {}
+    elif shape == "small":
+        wl = W.workload("decode_16k_b1_h16", B=3, ctx=(16384,) * 3, pass_rate=(0.1,) * 3)
+        kw = dict(d_model=192, rank=128)
+    else:
+        wl = W.workload(shape)
+        kw = {}
+    e = W.encoder_inputs(wl, **kw)
+    d = dev()
+    q_f32 = torch.empty(wl.B, wl.Hn, wl.dn, dtype=torch.float32, device=d)
+    w_f32 = torch.empty(wl.B, wl.Hn, dtype=torch.float32, device=d)
+    status = torch.zeros(1, dtype=torch.int32, device=d)
+    q, w = L.query_encoder(bf16(e["h"], d), bf16(e["w_down"], d), bf16(e["w_up"], d), bf16(e["w_head"], d),
+                           wl.Hn, wl.dn, q_f32=q_f32, w_f32=w_f32, status=status)
+    assert status.item() == 0
+    ref_q, ref_w = oracle.query_encoder(e["h"], e["w_down"], e["w_up"], e["w_head"], wl.Hn, wl.dn)
+    f = lambda a: W.bf16_bits_to_f32(a).astype(np.float64)
+    H_, WD, WU, WH = np.abs(f(e["h"])), np.abs(f(e["w_down"])), np.abs(f(e["w_up"])), np.abs(f(e["w_head"]))
+    bound_q = 1e-4 * ((H_ @ WD.T) @ WU.T).reshape(ref_q.shape) + 1e-30
+    bound_w = 1e-4 * (H_ @ WH.T) + 1e-30
+    gq, gw = q_f32.cpu().numpy().astype(np.float64), w_f32.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(gq - ref_q) <= bound_q), float(np.max(np.abs(gq - ref_q) / bound_q))
+    assert np.all(np.abs(gw - ref_w) <= bound_w), float(np.max(np.abs(gw - ref_w) / bound_w))
+    qb = q.view(torch.int16).cpu().numpy().view(np.uint16)
+    wb = w.view(torch.int16).cpu().numpy().view(np.uint16)
+    np.testing.assert_array_equal(qb, _bf16_rne(gq))
+    np.testing.assert_array_equal(wb, _bf16_rne(gw))
+    for got, ref in ((qb, ref_q), (wb, ref_w)):
+        step = np.abs(f(got) - f(_bf16_rne(ref)))
+        ulp = np.abs(f(_bf16_rne(ref))) * 2.0 ** -7 + 1e-30
+        assert np.all(step <= ulp)
+
+
+def test_query_encoder_rejects_too_many_tokens(L):
+    d = dev()
+    h = torch.zeros(33, 128, dtype=torch.bfloat16, device=d)
+    wd = torch.zeros(64, 128, dtype=torch.bfloat16, device=d)
+    with pytest.raises(L.LSAError) as e:
+        L.query_encoder(h, wd, torch.zeros(64, 64, dtype=torch.bfloat16, device=d),
+                        torch.zeros(8, 128, dtype=torch.bfloat16, device=d), 8, 8)
+    assert e.value.code == 2
+
+
 # -------------------------------------------------------------- a2 + a3 ---
 
 def _small_mla(**kw):
