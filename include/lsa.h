@@ -262,6 +262,23 @@ int lsa_sparse_decode(const lsa_bf16 *q, const lsa_bf16 *k_pool, int64_t k_row_s
 size_t lsa_sparse_decode_workspace_size(int B, int Hq, int dqk, int dv, int k, int max_window_len);
 
 /*
+ * a4 -- merge of attention results over disjoint row sets of the same queries.
+ * Passage: as lsa_sparse_decode (softmax attention over the union of the row
+ * sets); the split itself is this library's: the window rows and the top-k
+ * rows of a step can be attended in two calls (the window part while cold
+ * chunks are still being fetched), and a long sequence can be attended in
+ * pieces, one per device.
+ *
+ *   o_parts [R, B, Hq, dv], lse_parts [R, B, Hq] fp32 (device): part r as written
+ *   by lsa_sparse_decode over its rows (lse_r = -inf for a part without rows)
+ *   out [B, Hq, dv], lse [B, Hq] (optional) fp32 (device, out):
+ *     lse = log sum_r exp(lse_r),  out = sum_r exp(lse_r - lse) o_r
+ *   (no rows in any part: out = 0, lse = -inf).  dv a multiple of 4.
+ */
+int lsa_merge_attention(const float *o_parts, const float *lse_parts, int R, int B, int Hq, int dv,
+                        float *out, float *lse, lsa_stream_t stream);
+
+/*
  * a5 -- lookahead reuse: append the decoded token to the recent window.
  * Passage: gist.science explainer 2.1 ("Periodische Triggerung", tau = 64);
  * cjcn.com.cn article section 2 (the selection serves the next 64 steps).
@@ -302,6 +319,62 @@ int lsa_gather_chunks(int n_pools, const void *const *host_pools, const size_t *
                       const int32_t *kept_idx_host, int kept_count_host, int first_window_chunk,
                       int first_free_slot, int32_t *chunk_table_host, int32_t *chunk_table_dev,
                       int table_len, lsa_stream_t stream, lsa_event_t done, int *n_fetched);
+
+/*
+ * a6, device-driven -- residency plan of the next lookahead window (one sequence).
+ * Passage: cjcn.com.cn article section 2 (every 64 steps the indexer predicts
+ * the chunks the next 64 steps will need and only those are moved from the
+ * CPU cold pool to GPU memory); gist.science explainer 2.1 ("Dynamisches
+ * Fetching" from the CPU cold pool).
+ *
+ * The next window needs its window chunks [first_window_chunk,
+ * window_end_chunk) -- the last of them receives the window's appended tokens --
+ * and every chunk of the kept list (kept_idx[0 .. kept_count[0]), device, as
+ * written by lsa_nmi_select with B = 1).  table_next (device, out, table_len
+ * entries) keeps the slot of every needed chunk that table_cur already maps,
+ * gives every other needed chunk a slot that table_cur leaves free (ascending
+ * chunk and slot order), and holds -1 elsewhere.  Needed chunks before the
+ * window that received a new slot are the copy list: copy_chunk / copy_slot
+ * (device, out, ascending chunk order) and copy_count[0] (device, out).  So only
+ * the delta against what is resident moves, and slots of chunks that are no
+ * longer needed are free again once table_next replaces table_cur.
+ * Not enough free slots, or more than copy_cap copies, sets LSA_DEV_CAPACITY
+ * (the chunks without a slot get -1).  Slots are < n_slots.
+ * Nothing here waits for the host: the call can run on a side stream while the
+ * current window's steps run, since it only reads table_cur.
+ */
+int lsa_plan_residency(const int32_t *table_cur, int32_t *table_next, int table_len,
+                       const int32_t *kept_idx, const int32_t *kept_count, int kept_cap,
+                       int first_window_chunk, int window_end_chunk, int64_t n_slots,
+                       int32_t *copy_chunk, int32_t *copy_slot, int32_t *copy_count, int copy_cap,
+                       int32_t *dev_status, void *ws, size_t ws_bytes, lsa_stream_t stream);
+size_t lsa_plan_residency_workspace_size(int table_len, int64_t n_slots);
+
+/*
+ * a6, device-driven -- copy listed chunks from the pinned host pools.
+ * Passage: as lsa_plan_residency.
+ *
+ * For j < copy_count[0] (device): chunk copy_chunk[j] of every pool i is copied
+ * from host_pools[i] + copy_chunk[j] * chunk_bytes[i] to dev_pools[i] +
+ * copy_slot[j] * chunk_bytes[i].  A kernel reads the host pools through their
+ * device mapping over the host link (one launch for the whole list, no
+ * per-chunk copy calls and no host round trip for the list).  host_pools[i]
+ * must be page-locked host memory (cudaHostAlloc / cudaHostRegister; checked,
+ * LSA_ERR_INVALID_ARG otherwise); chunk_bytes[i] a multiple of 16.  A chunk or
+ * slot out of range is skipped and sets LSA_DEV_TABLE.
+ */
+int lsa_fetch_chunks(int n_pools, const void *const *host_pools, const size_t *chunk_bytes,
+                     void *const *dev_pools, int64_t n_host_chunks, int64_t n_slots,
+                     const int32_t *copy_chunk, const int32_t *copy_slot, const int32_t *copy_count,
+                     int copy_cap, int32_t *dev_status, lsa_stream_t stream);
+
+/*
+ * a5 -- start of the next lookahead window: window_start[b] += by (a multiple of
+ * 64: the window slides by the tokens decoded in the last window) and
+ * window_len[b] = new_len, for every b < B (device arrays).
+ */
+int lsa_advance_window(int32_t *window_start, int32_t *window_len, int B, int by, int new_len,
+                       lsa_stream_t stream);
 
 /*
  * a7 (offline) -- cross-layer majority-vote labels for one decode window.

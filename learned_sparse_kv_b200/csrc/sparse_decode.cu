@@ -345,6 +345,36 @@ static int launch_merge(const float *o_part, const float *m_part, const float *l
     return check_launch("lse_merge_kernel");
 }
 
+// Merge of R attention results of the same queries over disjoint row sets, each
+// already normalised (o_r = softmax-weighted mean over its rows, lse_r = log of
+// its exp-sum):  lse = log sum_r exp(lse_r),  out = sum_r exp(lse_r - lse) o_r.
+// A part without rows (lse_r = -inf) adds nothing; with no rows at all the
+// result is out = 0, lse = -inf.  grid B * Hq, one float4 column group per thread.
+__global__ void __launch_bounds__(128) part_merge_kernel(const float *__restrict__ o_parts,
+                                                         const float *__restrict__ lse_parts, int R, int BH, int dv,
+                                                         float *__restrict__ out, float *__restrict__ lse) {
+    const int row = blockIdx.x;   // (b, h)
+    float M = -INFINITY;
+    for (int r = 0; r < R; ++r) M = fmaxf(M, lse_parts[(size_t)r * BH + row]);
+    float L = 0.f;
+    for (int r = 0; r < R; ++r) {
+        const float x = lse_parts[(size_t)r * BH + row];
+        L += x == -INFINITY ? 0.f : expf(x - M);
+    }
+    for (int c = threadIdx.x; c < dv / 4; c += blockDim.x) {
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int r = 0; r < R; ++r) {
+            const float x = lse_parts[(size_t)r * BH + row];
+            if (x == -INFINITY) continue;
+            const float w = expf(x - M) / L;
+            const float4 v = reinterpret_cast<const float4 *>(o_parts + ((size_t)r * BH + row) * dv)[c];
+            a.x += w * v.x; a.y += w * v.y; a.z += w * v.z; a.w += w * v.w;
+        }
+        reinterpret_cast<float4 *>(out + (size_t)row * dv)[c] = a;
+    }
+    if (lse && threadIdx.x == 0) lse[row] = L > 0.f ? M + logf(L) : -INFINITY;
+}
+
 using CfgSep16 = DecodeCfg<16, 128, 128, 4, false>;
 using CfgMla64 = DecodeCfg<64, 576, 512, 8, true>;
 
@@ -470,4 +500,13 @@ extern "C" int lsa_sparse_decode(const lsa_bf16 *q, const lsa_bf16 *k_pool, int6
     if (rc) return rc;
     return dv == 512 ? launch_merge<512>(o_part, m_part, l_part, ns, Hq, B, out, lse, stream)
                      : launch_merge<128>(o_part, m_part, l_part, ns, Hq, B, out, lse, stream);
+}
+
+extern "C" int lsa_merge_attention(const float *o_parts, const float *lse_parts, int R, int B, int Hq, int dv,
+                                   float *out, float *lse, lsa_stream_t stream) {
+    LSA_REQUIRE(o_parts && lse_parts && out, LSA_ERR_INVALID_ARG, "lsa_merge_attention: null pointer");
+    LSA_REQUIRE(R >= 1 && B >= 1 && Hq >= 1 && dv >= 4 && dv % 4 == 0 && (int64_t)B * Hq < (1 << 30),
+                LSA_ERR_INVALID_ARG, "lsa_merge_attention: bad sizes (R=%d B=%d Hq=%d dv=%d)", R, B, Hq, dv);
+    part_merge_kernel<<<B * Hq, 128, 0, stream>>>(o_parts, lse_parts, R, B * Hq, dv, out, lse);
+    return check_launch("part_merge_kernel");
 }

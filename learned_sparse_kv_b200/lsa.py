@@ -46,8 +46,13 @@ def _load():
         "lsa_topk_from_scores": ([P, P, I, I, I, P, P, P, SZ, P], I),
         "lsa_sparse_decode": ([P, P, I64, P, I64, I64, P, I, P, P, I, P, P, I, I, I, I, I, F, P, P, P, P, SZ, P], I),
         "lsa_sparse_decode_workspace_size": ([I, I, I, I, I, I], SZ),
+        "lsa_merge_attention": ([P, P, I, I, I, I, P, P, P], I),
         "lsa_append_token": ([P, P, P, P, I64, I, P, I64, I, P, I, I64, P, I, P, P, I, P, P], I),
         "lsa_gather_chunks": ([I, P, P, P, I64, I64, P, I, I, I, P, P, I, P, P, P], I),
+        "lsa_plan_residency": ([P, P, I, P, P, I, I, I, I64, P, P, P, I, P, P, SZ, P], I),
+        "lsa_plan_residency_workspace_size": ([I, I64], SZ),
+        "lsa_fetch_chunks": ([I, P, P, P, I64, I64, P, P, P, I, P, P], I),
+        "lsa_advance_window": ([P, P, I, I, I, P], I),
         "lsa_label_vote": ([P, I, I, I, F, I, I, P, P, P, SZ, P], I),
         "lsa_label_vote_workspace_size": ([I, I, I], SZ),
         "lsa_last_error": ([], ctypes.c_char_p),
@@ -281,6 +286,19 @@ def sparse_decode(q, k_pool, v_pool, chunk_table, topk_idx, topk_count, window_s
     return out, lse
 
 
+def merge_attention(o_parts, lse_parts, *, out=None, lse=None, stream=None):
+    """o_parts [R, B, Hq, dv], lse_parts [R, B, Hq] fp32 -> (out [B, Hq, dv], lse [B, Hq])."""
+    _dev(o_parts, torch.float32, "o_parts"); _dev(lse_parts, torch.float32, "lse_parts")
+    R, B, Hq, dv = o_parts.shape
+    if out is None:
+        out = torch.empty(B, Hq, dv, dtype=torch.float32, device=o_parts.device)
+    if lse is None:
+        lse = torch.empty(B, Hq, dtype=torch.float32, device=o_parts.device)
+    _check(_lib.lsa_merge_attention(_ptr(o_parts), _ptr(lse_parts), R, B, Hq, dv, _ptr(out), _ptr(lse),
+                                    _stream(stream)))
+    return out, lse
+
+
 # ------------------------------------------------------------- a5, a6 ----
 
 def append_token(new_k, new_v, new_li, k_pool, v_pool, li_pool, chunk_table, window_start, window_len, *,
@@ -318,6 +336,42 @@ def gather_chunks(host_pools, dev_pools, kept_idx_host, first_window_chunk, firs
                                   _ptr(chunk_table_dev), chunk_table_host.numel(), _stream(stream),
                                   None if done is None else ctypes.c_void_p(done.cuda_event), ctypes.byref(nf)))
     return nf.value
+
+
+def plan_residency_workspace_size(table_len, n_slots):
+    return _lib.lsa_plan_residency_workspace_size(table_len, n_slots)
+
+
+def plan_residency(table_cur, table_next, kept_idx, kept_count, first_window_chunk, window_end_chunk, n_slots,
+                   copy_chunk, copy_slot, copy_count, *, status=None, ws=None, stream=None):
+    """Next window's chunk table and copy list (device tensors, one sequence)."""
+    for name, t in (("table_cur", table_cur), ("table_next", table_next), ("kept_idx", kept_idx),
+                    ("kept_count", kept_count), ("copy_chunk", copy_chunk), ("copy_slot", copy_slot),
+                    ("copy_count", copy_count)):
+        _dev(t, torch.int32, name)
+    n = table_cur.numel()
+    ws = _ws(plan_residency_workspace_size(n, n_slots), table_cur.device, ws)
+    _check(_lib.lsa_plan_residency(_ptr(table_cur), _ptr(table_next), n, _ptr(kept_idx), _ptr(kept_count),
+                                   kept_idx.numel(), first_window_chunk, window_end_chunk, n_slots, _ptr(copy_chunk),
+                                   _ptr(copy_slot), _ptr(copy_count), copy_chunk.numel(), _ptr(status), _ptr(ws),
+                                   ws.numel(), _stream(stream)))
+
+
+def fetch_chunks(host_pools, dev_pools, copy_chunk, copy_slot, copy_count, *, status=None, stream=None):
+    """Copies the listed chunks from pinned host pools [n_chunks, ...] into device pools [n_slots, ...]."""
+    n = len(host_pools)
+    HP = (ctypes.c_void_p * n)(*[t.data_ptr() for t in host_pools])
+    DP = (ctypes.c_void_p * n)(*[t.data_ptr() for t in dev_pools])
+    CB = (ctypes.c_size_t * n)(*[t[0].numel() * t.element_size() for t in host_pools])
+    _check(_lib.lsa_fetch_chunks(n, HP, CB, DP, host_pools[0].shape[0], dev_pools[0].shape[0], _ptr(copy_chunk),
+                                 _ptr(copy_slot), _ptr(copy_count), copy_chunk.numel(), _ptr(status),
+                                 _stream(stream)))
+
+
+def advance_window(window_start, window_len, by, new_len, *, stream=None):
+    _dev(window_start, torch.int32, "window_start"); _dev(window_len, torch.int32, "window_len")
+    _check(_lib.lsa_advance_window(_ptr(window_start), _ptr(window_len), window_start.numel(), by, new_len,
+                                   _stream(stream)))
 
 
 # ------------------------------------------------------------------- a7 ----

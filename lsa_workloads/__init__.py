@@ -27,7 +27,7 @@ definition):
 from .generate import (  # noqa: F401
     CHUNK, WINDOW, STEPS, Workload, WORKLOADS, LABEL_VOTE, workload,
     to_bf16_bits, bf16_bits_to_f32, normal_bf16,
-    nmi_inputs, resident_layout, cold_layout, chunk_rows, kv_pools, host_pool,
+    nmi_inputs, next_window_plant, resident_layout, cold_layout, chunk_rows, kv_pools, host_pool,
     step_inputs, label_vote_scores, redraw_slice, nudge_bits,
     encoder_inputs, ENCODER_D_MODEL, ENCODER_RANK,
 )

@@ -17,7 +17,7 @@ chunks and the oracle view is the whole host pool.
 import numpy as np
 import torch
 
-from .generate import (CHUNK, Workload, cold_layout, host_pool, kv_pools, nmi_inputs, resident_layout,
+from .generate import (CHUNK, Workload, cold_layout, host_pool, kv_pools, next_window_plant, nmi_inputs, resident_layout,
                        step_inputs)
 
 
@@ -56,40 +56,57 @@ BF16_NAN = np.uint16(0x7FC0)
 
 
 def _poison_new_rows(wl, pools, table, steps):
-    """bf16 NaN in the device rows of the tokens appended during the window."""
+    """bf16 NaN in the device rows of the tokens appended during the window (where the
+    table already gives their chunk a slot)."""
     for s in range(steps):
         for b in range(wl.B):
             pos = wl.ctx[b] + s
             slot, row = table[b, pos // CHUNK], pos % CHUNK
+            if slot < 0:
+                continue
             for k in pools:
                 pools[k][slot, row] = BF16_NAN
 
 
 def host_build(wl: Workload, steps: int = None, nmi=None, structural: bool = True, fetch_fraction: float = 0.25,
-               n_indexers: int = 1):
+               n_indexers: int = 1, windows: int = 1, overlap: float = 0.8):
     """Host-side arrays of one window.  With n_indexers > 1 the gate is the OR-mode union of
     that many independent indexers (host["nmi_union"]: one nmi_inputs() draw each, the
-    first being host["nmi"])."""
+    first being host["nmi"]).  With windows > 1 (cold workloads) the arrays cover that many
+    consecutive lookahead windows: steps 64 w .. 64 w + 63 belong to window w, whose
+    context is ctx + 64 w and whose gate inputs are host["nmi_windows"][w] (its plant keeps
+    `overlap` of the previous window's)."""
     steps = wl.steps if steps is None else steps
     assert all(L % CHUNK == 0 and L >= wl.window for L in wl.ctx), "contexts are whole chunks, at least the window"
     assert steps <= CHUNK, "one lookahead window appends at most one chunk"
+    assert windows == 1 or (wl.cold and steps == CHUNK), "several windows: cold workloads of full windows"
     nm = nmi if nmi is not None else nmi_inputs(wl, structural=structural)
+    first_steps = steps
+    steps = steps * windows
     st = stacked_steps(wl, steps)
     host = dict(wl=wl, steps=steps, nmi=nm, step=st, max_chunks=max(wl.n_ch), kept_cap=max(wl.n_ch))
+    if windows > 1:
+        nws = [nm]
+        for w in range(1, windows):
+            plant = next_window_plant(wl, nws[-1]["planted"], w, overlap)
+            nws.append(nmi_inputs(wl.shrink(ctx=tuple(L + CHUNK * w for L in wl.ctx)), structural=structural,
+                                  seed_offset=1000 * w, planted=plant))
+        host["nmi_windows"] = nws
+    host["windows"] = windows
     if n_indexers > 1:
         host["nmi_union"] = [nm] + [nmi_inputs(wl, structural=structural, seed_offset=101 * i)
                                     for i in range(1, n_indexers)]
     if wl.cold:
-        lay = cold_layout(wl, kept_cap=int(np.ceil(fetch_fraction * wl.n_ch[0])))
+        lay = cold_layout(wl, kept_cap=int(np.ceil(fetch_fraction * wl.n_ch[0])), windows=windows)
         fw = lay["first_window_chunk"]
         host["pools"] = kv_pools(wl, lay, chunks_of=lambda b: np.arange(fw, wl.n_ch[b]))
         hp = host_pool(wl, 0)
         host["cold_pools"] = hp
-        # oracle view: chunk c at slot c, the appended chunk at slot n_ch
-        otab = np.arange(wl.n_ch[0] + 1, dtype=np.int32)[None, :]
-        opools = {k: np.concatenate([hp[k], np.zeros((1,) + hp[k].shape[1:], np.uint16)]) for k in _kinds(wl)}
+        # oracle view: chunk c at slot c, the appended chunk of window w at slot n_ch + w
+        otab = np.arange(wl.n_ch[0] + windows, dtype=np.int32)[None, :]
+        opools = {k: np.concatenate([hp[k], np.zeros((windows,) + hp[k].shape[1:], np.uint16)]) for k in _kinds(wl)}
         _write_new_rows(wl, opools, otab, st, steps)
-        _poison_new_rows(wl, host["pools"], lay["chunk_table"], steps)
+        _poison_new_rows(wl, host["pools"], lay["chunk_table"], first_steps)
         host.update(oracle_pools=opools, oracle_table=otab, first_window_chunk=fw, first_free_slot=lay["fetch_base"])
     else:
         lay = resident_layout(wl)
@@ -127,6 +144,10 @@ def upload(host, device):
                     dev_pools=[t[k] for k in _kinds(wl)],
                     first_window_chunk=host["first_window_chunk"], first_free_slot=host["first_free_slot"],
                     table_host=torch.from_numpy(host["chunk_table"][0].copy()).pin_memory())
+    if host.get("windows", 1) > 1:
+        t["nmi_windows"] = [(bf16(n["q"], device), bf16(n["w"], device), bf16(n["khat"], device),
+                             torch.from_numpy(n["seq_chunk_offset"]).to(device)) for n in host["nmi_windows"]]
     shapes = dict(B=wl.B, Hn=wl.Hn, dn=wl.dn, Hl=wl.Hl, dl=wl.dl, k=wl.k, Hq=wl.Hq, dqk=wl.dqk, dv=wl.dv,
-                  latent=wl.latent, window=wl.window, steps=host["steps"], scale=wl.scale)
+                  latent=wl.latent, window=wl.window, steps=host["steps"] // host.get("windows", 1),
+                  scale=wl.scale)
     return shapes, t, host["max_chunks"], host["kept_cap"], cold

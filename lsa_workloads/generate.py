@@ -124,7 +124,7 @@ def _with_sign(mag_bits: np.ndarray, negative: np.ndarray) -> np.ndarray:
 
 # ----------------------------------------------------------------- NMI (a1) --
 
-def nmi_inputs(wl: Workload, structural: bool = True, seed_offset: int = 0):
+def nmi_inputs(wl: Workload, structural: bool = True, seed_offset: int = 0, planted=None):
     """NMI query heads, head weights, one compressed key per chunk, planted set.
 
     q, w ~ N(0, 1/8) and khat ~ N(0, 1) marginally (bf16 bits).  With
@@ -134,7 +134,9 @@ def nmi_inputs(wl: Workload, structural: bool = True, seed_offset: int = 0):
     other key -sigma_d.  Every term w_h * q_hd * khat_d then has the chunk's
     sign, so exactly the planted chunks pass, far from the threshold.  Without
     `structural` all entries are independent (the caller decides the set).
+    `planted` (one ascending index array per sequence) replaces the random plant.
     """
+    given = planted
     r = _rng(wl.seed + seed_offset, _S_NMI)
     B, Hn, dn = wl.B, wl.Hn, wl.dn
     std8 = math.sqrt(1.0 / 8.0)
@@ -149,6 +151,8 @@ def nmi_inputs(wl: Workload, structural: bool = True, seed_offset: int = 0):
     for b in range(B):
         cnt = int(round(wl.pass_rate[b] * n_ch[b]))
         planted.append(np.sort(pr.choice(n_ch[b], size=cnt, replace=False)).astype(np.int32))
+    if given is not None:
+        planted = [np.asarray(x, np.int32) for x in given]
     if structural:
         sigma_neg = pr.integers(0, 2, size=(B, dn)).astype(bool)
         w_neg = (w >> np.uint16(15)).astype(bool)
@@ -159,6 +163,23 @@ def nmi_inputs(wl: Workload, structural: bool = True, seed_offset: int = 0):
             rows = slice(int(off[b]), int(off[b + 1]))
             khat[rows] = _with_sign(khat[rows], sigma_neg[b][None, :] ^ (~mark)[:, None])
     return dict(q=q, w=w, khat=khat, seq_chunk_offset=off, planted=planted)
+
+
+def next_window_plant(wl: Workload, prev_planted, window: int, overlap: float = 0.8):
+    """Planted chunks of lookahead window `window` (context ctx + 64 * window), given those of
+    the window before: a random `overlap` share of the previous plant stays, and new random
+    chunks bring the count back to pass_rate of the grown chunk count."""
+    out = []
+    for b in range(wl.B):
+        r = _rng(wl.seed, _S_PLANT, 1000 + window, b)
+        n_ch = wl.n_ch[b] + window
+        prev = np.asarray(prev_planted[b])
+        keep = r.choice(prev, size=int(round(overlap * prev.size)), replace=False) if prev.size else prev
+        want = int(round(wl.pass_rate[b] * n_ch))
+        pool = np.setdiff1d(np.arange(n_ch), keep)
+        add = r.choice(pool, size=max(0, min(pool.size, want - keep.size)), replace=False)
+        out.append(np.sort(np.concatenate([keep, add])).astype(np.int32))
+    return out
 
 
 # ------------------------------------------------------------ chunk layout --
@@ -181,17 +202,18 @@ def resident_layout(wl: Workload):
                 window_start=window_start)
 
 
-def cold_layout(wl: Workload, kept_cap: Optional[int] = None):
+def cold_layout(wl: Workload, kept_cap: Optional[int] = None, windows: int = 1):
     """Device slots for the window chunks and the appended chunk; the rest is cold.
 
     Slots 0..124 hold the window chunks in order, slot 125 the appended chunk,
     and slots from 126 on receive fetched cold chunks.  Only batch 1 is laid out.
+    The table has a column for the appended chunk of each of `windows` windows.
     """
     assert wl.B == 1
     n_ch = wl.n_ch[0]
     wc = wl.window // CHUNK
     first_w = n_ch - wc
-    table = np.full((1, n_ch + 1), -1, np.int32)
+    table = np.full((1, n_ch + windows), -1, np.int32)
     table[0, first_w:n_ch + 1] = np.arange(wc + 1)
     fetch_cap = first_w if kept_cap is None else kept_cap
     return dict(chunk_table=table, n_slots=wc + 1 + fetch_cap, fetch_base=wc + 1,

@@ -14,7 +14,13 @@ import lsa_workloads as W
 CH = W.CHUNK
 
 
-def kept_lists(host):
+def kept_lists(host, window=0):
+    """Oracle kept lists of lookahead window `window` (0 unless the host has several)."""
+    if window > 0:
+        nm = host["nmi_windows"][window]
+        lists, logits, _, rc, cnt = oracle.nmi_select(nm["q"], nm["w"], nm["khat"], nm["seq_chunk_offset"],
+                                                      kept_cap=host["kept_cap"])
+        return lists, logits, rc, cnt
     if "selector" in host:
         sel = host["selector"]
         lists, rc, cnt = oracle.select_baseline(sel["mode"], host["window_start"], seed=sel.get("seed", 0),
@@ -53,15 +59,20 @@ def repair_nmi_margin(host, margin=1e-3, rel=1e-4, seed=99, max_iter=50):
     raise AssertionError("could not open NMI margins")
 
 
-def _cand_positions(host, kept, b):
-    fw = int(host["window_start"][b]) // CH
+def window_start(host, b, s):
+    """Window start of sequence b at global step s (steps 64 w .. 64 w + 63 form window w)."""
+    return int(host["window_start"][b]) + CH * (s // W.STEPS)
+
+
+def _cand_positions(host, kept, b, s=0):
+    fw = window_start(host, b, s) // CH
     cold = [int(c) for c in kept if c < fw]
     return np.array([c * CH + r for c in cold for r in range(CH)], np.int64)
 
 
 def li_scores(host, kept, b, s):
     pools, table = host["oracle_pools"], host["oracle_table"][b]
-    pos = _cand_positions(host, kept, b)
+    pos = _cand_positions(host, kept, b, s)
     keys = pools["li"][table[pos // CH], pos % CH] if pos.size else np.zeros((0, host["wl"].dl), np.uint16)
     st = host["step"]
     return pos, oracle.li_scores(st["q_li"][s, b], st["w_li"][s, b], keys)
@@ -106,7 +117,7 @@ def oracle_step(host, kept, b, s, k=None):
     kp = pools["kv"] if wl.latent else pools["k"]
     vp = None if wl.latent else pools["v"]
     return oracle.decode_step(st["q_li"][s, b], st["w_li"][s, b], pools["li"], st["q"][s, b], kp, vp, wl.dv,
-                              wl.scale, table, kept, int(host["window_start"][b]), wl.window + s + 1,
+                              wl.scale, table, kept, window_start(host, b, s), wl.window + s % W.STEPS + 1,
                               wl.k if k is None else k)
 
 

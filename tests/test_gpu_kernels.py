@@ -363,6 +363,42 @@ def test_sparse_decode_matches_oracle(L, shape, q_scale):
             np.testing.assert_allclose(lse[b], refs[b]["lse"], rtol=1e-5, atol=2e-4)
 
 
+def test_merge_of_disjoint_parts_equals_attention_over_their_union(L):
+    """Top-k rows, the first half of the window and the rest of the window attended in three
+    calls (plus an empty fourth part), merged: equals the oracle over all rows at once."""
+    wl = _small_mla(k=400, steps=1)
+    host = host_build(wl)
+    sel = _oracle_topk(host, wl)
+    d = dev()
+    ws0 = host["window_start"].astype(np.int64)
+    half = wl.window // 2
+    parts = [(sel, ws0, np.zeros(wl.B, np.int64)),                                  # top-k only
+             ([np.zeros(0, np.int64)] * wl.B, ws0, np.full(wl.B, half)),           # window, first half
+             ([np.zeros(0, np.int64)] * wl.B, ws0 + half, np.full(wl.B, wl.window - half)),
+             ([np.zeros(0, np.int64)] * wl.B, ws0, np.zeros(wl.B, np.int64))]       # no rows
+    outs, lses = [], []
+    for tsel, wstart, wlen in parts:
+        tk = np.full((wl.B, wl.k), -1, np.int32)
+        tc = np.zeros(wl.B, np.int32)
+        for b in range(wl.B):
+            tk[b, :len(tsel[b])] = tsel[b]
+            tc[b] = len(tsel[b])
+        o, l = L.sparse_decode(bf16(host["step"]["q"][0], d), bf16(host["oracle_pools"]["kv"], d), None,
+                               i32(host["oracle_table"], d), i32(tk, d), i32(tc, d), i32(wstart, d), i32(wlen, d),
+                               wl.window, wl.dv, wl.scale)
+        outs.append(o)
+        lses.append(l)
+    assert bool(torch.isinf(lses[3]).all()) and bool((outs[3] == 0).all())
+    out, lse = L.merge_attention(torch.stack(outs), torch.stack(lses))
+    for b in range(wl.B):
+        pos = np.r_[sel[b], np.arange(int(ws0[b]), int(ws0[b]) + wl.window)]
+        ref, ref_lse = _rows_reference(host, wl, b, pos)
+        H.assert_close_attention(out[b].cpu().numpy(), ref)
+        np.testing.assert_allclose(lse[b].cpu().numpy(), ref_lse, rtol=1e-5, atol=2e-4)
+    empty, empty_lse = L.merge_attention(outs[3][None].contiguous(), lses[3][None].contiguous())
+    assert bool((empty == 0).all()) and bool(torch.isinf(empty_lse).all())
+
+
 def test_sparse_decode_window_only(L):
     wl = _small_mla(k=64, window=CH, steps=1)
     host = host_build(wl)

@@ -170,6 +170,54 @@ def test_window_512k_cold_recency_only_baseline():
     _check_window(host, win, pairs)
 
 
+def test_cold_pipeline_two_windows_fetches_only_the_delta():
+    """Two consecutive lookahead windows on the cold 512K workload.  Window 0's kept cold chunks
+    are fetched by the device-driven plan and fetch while its first step attends the window;
+    window 1's gate, plan and fetch run during window 0, and only the chunks of window 1 that
+    were not resident (its plant keeps 80 % of window 0's) are copied.  Checks: kept lists and
+    copy counts, the bytes of every resident chunk against the host pool, the next table, and
+    oracle parity at sampled steps of both windows (window 0's first, overlapped step included)."""
+    wl = W.workload("decode_512k_b1_mla_cold")
+    host = host_build(wl, windows=2)
+    kept0, _, _, _ = H.kept_lists(host, 0)
+    kept1, _, _, _ = H.kept_lists(host, 1)
+    pairs0, pairs1 = [(0, 0), (0, 29), (0, 63)], [(0, 64), (0, 64 + 41), (0, 127)]
+    for _ in range(2):
+        H.open_topk_gap(host, kept0, pairs0)
+        H.open_topk_gap(host, kept1, pairs1)
+    win = _window(host)
+    assert win.device_status() == 0
+    fw0 = host["first_window_chunk"]
+    cold0 = {int(c) for c in kept0[0] if c < fw0}
+    cold1 = {int(c) for c in kept1[0] if c < fw0 + 1}
+    log = win.fetch_log.cpu().tolist()
+    assert log[0] == len(cold0)
+    assert log[1] == len(cold1 - cold0 - {fw0}) and 0 < log[1] < len(cold1) // 3
+    for w, kept in ((0, kept0), (1, kept1)):
+        c = int(win.kept_count_w[w][0])
+        np.testing.assert_array_equal(win.kept_w[w][0, :c].cpu().numpy(), kept[0])
+    # after window 1: its cold chunks are resident with the host pool's bytes, nothing else before its window
+    table = win.t["chunk_table"][0].cpu().numpy()
+    kv, li = win.t["kv"].cpu().view(torch.int16), win.t["li"].cpu().view(torch.int16)
+    hkv = torch.from_numpy(host["cold_pools"]["kv"].view(np.int16))
+    hli = torch.from_numpy(host["cold_pools"]["li"].view(np.int16))
+    for c in range(fw0 + 1):
+        if c in cold1:
+            assert table[c] >= 0 and torch.equal(kv[table[c]], hkv[c]) and torch.equal(li[table[c]], hli[c])
+        else:
+            assert table[c] == -1
+    assert len({int(table[c]) for c in cold1} | {int(x) for x in table[fw0 + 1:] if x >= 0}) == \
+        len(cold1) + int((table[fw0 + 1:] >= 0).sum())           # no slot serves two chunks
+    tk, tc = win.topk_w.cpu().numpy(), win.topk_count_w.cpu().numpy()
+    for w, kept, pairs in ((0, kept0, pairs0), (1, kept1, pairs1)):
+        for b, s in pairs:
+            ref = H.oracle_step(host, kept[b], b, s)
+            ls = s % W.STEPS
+            np.testing.assert_array_equal(tk[w, ls, b, :tc[w, ls, b]], ref["topk"][:ref["topk_count"]])
+            H.assert_close_attention(win.out_w[w, ls, b].cpu().numpy(), ref["out"])
+            np.testing.assert_allclose(win.lse_w[w, ls, b].cpu().numpy(), ref["lse"], rtol=1e-5, atol=2e-4)
+
+
 def test_window_context_is_window_plus_one_chunk():
     wl = W.workload("decode_128k_b8_mla", B=2, ctx=(8064, 8128), pass_rate=(1.0, 0.5), steps=4)
     host = host_build(wl)
