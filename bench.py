@@ -43,6 +43,7 @@ def parse():
     p.add_argument("--workload", default=DEFAULT_WORKLOAD)
     p.add_argument("--no-cold", action="store_true", help="skip the 512K cold-pool figure")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-extra", action="store_true", help="skip the other workloads, selectors and encoder")
     p.add_argument("--profile-window", action="store_true",
                    help="no timing: run two eager windows of the workload's kernels on 24K-token contexts "
                         "(pools of ~230 MB) for a profiler capture, then exit")
@@ -154,40 +155,59 @@ def barrier(world):
 
 # ------------------------------------------------------------ workload I/O --
 
-def make_window(name, device, seed_offset=0):
+def make_window(name, device, seed_offset=0, selector=None, tensors=None):
+    """A resident workload's window with pools drawn on the device (see upload_fast); `tensors`
+    reuses another window's inputs (same workload) with a different selector."""
     import lsa_workloads as W
-    from lsa_workloads.device import host_build, upload
+    from lsa_workloads.device import upload_fast
     from learned_sparse_kv_b200.decode import Shapes, Window
     wl = W.workload(name)
     if seed_offset:
         wl = wl.shrink(seed=wl.seed + seed_offset)
-    host = host_build(wl)
-    shapes, t, max_ch, kept_cap, cold = upload(host, device)
-    win = Window(Shapes(**shapes), t, max_ch, kept_cap, cold)
-    return wl, host, win
+    if tensors is None:
+        shapes, t, max_ch, kept_cap, cold = upload_fast(wl, device)
+    else:
+        shapes, t, max_ch, kept_cap, cold = tensors
+    win = Window(Shapes(**shapes), t, max_ch, kept_cap, cold, selector=selector)
+    return wl, (shapes, t, max_ch, kept_cap, cold), win
 
 
-def attention_bytes(win):
+def row_bytes(sh):
+    """Bytes of one attended KV row: the latent row, or a K row and a V row."""
+    return sh.dqk * 2 if sh.latent else (sh.dqk + sh.dv) * 2
+
+
+def attention_bytes(win, w=0):
     """Algorithmic bytes of the attention kernel per window: attended KV rows + queries."""
-    tc = win.topk_count.sum().item()
+    tc = win.topk_count_w[w].sum().item()
     B, S, W = win.s.B, win.s.steps, win.s.window
     rows = tc + B * sum(W + s + 1 for s in range(S))
-    return rows * win.s.dqk * 2 + S * B * win.s.Hq * win.s.dqk * 2, rows
+    return rows * row_bytes(win.s) + S * B * win.s.Hq * win.s.dqk * 2, rows
 
 
-def window_bytes(win):
+def attention_flops(win, rows):
+    """Tensor-core work of the attention per window: useful (S = QK^T over dqk, O += PV over dv)
+    and issued (P enters P.V as two bf16 parts in the 128-head latent kernel)."""
+    sh = win.s
+    useful = 2.0 * sh.Hq * rows * (sh.dqk + sh.dv)
+    issued = 2.0 * sh.Hq * rows * (sh.dqk + (2 * sh.dv if (sh.latent and sh.Hq == 128) else sh.dv))
+    return useful, issued
+
+
+def window_bytes(win, w=0, kept=None, kc=None, ws=None):
     """Algorithmic bytes of one whole window (every kernel of the path)."""
-    att, _ = attention_bytes(win)
+    att, _ = attention_bytes(win, w)
     S, B = win.s.steps, win.s.B
-    kc = win.kept_count.cpu().numpy()
-    kept = win.kept_idx.cpu().numpy()
-    ws = win.t["window_start"].cpu().numpy()
+    kc = win.kept_count.cpu().numpy() if kc is None else kc
+    kept = win.kept_idx.cpu().numpy() if kept is None else kept
+    ws = win.t["window_start"].cpu().numpy() if ws is None else ws
     n_cand = sum(int((kept[b, :kc[b]] < ws[b] // 64).sum()) * 64 for b in range(B))
     li = S * n_cand * (win.s.dl * 2 + 4)               # keys read + scores written
     topk = S * (n_cand * 4 + B * win.s.k * 4)          # scores read + positions written
     out = S * B * win.s.Hq * win.s.dv * 4              # attention output
     sel = win.t["khat"].numel() * 2 + B * win.kept_cap * 4
-    return att + li + topk + out + sel
+    append = S * B * (row_bytes(win.s) + win.s.dl * 2) * 2    # new rows read and written
+    return att + li + topk + out + sel + append
 
 
 def sha(*paths):
@@ -269,10 +289,23 @@ def time_attention_kernels(win, windows):
 
 # --------------------------------------------------------------- the arms --
 
+def time_windows(win, n):
+    """Device time of n whole windows (graph replays), ms per window."""
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(n):
+        win.run()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / n
+
+
 def run_lsa(args, world, rank, local):
     device = torch.device("cuda", local)
     hbm_peak, tf_peak, peak_kind = peaks()
-    wl, host, win = make_window(args.workload, device, seed_offset=rank)
+    tf_sustained = sustained_tflops()
+    wl, tensors, win = make_window(args.workload, device, seed_offset=rank)
     win.capture()
     for _ in range(args.warmup):
         win.run()
@@ -302,10 +335,12 @@ def run_lsa(args, world, rank, local):
     att_bytes, att_rows = attention_bytes(win)
     per_launch = att_bytes / wl.steps
     achieved = per_launch / (att_ms / 1e3) / 1e9
+    useful, issued = attention_flops(win, att_rows)
     csrc = os.path.join(ROOT, "learned_sparse_kv_b200", "csrc")
     traffic = recorded_traffic(*(os.path.join(csrc, f) for f in ("sparse_decode_sm100.cu", "sm100.cuh", "common.cuh")))
     wbytes = window_bytes(win)
-    window_gbs = wbytes / (ms_local / args.steps / 1e3) / 1e9
+    step_s = ms_local / args.steps / 1e3
+    window_gbs = wbytes / step_s / 1e9
 
     result = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -316,22 +351,133 @@ def run_lsa(args, world, rank, local):
                    "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2: one window touches ~%.1f GB" % (wbytes / 1e9)},
         "window_gbs": window_gbs, "window_bytes": wbytes,
+        "step_frac": window_gbs / hbm_peak,
         "roofline": {"kernel": "sparse_decode (split-K + merge)", "bound": "hbm", "achieved": achieved,
                      "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": traffic,
                      "peak_kind": peak_kind, "bytes_per_launch": per_launch, "ms_per_launch": att_ms,
-                     "rows_per_launch": att_rows / wl.steps},
+                     "rows_per_launch": att_rows / wl.steps,
+                     "tensor": {"useful_tflops": useful / wl.steps / (att_ms / 1e3) / 1e12,
+                                "issued_tflops": issued / wl.steps / (att_ms / 1e3) / 1e12,
+                                "peak": tf_sustained, "unit": "TFLOP/s", "peak_kind": "measured sustained",
+                                "frac_useful": useful / wl.steps / (att_ms / 1e3) / 1e12 / tf_sustained,
+                                "frac_issued": issued / wl.steps / (att_ms / 1e3) / 1e12 / tf_sustained}},
         "gpu_launches": args.steps * win.launches_per_window(),
         "clocks": clocks, "device_status": status,
     }
     if not args.no_e2e:
         result["e2e"] = run_e2e(win, wl, args, world)
-    if world == 1 and rank == 0 and not args.no_cold:
+    if world == 1 and rank == 0 and not args.no_extra:
+        result["selectors"] = run_selectors(wl, tensors, win, device, args)
+        del win
+        result["configs"] = run_configs(args, device, hbm_peak)
+    if world == 1 and rank == 0:
+        result["cpu_baseline"] = cpu_baseline(wl)
+    return result
+
+
+def sustained_tflops():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d.get("bf16_tflops_sustained", d["bf16_tflops"]))
+    return 1400.0
+
+
+def run_selectors(wl, tensors, win, device, args):
+    """Cost of the same window with the pages' baselines in place of the gate (cjcn.com.cn
+    article section 5): recency only and random 10 % of the older chunks."""
+    from learned_sparse_kv_b200 import lsa
+    out = {"workload": wl.name, "gate": {"tokens_per_s": wl.B * wl.steps / (time_windows(win, 3) / 1e3),
+                                         "kept_chunks": int(win.kept_count.sum())}}
+    for name, sel in (("recency_only", dict(mode=lsa.SELECT_RECENT)),
+                      ("random_10pct", dict(mode=lsa.SELECT_RANDOM, seed=1, keep_num=1, keep_den=10))):
+        _, _, w2 = make_window(wl.name, device, selector=sel, tensors=tensors)
+        w2.capture()
+        w2.run()
+        ms = time_windows(w2, 3)
+        out[name] = {"tokens_per_s": wl.B * wl.steps / (ms / 1e3), "ms_per_window": ms,
+                     "kept_chunks": int(w2.kept_count.sum()), "device_status": w2.device_status()}
+        del w2
+    # restore the gate's state of the shared buffers for whatever runs next
+    win.run()
+    torch.cuda.synchronize()
+    return out
+
+
+def run_configs(args, device, hbm_peak):
+    """Throughput of the other workloads, each against the HBM roofline of the bytes it touches."""
+    out = {}
+    for name in ("decode_16k_b1_h16", "decode_ragged_b32_mla"):
+        wl, _, win = make_window(name, device)
+        win.capture()
+        for _ in range(2):
+            win.run()
+        n = 20 if wl.B == 1 else 4
+        ms = time_windows(win, n)
+        wb = window_bytes(win)
+        out[name] = {"tokens_per_s": wl.B * wl.steps / (ms / 1e3), "ms_per_window": ms, "window_bytes": wb,
+                     "achieved_gbs": wb / (ms / 1e3) / 1e9, "step_frac": wb / (ms / 1e3) / 1e9 / hbm_peak,
+                     "windows_timed": n, "device_status": win.device_status(),
+                     "gpu_launches_per_window": win.launches_per_window()}
         del win
         torch.cuda.empty_cache()
-        result["cold_512k"] = run_cold(args, device)
-    if world == 1 and rank == 0:
-        result["cpu_baseline"] = cpu_baseline(wl, host)
-    return result
+    if not args.no_cold:
+        out[COLD_WORKLOAD] = run_cold(args, device, hbm_peak)
+    out["label_vote_128k_l32"] = run_vote(hbm_peak)
+    out["query_encoder_128k_b8"] = run_encoder(device, hbm_peak)
+    return out
+
+
+def run_vote(hbm_peak):
+    import lsa_workloads as W
+    from learned_sparse_kv_b200 import lsa
+    p = W.LABEL_VOTE
+    d = W.label_vote_scores(p["layers"], p["steps"], p["chunks"], p["planted"], p["seed"])
+    scores = torch.from_numpy(d["scores"]).cuda()
+    ws = torch.empty(lsa.label_vote_workspace_size(p["layers"], p["steps"], p["chunks"]), dtype=torch.uint8,
+                     device="cuda")
+    for _ in range(3):
+        lsa.label_vote(scores, p["top_p"], p["min_layers"], 0, ws=ws)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = 20
+    e0.record()
+    for _ in range(n):
+        lsa.label_vote(scores, p["top_p"], p["min_layers"], 0, ws=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    nbytes = scores.numel() * 4 + p["chunks"] * 5
+    return {"windows_per_s": 1e3 / ms, "ms_per_window": ms, "bytes": nbytes, "achieved_gbs": nbytes / ms / 1e6,
+            "frac": nbytes / ms / 1e6 / hbm_peak, "bound": "latency (2,048 sorts of 2,048 keys)"}
+
+
+def run_encoder(device, hbm_peak):
+    import lsa_workloads as W
+    from lsa_workloads.device import bf16
+    from learned_sparse_kv_b200 import lsa
+    wl = W.workload(DEFAULT_WORKLOAD)
+    e = W.encoder_inputs(wl)
+    h, wd, wu, wh = (bf16(e[k], device) for k in ("h", "w_down", "w_up", "w_head"))
+    ws = torch.empty(lsa.query_encoder_workspace_size(wl.B, h.shape[1], wd.shape[0], wl.Hn, wl.dn),
+                     dtype=torch.uint8, device=device)
+    q = torch.empty(wl.B, wl.Hn, wl.dn, dtype=torch.bfloat16, device=device)
+    w = torch.empty(wl.B, wl.Hn, dtype=torch.bfloat16, device=device)
+    for _ in range(3):
+        lsa.query_encoder(h, wd, wu, wh, wl.Hn, wl.dn, q_out=q, w_out=w, ws=ws)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)     # larger than L2
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(10)]
+    for a, b in evs:
+        flush.fill_(1)
+        a.record()
+        lsa.query_encoder(h, wd, wu, wh, wl.Hn, wl.dn, q_out=q, w_out=w, ws=ws)
+        b.record()
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
+    nbytes = (wd.numel() + wu.numel() + wh.numel()) * 2
+    return {"us_per_call": ms * 1e3, "weight_bytes": nbytes, "achieved_gbs": nbytes / ms / 1e6,
+            "frac": nbytes / ms / 1e6 / hbm_peak, "tokens": wl.B, "d_model": h.shape[1], "rank": wd.shape[0],
+            "l2": "flushed before every call"}
 
 
 def run_e2e(win, wl, args, world):
@@ -422,86 +568,115 @@ def run_e2e(win, wl, args, world):
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
 
-def run_cold(args, device):
-    """512K batch-1 cold pool: select, D2H of the kept list, H2D fetch of kept cold chunks, 64 steps."""
-    wl, host, win = make_window(COLD_WORKLOAD, device)
+def run_cold(args, device, hbm_peak, n_windows=4):
+    """512K batch-1 cold pool over consecutive windows: window 0 gates, plans and fetches its
+    kept cold chunks while its first step attends the window; windows 1.. are prefetched by
+    the lookahead pipeline during the window before."""
+    import lsa_workloads as W
+    from lsa_workloads.device import host_build, upload
+    from learned_sparse_kv_b200.decode import Shapes, Window
+    wl = W.workload(COLD_WORKLOAD)
+    host = host_build(wl, windows=n_windows)
+    shapes, t, max_ch, kept_cap, cold = upload(host, device)
+    win = Window(Shapes(**shapes), t, max_ch, kept_cap, cold)
     win.capture()
-    for _ in range(max(1, args.warmup)):
-        win.run()
+    win.run()
     torch.cuda.synchronize()
-    n = max(2, min(args.steps, 5))
-    t0 = time.perf_counter()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(n):
-        win.run()
-    e1.record()
+    reps = 3
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    marks = [[ev() for _ in range(n_windows + 1)] for _ in range(reps)]
+    fmarks = [[[ev() for _ in range(3)] for _ in range(n_windows)] for _ in range(reps)]
+    for r in range(reps):
+        win.fetch_marks = fmarks[r]
+        win.run_cold(marks=marks[r])
     torch.cuda.synchronize()
-    wall = (time.perf_counter() - t0) * 1e3 / n
-    ms = e0.elapsed_time(e1) / n
-    # the 64 steps alone (graph replay after a fetch)
-    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    g0.record()
-    for _ in range(n):
-        win.graph.replay()
-    g1.record()
-    torch.cuda.synchronize()
-    steps_ms = g0.elapsed_time(g1) / n
-    fetched_bytes = win.n_fetched * 64 * (wl.dqk * 2 + wl.dl * 2)
-    out = {"workload": wl.name, "value": wl.B * wl.steps / (ms / 1e3), "unit": "tokens/s",
-           "ms_per_window": ms, "wall_ms_per_window": wall, "steps_only_ms": steps_ms,
-           "steady_step_us": steps_ms / wl.steps * 1e3, "fetched_chunks": win.n_fetched,
-           "h2d_bytes_per_window": fetched_bytes, "h2d_gbs": fetched_bytes / ((ms - steps_ms) / 1e3) / 1e9
-           if ms > steps_ms else None}
+    win.fetch_marks = None
+    per_w = [[marks[r][w].elapsed_time(marks[r][w + 1]) for w in range(n_windows)] for r in range(reps)]
+    fetch = [[fmarks[r][w][1].elapsed_time(fmarks[r][w][2]) for w in range(n_windows)] for r in range(reps)]
+    log = win.fetch_log.cpu().tolist()
+    chunk_bytes = 64 * (wl.dqk + wl.dl) * 2
+    first = statistics.median(x[0] for x in per_w)
+    steady = statistics.median(v for x in per_w for v in x[1:])
+    fetch0 = statistics.median(x[0] for x in fetch)
+    fetch_n = statistics.median(v for x in fetch for v in x[1:])
+    kc = win.kept_count_w.cpu().numpy()
+    kept = win.kept_w.cpu().numpy()
+    ws0 = int(host["window_start"][0])
+    wb = statistics.mean(window_bytes(win, w, kept=kept[w], kc=kc[w], ws=np.array([ws0 + 64 * w]))
+                         for w in range(1, n_windows))
+    out = {"workload": wl.name, "windows": n_windows, "tokens_per_s_steady": wl.steps / (steady / 1e3),
+           "tokens_per_s_first_window": wl.steps / (first / 1e3),
+           "tokens_per_s_all": n_windows * wl.steps / ((first + (n_windows - 1) * steady) / 1e3),
+           "ms_first_window": first, "ms_steady_window": steady,
+           "fetched_chunks_per_window": log, "fetch_bytes_first": log[0] * chunk_bytes,
+           "fetch_ms_first": fetch0, "fetch_gbs_first": log[0] * chunk_bytes / fetch0 / 1e6 if fetch0 > 0 else None,
+           "fetch_ms_later": fetch_n, "steady_window_bytes": wb, "steady_gbs": wb / (steady / 1e3) / 1e9,
+           "step_frac_steady": wb / (steady / 1e3) / 1e9 / hbm_peak, "device_status": win.device_status(),
+           "gpu_launches_per_run": win.launches_cold(n_windows),
+           "timing": "CUDA events on the compute stream at window boundaries (fetch: events on the side "
+                     "stream around the fetch kernel); median of %d runs of %d windows" % (reps, n_windows)}
     del win
     torch.cuda.empty_cache()
     return out
 
 
-def cpu_baseline(wl, host):
-    """The oracle on this host: sequence 0, decode step 0, plus 1/64 of its chunk selection."""
+def _oracle_samples(wl, n_samples):
+    """Oracle time per decode token on (sequence, step) samples of the workload, plus the
+    sequences' share of the chunk selection.  The samples are decode steps of a one-sequence
+    workload of the same shapes (the selection is timed on the whole batch)."""
+    import lsa_workloads as W
     import oracle
+    from lsa_workloads.device import host_build
     from tests import helpers as H
+    one = wl.shrink(B=1, ctx=wl.ctx[:1], pass_rate=wl.pass_rate[:1])
+    host = host_build(one, steps=min(wl.steps, n_samples))
+    nm = W.nmi_inputs(wl)
     t0 = time.perf_counter()
-    kept, _, _, _ = H.kept_lists(host)
+    oracle.nmi_select(nm["q"], nm["w"], nm["khat"], nm["seq_chunk_offset"])
     t_sel = time.perf_counter() - t0
-    t1 = time.perf_counter()
-    H.oracle_step(host, kept[0], 0, 0)
-    t_step = time.perf_counter() - t1
-    per_token = t_step + t_sel / wl.B / wl.steps
+    kept, _, _, _ = H.kept_lists(host)
+    times = []
+    for s in range(n_samples):
+        t1 = time.perf_counter()
+        H.oracle_step(host, kept[0], 0, s % host["steps"])
+        times.append(time.perf_counter() - t1)
+    return times, t_sel
+
+
+def cpu_baseline(wl, n_samples=8):
+    """The oracle on this host: n_samples (sequence 0, step s) decode steps, plus the per-token
+    share of the chunk selection over all sequences."""
+    times, t_sel = _oracle_samples(wl, n_samples)
+    per_token = statistics.mean(times) + t_sel / wl.B / wl.steps
     return {"value": 1.0 / per_token, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{wl.name}: sequence 0 decode step 0 (indexer scores, top-k, attention) "
-                      f"+ 1/64 of its chunk selection; single-threaded fp64 C",
-            "select_s_all_sequences": t_sel, "step_s": t_step}
+            "sample": f"{wl.name}: {n_samples} decode steps of one sequence of the workload's shapes "
+                      f"(indexer scores, top-k, attention, each timed) + the per-token share of the chunk "
+                      f"selection of all {wl.B} sequences; single-threaded fp64 C",
+            "step_s_each": times, "select_s_all_sequences": t_sel}
 
 
 def run_reference(args, world, rank):
-    """The oracle arm: each step is one (sequence, decode step) sample of the workload."""
+    """The oracle arm: each step is one timed (sequence 0, decode step) sample of the workload."""
     import lsa_workloads as W
-    from lsa_workloads.device import host_build
-    from tests import helpers as H
     if rank != 0:
         return None
     wl = W.workload(args.workload)
-    host = host_build(wl, steps=max(1, min(wl.steps, args.steps + args.warmup)))
-    t0 = time.perf_counter()
-    kept, _, _, _ = H.kept_lists(host)
-    t_sel = time.perf_counter() - t0
-    for s in range(args.warmup):
-        H.oracle_step(host, kept[s % wl.B], s % wl.B, s % host["steps"])
-    t1 = time.perf_counter()
-    for s in range(args.steps):
-        H.oracle_step(host, kept[s % wl.B], s % wl.B, (args.warmup + s) % host["steps"])
-    t_steps = time.perf_counter() - t1
-    per_token = t_steps / args.steps + t_sel / wl.B / wl.steps
-    value = 1.0 / per_token
-    sample = (f"{wl.name}: {args.steps} single (sequence, decode step) samples + 1/64 of chunk selection; "
-              f"single-threaded fp64 C oracle")
+    times, t_sel = _oracle_samples(wl, args.warmup + args.steps)
+    timed = times[args.warmup:]
+    per_step_s = statistics.mean(timed) + t_sel / wl.B / wl.steps
+    value = 1.0 / per_step_s
+    sample = (f"{wl.name}: each step is one decode step of one sequence of the workload's shapes (indexer "
+              f"scores, top-k, attention) "
+              f"plus the per-token share of the chunk selection of all {wl.B} sequences; single-threaded "
+              f"fp64 C oracle; {args.steps} steps timed after {args.warmup} warm-up steps")
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_token * 1e3 * wl.B * wl.steps,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step_s * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded; see lsa_workloads)",
-            "config": {"workload": wl.name, "batch": wl.B, "context": wl.ctx[0], "top_k": wl.k},
+            "config": {"workload": wl.name, "batch": wl.B, "context": wl.ctx[0], "top_k": wl.k, "query_heads": wl.Hq,
+                       "kv_width": wl.dqk, "window": wl.window, "decode_steps_per_step": wl.steps,
+                       "parallelism": f"replicas x{world}"},
+            "window_ms_extrapolated": per_step_s * 1e3 * wl.B * wl.steps,
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 

@@ -106,6 +106,7 @@ class Window:
         self.v_pool = None if shapes.latent else t["v"]
         self.graph = None
         self.graphs: List[torch.cuda.CUDAGraph] = []
+        self.fetch_marks = None        # per window (plan start, fetch start, fetch end) events, when timing
         if cold:
             assert B == 1, "cold pools are laid out for one sequence"
             n_tab = t["chunk_table"].shape[1]
@@ -181,13 +182,19 @@ class Window:
         """Side stream: next table and copy list for window w, then the copies."""
         c = self.cold
         fw = self.fw0 + w
+        if self.fetch_marks is not None:
+            self.fetch_marks[w][0].record(self.fetch_stream)
         lsa.plan_residency(self.t["chunk_table"][0], self.table_next[0], kept_idx[0], kept_count,
                            fw, self.n_ch0 + w + 1, self.n_slots, self.copy_chunk, self.copy_slot, self.copy_count,
                            status=self.status, ws=self.ws_plan, stream=self.fetch_stream)
         with torch.cuda.stream(self.fetch_stream):
             self.fetch_log[w:w + 1].copy_(self.copy_count)
+        if self.fetch_marks is not None:
+            self.fetch_marks[w][1].record(self.fetch_stream)
         lsa.fetch_chunks(c["host_pools"], c["dev_pools"], self.copy_chunk, self.copy_slot, self.copy_count,
                          status=self.status, stream=self.fetch_stream)
+        if self.fetch_marks is not None:
+            self.fetch_marks[w][2].record(self.fetch_stream)
         self.fetch_done.record(self.fetch_stream)
 
     def _install_next_table(self):
@@ -234,10 +241,15 @@ class Window:
             self.kept_w[w].copy_(self.kept_idx)
             self.kept_count_w[w].copy_(self.kept_count)
 
-    def run_cold(self, n_windows: Optional[int] = None, use_graph: bool = True):
-        """The cold pipeline over n_windows consecutive windows (default: all prepared)."""
+    def run_cold(self, n_windows: Optional[int] = None, use_graph: bool = True, marks=None):
+        """The cold pipeline over n_windows consecutive windows (default: all prepared).
+
+        marks (optional): n_windows + 1 CUDA events recorded on the compute stream at the start
+        and after each window's steps."""
         nw = self.n_windows if n_windows is None else n_windows
         compute = torch.cuda.current_stream()
+        if marks is not None:
+            marks[0].record(compute)
         self._reset_cold()
         self.select()
         self.fetch_stream.wait_stream(compute)
@@ -258,6 +270,8 @@ class Window:
                 self.graphs[w].replay()
             else:
                 self.steps(w, first=1 if w == 0 else 0)
+            if marks is not None:
+                marks[w + 1].record(compute)
 
     # -- whole windows ----------------------------------------------------------
     def capture(self):

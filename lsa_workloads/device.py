@@ -17,8 +17,8 @@ chunks and the oracle view is the whole host pool.
 import numpy as np
 import torch
 
-from .generate import (CHUNK, Workload, cold_layout, host_pool, kv_pools, next_window_plant, nmi_inputs, resident_layout,
-                       step_inputs)
+from .generate import (CHUNK, Workload, cold_layout, host_pool, kv_pools, next_window_plant, nmi_inputs,
+                       resident_layout, step_inputs)
 
 
 def bf16(bits: np.ndarray, device=None) -> torch.Tensor:
@@ -151,3 +151,32 @@ def upload(host, device):
                   latent=wl.latent, window=wl.window, steps=host["steps"] // host.get("windows", 1),
                   scale=wl.scale)
     return shapes, t, host["max_chunks"], host["kept_cap"], cold
+
+
+def upload_fast(wl: Workload, device, seed_offset: int = 0, slots_per_draw: int = 2048):
+    """The layout of upload(host_build(wl)) for a resident workload, with the KV and indexer-key
+    pools drawn on the device by torch's seeded generator (N(0, 1) rounded to bf16, like the
+    numpy draws but not the same values).  For throughput runs: the parity tests use host_build,
+    whose pools the oracle can read.  Returns the same tuple as upload()."""
+    assert not wl.cold
+    nm = nmi_inputs(wl)
+    st = stacked_steps(wl, wl.steps)
+    lay = resident_layout(wl)
+    g = torch.Generator(device=device)
+    g.manual_seed(int(wl.seed + seed_offset))
+    t = {"q_nmi": bf16(nm["q"], device), "w_nmi": bf16(nm["w"], device), "khat": bf16(nm["khat"], device),
+         "seq_chunk_offset": torch.from_numpy(nm["seq_chunk_offset"]).to(device)}
+    for key, v in st.items():
+        t[key] = bf16(v, device)
+    widths = {"kv": wl.dqk, "k": wl.dqk, "v": wl.dv, "li": wl.dl}
+    for kind in _kinds(wl):
+        pool = torch.empty(lay["n_slots"], CHUNK, widths[kind], dtype=torch.bfloat16, device=device)
+        for s0 in range(0, lay["n_slots"], slots_per_draw):
+            n = min(slots_per_draw, lay["n_slots"] - s0)
+            pool[s0:s0 + n] = torch.randn(n, CHUNK, widths[kind], generator=g, device=device).to(torch.bfloat16)
+        t[kind] = pool
+    t["chunk_table"] = i32(lay["chunk_table"], device)
+    t["window_start"] = i32(lay["window_start"], device)
+    shapes = dict(B=wl.B, Hn=wl.Hn, dn=wl.dn, Hl=wl.Hl, dl=wl.dl, k=wl.k, Hq=wl.Hq, dqk=wl.dqk, dv=wl.dv,
+                  latent=wl.latent, window=wl.window, steps=wl.steps, scale=wl.scale)
+    return shapes, t, max(wl.n_ch), max(wl.n_ch), None
