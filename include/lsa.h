@@ -71,6 +71,20 @@ const char *lsa_last_error(void);
 const char *lsa_version(void);
 
 /*
+ * Failure-path test switch (no counterpart in the paper).  The next launch of
+ * the named tcgen05 kernel -- LSA_TEST_STALL_ATTENTION: the 128-head latent
+ * attention of lsa_sparse_decode; LSA_TEST_STALL_INDEXER: the indexer scoring
+ * of lsa_topk -- makes its first bounded wait wait on a barrier that nothing
+ * arrives on, for 2 ms.  That wait runs out: the kernel sets LSA_DEV_TIMEOUT in
+ * dev_status, its other waits return, the copies and tensor-core work it
+ * already issued complete, and it returns; the stream and context stay
+ * usable.  Only for tests of that path; the switch clears itself at that launch.
+ */
+#define LSA_TEST_STALL_ATTENTION 1
+#define LSA_TEST_STALL_INDEXER 2
+int lsa_test_stall_next_wait(int which);
+
+/*
  * a1 -- Neural Memory Indexer chunk gate.
  * Passage: gist.science explainer 2.1 ("Scoring-Mechanismus", "Dynamisches
  * Fetching"); cjcn.com.cn article section 2 (ReLU replaced by Sigmoid, fixed

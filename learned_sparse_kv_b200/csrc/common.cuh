@@ -18,6 +18,9 @@ void set_error(const char *fmt, ...);
 int fail(int code, const char *fmt, ...);
 int check_launch(const char *what);  // returns LSA_ERR_CUDA and records the message on error
 int sm_count();                      // multiprocessor count of the current device (cached per device)
+// Failure-path test switch (lsa_test_stall_next_wait): true once for the next
+// launch of the named kernel after the switch was set.
+int take_test_stall(int which);
 
 #define LSA_REQUIRE(cond, code, ...)                   \
     do {                                               \

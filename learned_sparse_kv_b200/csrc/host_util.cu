@@ -2,6 +2,8 @@
 #include <stdarg.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "common.cuh"
 
 namespace lsa {
@@ -41,8 +43,19 @@ int sm_count() {
     return cached[dev];
 }
 
+static std::atomic<int> g_test_stall{0};
+
+int take_test_stall(int which) { return (g_test_stall.fetch_and(~which) & which) ? 1 : 0; }
+
 }  // namespace lsa
 
 extern "C" const char *lsa_last_error(void) { return lsa::g_last_error; }
+
+extern "C" int lsa_test_stall_next_wait(int which) {
+    if (which != LSA_TEST_STALL_ATTENTION && which != LSA_TEST_STALL_INDEXER)
+        return lsa::fail(LSA_ERR_INVALID_ARG, "lsa_test_stall_next_wait: unknown kernel %d", which);
+    lsa::g_test_stall.fetch_or(which);
+    return LSA_OK;
+}
 
 extern "C" const char *lsa_version(void) { return "lsa-b200 0.1 (sm_100a)"; }

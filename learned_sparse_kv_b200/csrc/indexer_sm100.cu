@@ -40,6 +40,11 @@ struct __align__(1024) Smem {
     float w[MAX_H];                                 // head weights of the epilogue's current sequence
     uint32_t tmem_base;
     int abort_flag;
+    // drain bookkeeping: last tile / query load issued into each slot (-1: none), and how
+    // many of them the MMA issuer saw land
+    int k_last[STAGES], q_last[2];
+    int k_consumed, q_consumed;
+    uint64_t never;                                 // no arrival ever: the failure-path test's wait
 };
 
 struct Params {
@@ -53,6 +58,7 @@ struct Params {
     int32_t *status;
     int64_t n_slots;
     int B, H, D, table_stride, kept_cap;
+    int stall;                    // failure-path test: the first wait waits on a barrier nothing arrives on
 };
 
 // 1-CTA MMA and commit
@@ -125,11 +131,12 @@ __device__ __forceinline__ int tile_seq(const Work &wk, int B, int t) {
     return b;
 }
 
-__device__ __forceinline__ bool bounded(Smem &sm, const uint64_t *bar, uint32_t parity, int32_t *status) {
+__device__ __forceinline__ bool bounded(Smem &sm, const uint64_t *bar, uint32_t parity, int32_t *status,
+                                        uint64_t limit = WAIT_NS) {
     if (sm.abort_flag) return false;
-    if (mbar_wait(bar, parity, WAIT_NS)) return true;
+    if (mbar_wait(bar, parity, limit, &sm.abort_flag)) return true;
+    if (!sm.abort_flag) flag(status, LSA_DEV_TIMEOUT);
     sm.abort_flag = 1;
-    flag(status, LSA_DEV_TIMEOUT);
     return false;
 }
 
@@ -149,6 +156,10 @@ li_score_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_consta
             mbar_init(&sm.acc_full[i], 1); mbar_init(&sm.acc_empty[i], 1);
         }
         mbar_init(&sm.mma_done, 1);
+        mbar_init(&sm.never, 1);
+        for (int i = 0; i < STAGES; ++i) sm.k_last[i] = -1;
+        sm.q_last[0] = sm.q_last[1] = -1;
+        sm.k_consumed = sm.q_consumed = 0;
         sm.abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
@@ -203,6 +214,7 @@ li_score_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_consta
                 if (lane == 0) {
                     expect_tx(&sm.q_full[qbuf], (uint32_t)(atoms * p.H * 128));
                     for (int a = 0; a < atoms; ++a) tma_load_2d_local(sm.q[qbuf][a], &q_map, 64 * a, b * p.H, &sm.q_full[qbuf]);
+                    sm.q_last[qbuf] = qswitch - 1;
                 }
                 __syncwarp();
             }
@@ -217,6 +229,7 @@ li_score_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_consta
                         tma_load_2d_local(sm.keys[kslot][a] + i * 64 * 128, &key_map, 64 * a, slot * LSA_CHUNK,
                                           &sm.k_full[kslot]);
                 }
+                sm.k_last[kslot] = t - t0;
             }
             __syncwarp();
             if (++kslot == STAGES) { kslot = 0; kpar ^= 1u; }
@@ -228,6 +241,7 @@ li_score_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_consta
         uint32_t kpar = 0;
         int cur_b = -1, qbuf = 1, qswitch = 0;
         bool ok = true;
+        if (p.stall) ok = bounded(sm, &sm.never, 0, p.status, TEST_STALL_NS);
         for (int t = t0, u = 0; t < t1 && ok; ++t, ++u) {
             const int b = tile_seq(wk, p.B, t);
             if (b != cur_b) {
@@ -237,10 +251,12 @@ li_score_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_consta
                 ok = bounded(sm, &sm.q_full[qbuf], (qswitch >> 1) & 1, p.status);
                 ++qswitch;
                 if (!ok) break;
+                if (lane == 0) sm.q_consumed = qswitch;
             }
             const int ab = u & 1;
             if (u >= 2 && !(ok = bounded(sm, &sm.acc_empty[ab], ((u - 2) >> 1) & 1, p.status))) break;
             if (!(ok = bounded(sm, &sm.k_full[kslot], kpar, p.status))) break;
+            if (lane == 0) sm.k_consumed = u + 1;
             tc_fence_after();
             if (lane == 0) {
                 const uint32_t d = tmem + 64 * ab * (p.H > 64 ? 2 : 1);
@@ -309,6 +325,19 @@ li_score_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_consta
         }
     }
     __syncthreads();
+    if (sm.abort_flag) {
+        // After an abort every TMA load issued lands before the CTA leaves: per key slot
+        // and query buffer the last load whose full phase the MMA issuer did not see.
+        if (threadIdx.x == 0) {
+            for (int i = 0; i < STAGES; ++i)
+                if (sm.k_last[i] >= sm.k_consumed)
+                    (void)mbar_wait(&sm.k_full[i], (uint32_t)(sm.k_last[i] / STAGES) & 1u, WAIT_NS);
+            for (int j = 0; j < 2; ++j)
+                if (sm.q_last[j] >= sm.q_consumed)
+                    (void)mbar_wait(&sm.q_full[j], (uint32_t)(sm.q_last[j] >> 1) & 1u, WAIT_NS);
+        }
+        __syncthreads();
+    }
     if (warp == 1) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(256));
@@ -356,6 +385,7 @@ int launch(const uint16_t *q_li, const uint16_t *w_li, const uint16_t *li_pool, 
     prm.w_li = w_li; prm.table = table; prm.kept_idx = kept_idx; prm.kept_count = kept_count;
     prm.window_start = window_start; prm.cold = cold; prm.scores = scores; prm.status = status; prm.n_slots = n_slots;
     prm.B = B; prm.H = H; prm.D = D; prm.table_stride = table_stride; prm.kept_cap = kept_cap;
+    prm.stall = take_test_stall(LSA_TEST_STALL_INDEXER);
     const size_t smem = sizeof(Smem) + 1024;
     LSA_CUDA(cudaFuncSetAttribute(li_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     li_score_kernel<<<sm_count(), THREADS, smem, stream>>>(key_map, q_map, prm);

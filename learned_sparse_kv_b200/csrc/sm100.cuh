@@ -90,26 +90,33 @@ constexpr uint64_t WAIT_NS = 1000000000ull;
 
 // Waits for the phase with the given parity to complete; returns false once
 // `limit_ns` nanoseconds have passed without it (each try_wait may itself
-// suspend the thread for a while, so the bound is taken on the clock).
-__device__ __forceinline__ bool mbar_wait(const uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+// suspend the thread for a while, so the bound is taken on the clock), or as
+// soon as *abort (a flag in shared memory, if given) is set by another warp.
+__device__ __forceinline__ bool mbar_wait(const uint64_t *bar, uint32_t parity, uint64_t limit_ns,
+                                          const volatile int *abort = nullptr) {
     const uint32_t a = smem_addr(bar);
     if (mbar_try_wait(a, parity)) return true;
     const uint64_t t0 = global_ns();
     for (;;) {
         if (mbar_try_wait(a, parity)) return true;
-        if (global_ns() - t0 > limit_ns) return false;
+        if (global_ns() - t0 > limit_ns || (abort && *abort)) return false;
     }
 }
 
-__device__ __forceinline__ bool mbar_wait_cluster(const uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+__device__ __forceinline__ bool mbar_wait_cluster(const uint64_t *bar, uint32_t parity, uint64_t limit_ns,
+                                                  const volatile int *abort = nullptr) {
     const uint32_t a = smem_addr(bar);
     if (mbar_try_wait_cluster(a, parity)) return true;
     const uint64_t t0 = global_ns();
     for (;;) {
         if (mbar_try_wait_cluster(a, parity)) return true;
-        if (global_ns() - t0 > limit_ns) return false;
+        if (global_ns() - t0 > limit_ns || (abort && *abort)) return false;
     }
 }
+
+// Wait limit of a failure-path test: the first wait of a kernel launched with
+// its stall switch on waits for a phase that never completes, for this long.
+constexpr uint64_t TEST_STALL_NS = 2000000ull;
 
 // ------------------------------------------------------------- cluster ----
 

@@ -34,7 +34,9 @@
 // The online softmax is evaluated in the log2 domain; the reference maximum
 // is only moved when a row maximum grows by more than 2^8, which keeps P <= 256
 // in bf16 and makes O rescales rare.  Every mbarrier wait is bounded: on
-// timeout the kernel sets LSA_DEV_TIMEOUT, drains and exits.
+// timeout the kernel sets LSA_DEV_TIMEOUT and the abort flag of both CTAs, the
+// other waits return, the tensor-core work issued so far completes, the even CTA
+// waits for every TMA load still in flight, and the pair exits.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -81,6 +83,11 @@ struct __align__(1024) Smem {
     float red[128];
     uint32_t tmem_base;
     int abort_flag;
+    // drain bookkeeping: the tile of the last TMA load this CTA issued into each stage
+    // (-1: none), and (even CTA) the tiles whose K / V full phase an issuer saw complete
+    int last_k_tma[STAGES], last_v_tma[STAGES];
+    int k_consumed, v_consumed, q_seen;
+    uint64_t never;                  // no arrival ever: the failure-path test's wait
 };
 static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory of one CTA");
 
@@ -97,6 +104,7 @@ struct Params {
     int64_t n_rows_pool;   // n_slots * 64
     int table_stride, k, n_splits;
     float scale_log2;
+    int stall;             // failure-path test: the first wait waits on a barrier nothing arrives on
 };
 
 // Tiles of one sequence: ceil(tk/64) top-k tiles, then the window chunk by chunk.
@@ -148,17 +156,28 @@ struct SeqTiles {
     }
 };
 
+// Sets the abort flag of both CTAs of the pair (the peer's through distributed
+// shared memory), so that every bounded wait of the pair returns at once.
 __device__ __forceinline__ void set_abort(Smem &sm, int32_t *status) {
     sm.abort_flag = 1;
+    asm volatile("st.shared::cluster.s32 [%0], %1;\n" ::"r"(map_to_rank(&sm.abort_flag, cluster_rank() ^ 1u)), "r"(1)
+                 : "memory");
     flag(status, LSA_DEV_TIMEOUT);
 }
 
+__device__ __forceinline__ int ld_peer_s32(const void *p) {
+    int v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];\n" : "=r"(v) : "r"(map_to_rank(p, cluster_rank() ^ 1u)) : "memory");
+    return v;
+}
+
 // Warp-uniform bounded wait (lane 0 polls, result broadcast).
-__device__ __forceinline__ bool warp_wait(Smem &sm, const uint64_t *bar, uint32_t parity, int32_t *status) {
+__device__ __forceinline__ bool warp_wait(Smem &sm, const uint64_t *bar, uint32_t parity, int32_t *status,
+                                          uint64_t limit = WAIT_NS) {
     bool ok = true;
     if ((threadIdx.x & 31) == 0) {
-        ok = sm.abort_flag == 0 && mbar_wait(bar, parity, WAIT_NS);
-        if (!ok) set_abort(sm, status);
+        ok = sm.abort_flag == 0 && mbar_wait(bar, parity, limit, &sm.abort_flag);
+        if (!ok && sm.abort_flag == 0) set_abort(sm, status);
     }
     return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
@@ -167,8 +186,8 @@ __device__ __forceinline__ bool warp_wait(Smem &sm, const uint64_t *bar, uint32_
 __device__ __forceinline__ bool warp_wait_cluster(Smem &sm, const uint64_t *bar, uint32_t parity, int32_t *status) {
     bool ok = true;
     if ((threadIdx.x & 31) == 0) {
-        ok = sm.abort_flag == 0 && mbar_wait_cluster(bar, parity, WAIT_NS);
-        if (!ok) set_abort(sm, status);
+        ok = sm.abort_flag == 0 && mbar_wait_cluster(bar, parity, WAIT_NS, &sm.abort_flag);
+        if (!ok && sm.abort_flag == 0) set_abort(sm, status);
     }
     return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
@@ -177,10 +196,20 @@ __device__ __forceinline__ bool warp_wait_cluster(Smem &sm, const uint64_t *bar,
 __device__ __forceinline__ bool group_wait(Smem &sm, const uint64_t *bar, uint32_t parity, int32_t *status, int g) {
     bool ok = true;
     if (g == 0) {
-        ok = sm.abort_flag == 0 && mbar_wait(bar, parity, WAIT_NS);
-        if (!ok) set_abort(sm, status);
+        ok = sm.abort_flag == 0 && mbar_wait(bar, parity, WAIT_NS, &sm.abort_flag);
+        if (!ok && sm.abort_flag == 0) set_abort(sm, status);
     }
     return named_barrier_and(2, GATHER_THREADS, ok);
+}
+
+// Waits until the TMA load of the last tile issued into a stage has landed, if no issuer
+// saw its full phase complete.  u0 / u1: that tile as issued by the even / odd CTA.
+__device__ __forceinline__ void drain_stage(uint64_t *full, int u0, int u1, int consumed) {
+    const int u = max(u0, u1);
+    if (u < consumed) return;            // completed and consumed, or nothing issued (u = -1)
+    if (u0 != u) mbar_arrive_local(full);   // the even CTA did not issue tile u
+    if (u1 != u) mbar_arrive_local(full);   // the odd CTA did not issue tile u
+    (void)mbar_wait(full, (uint32_t)(u >> 1) & 1u, WAIT_NS);
 }
 
 __device__ __forceinline__ int32_t gather_row(const SeqTiles &st, const Params &p, int b, int t, int i) {
@@ -209,6 +238,9 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         mbar_init(&sm.pv_done[1], 1);
         mbar_init(&sm.mma_done, 2);   // one commit from each MMA issuer
         for (int i = 0; i < INFO; ++i) { mbar_init(&sm.info_full[i], 1); mbar_init(&sm.info_empty[i], 1); }
+        mbar_init(&sm.never, 1);
+        for (int i = 0; i < STAGES; ++i) sm.last_k_tma[i] = sm.last_v_tma[i] = -1;
+        sm.k_consumed = sm.v_consumed = sm.q_seen = 0;
         sm.abort_flag = 0;
         fence_mbar_init_cluster();
     }
@@ -288,6 +320,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                         const uint32_t full = map_to_rank(&sm.k_full[s], 0);
                         mbar_arrive_expect_tx_cluster(full, K_BYTES);
                         tma_load_3d(sm.k[s][0], &k_map, 0, wy + 32 * (int)rank, 0, full);
+                        sm.last_k_tma[s] = u;
                     }
                 }
             } else {
@@ -299,6 +332,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                         const uint32_t full = map_to_rank(&sm.v_full[s], 0);
                         mbar_arrive_expect_tx_cluster(full, V_BYTES);
                         tma_load_4d(sm.v[s][0][0], &v_map, 0, wy, 2 * (int)rank, 0, full);
+                        sm.last_v_tma[s] = u;
                     }
                 }
             }
@@ -319,12 +353,15 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             constexpr uint64_t Q_CHUNK = (HPC * 128) >> 4, K_CHUNK = (32 * 128) >> 4, K_STAGE = K_BYTES >> 4;
             const uint64_t qd0 = smem_desc_sw128(smem_addr(sm.q[0]), 16, 1024);
             const uint64_t kd0 = smem_desc_sw128(smem_addr(sm.k[0][0]), 16, 1024);
-            ok = warp_wait(sm, &sm.q_full, 0, p.status);
+            if (p.stall) ok = warp_wait(sm, &sm.never, 0, p.status, TEST_STALL_NS);
+            ok = ok && warp_wait(sm, &sm.q_full, 0, p.status);
+            if (ok && lane == 0) sm.q_seen = 1;
             for (int u = 0; u < n_tiles && ok; ++u) {      // S(u) = Q K^T
                 const int sb = u & 1;
                 ok = warp_wait(sm, &sm.s_empty[sb], ((u >> 1) + 1) & 1, p.status) &&
                      warp_wait_cluster(sm, &sm.k_full[sb], (u >> 1) & 1, p.status);
                 if (!ok) break;
+                if (lane == 0) sm.k_consumed = u + 1;
                 tc_fence_after();
                 if (lane == 0) {
                     const uint32_t d = tmem + TM_S + 32 * sb;
@@ -350,6 +387,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 ok = warp_wait(sm, &sm.p_full[sb], (u >> 1) & 1, p.status) &&
                      warp_wait_cluster(sm, &sm.v_full[sb], (u >> 1) & 1, p.status);
                 if (!ok) break;
+                if (lane == 0) sm.v_consumed = u + 1;
                 tc_fence_after();
                 if (lane == 0) {
                     const uint64_t vb = vd0 + V_STAGE * sb;
@@ -456,9 +494,9 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         for (int u = 0; u < n_tiles; ++u) {
             const int s = u & 1;
             ok = ok && sm.abort_flag == 0;
-            if (ok) ok = mbar_wait(&sm.info_full[u % INFO], (u / INFO) & 1, WAIT_NS);
+            if (ok) ok = mbar_wait(&sm.info_full[u % INFO], (u / INFO) & 1, WAIT_NS, &sm.abort_flag);
             const uint32_t vmask = ok ? (uint32_t)(sm.info_mask[u % INFO] >> (32 * half)) : 0u;
-            if (ok) ok = mbar_wait(&sm.s_full[s], (u >> 1) & 1, WAIT_NS);
+            if (ok) ok = mbar_wait(&sm.s_full[s], (u >> 1) & 1, WAIT_NS, &sm.abort_flag);
             if (!ok && sm.abort_flag == 0) set_abort(sm, p.status);
             tc_fence_after();
             uint32_t raw[32];
@@ -504,7 +542,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             l += psum;
             // The P buffers are rewritten and O may be rescaled: P.V of tile u-1 must be done.
             if (u > 0 && ok) {
-                ok = mbar_wait(&sm.pv_done[(u - 1) & 1], ((u - 1) >> 1) & 1, WAIT_NS);
+                ok = mbar_wait(&sm.pv_done[(u - 1) & 1], ((u - 1) >> 1) & 1, WAIT_NS, &sm.abort_flag);
                 if (!ok && sm.abort_flag == 0) set_abort(sm, p.status);
             }
             // tcgen05.ld / st are warp-collective: the whole warp takes the rescale when
@@ -538,7 +576,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         }
         // ---- epilogue: wait for the last P.V, then write the partial
         if (n_tiles > 0 && ok) {
-            ok = mbar_wait(&sm.pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, WAIT_NS);
+            ok = mbar_wait(&sm.pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, WAIT_NS, &sm.abort_flag);
             if (!ok && sm.abort_flag == 0) set_abort(sm, p.status);
         }
         tc_fence_after();
@@ -580,8 +618,23 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         __syncwarp();
     }
     __syncthreads();
-    if (sm.abort_flag) __nanosleep(20000);   // let in-flight TMA loads land before the CTA exits
-    cluster_sync();
+    cluster_sync();   // neither CTA issues another copy from here on
+    const bool aborted = sm.abort_flag || ld_peer_s32(&sm.abort_flag);   // same answer in both CTAs
+    if (aborted) {
+      if (rank == 0 && threadIdx.x == 0 && n_tiles > 0) {
+        // After an abort, every TMA load either CTA issued lands before either CTA leaves:
+        // Q (issued by both producers before their loops), and per stage the last K and V
+        // tiles whose full phase no issuer saw complete.  Where only one CTA issued that
+        // tile, this thread arrives in place of the other, so the phase completes once the
+        // issued bytes have landed.  Every wait is bounded.
+        if (!sm.q_seen) (void)mbar_wait(&sm.q_full, 0, WAIT_NS);
+        for (int s = 0; s < STAGES; ++s) {
+            drain_stage(&sm.k_full[s], sm.last_k_tma[s], ld_peer_s32(&sm.last_k_tma[s]), sm.k_consumed);
+            drain_stage(&sm.v_full[s], sm.last_v_tma[s], ld_peer_s32(&sm.last_v_tma[s]), sm.v_consumed);
+        }
+      }
+      cluster_sync();   // the odd CTA leaves only after the drain
+    }
     if (warp == 3) {
         tc_fence_after();
         tmem_dealloc_pair(tmem, TM_COLS);
@@ -661,6 +714,7 @@ int launch(const uint16_t *q, const uint16_t *kv_pool, int64_t k_stride, int64_t
     prm.o_part = o_part; prm.m_part = m_part; prm.l_part = l_part; prm.status = status;
     prm.n_rows_pool = n_slots * LSA_CHUNK; prm.table_stride = table_stride; prm.k = k; prm.n_splits = n_splits;
     prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.stall = take_test_stall(LSA_TEST_STALL_ATTENTION);
     const size_t smem = smem_bytes();
     LSA_CUDA(cudaFuncSetAttribute(mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     cudaLaunchConfig_t cfg = {};

@@ -57,6 +57,7 @@ def _load():
         "lsa_label_vote_workspace_size": ([I, I, I], SZ),
         "lsa_last_error": ([], ctypes.c_char_p),
         "lsa_version": ([], ctypes.c_char_p),
+        "lsa_test_stall_next_wait": ([I], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -70,6 +71,15 @@ _lib = _load()
 
 def version() -> str:
     return _lib.lsa_version().decode()
+
+
+TEST_STALL_ATTENTION, TEST_STALL_INDEXER = 1, 2
+
+
+def test_stall_next_wait(which):
+    """Failure-path test switch: the next launch of the named tcgen05 kernel waits on a barrier
+    nothing arrives on, for 2 ms, then reports LSA_DEV_TIMEOUT and returns."""
+    _check(_lib.lsa_test_stall_next_wait(int(which)))
 
 
 def _check(rc):
