@@ -90,8 +90,11 @@ constexpr uint64_t WAIT_NS = 1000000000ull;
 
 // Waits for the phase with the given parity to complete; returns false once
 // `limit_ns` nanoseconds have passed without it (each try_wait may itself
-// suspend the thread for a while, so the bound is taken on the clock), or as
-// soon as *abort (a flag in shared memory, if given) is set by another warp.
+// suspend the thread for a while, so the bound is taken on the clock), or once
+// *abort (a flag in shared memory, if given) is set by another warp.  The flag
+// is only read once the wait has lasted ABORT_POLL_NS, longer than a whole
+// healthy launch: reading it sooner measurably slowed the attention kernel.
+constexpr uint64_t ABORT_POLL_NS = 100000;
 __device__ __forceinline__ bool mbar_wait(const uint64_t *bar, uint32_t parity, uint64_t limit_ns,
                                           const volatile int *abort = nullptr) {
     const uint32_t a = smem_addr(bar);
@@ -99,7 +102,8 @@ __device__ __forceinline__ bool mbar_wait(const uint64_t *bar, uint32_t parity, 
     const uint64_t t0 = global_ns();
     for (;;) {
         if (mbar_try_wait(a, parity)) return true;
-        if (global_ns() - t0 > limit_ns || (abort && *abort)) return false;
+        const uint64_t dt = global_ns() - t0;
+        if (dt > limit_ns || (abort && dt > ABORT_POLL_NS && *abort)) return false;
     }
 }
 
@@ -110,7 +114,8 @@ __device__ __forceinline__ bool mbar_wait_cluster(const uint64_t *bar, uint32_t 
     const uint64_t t0 = global_ns();
     for (;;) {
         if (mbar_try_wait_cluster(a, parity)) return true;
-        if (global_ns() - t0 > limit_ns || (abort && *abort)) return false;
+        const uint64_t dt = global_ns() - t0;
+        if (dt > limit_ns || (abort && dt > ABORT_POLL_NS && *abort)) return false;
     }
 }
 

@@ -158,7 +158,7 @@ struct SeqTiles {
 
 // Sets the abort flag of both CTAs of the pair (the peer's through distributed
 // shared memory), so that every bounded wait of the pair returns at once.
-__device__ __forceinline__ void set_abort(Smem &sm, int32_t *status) {
+__device__ __noinline__ void set_abort(Smem &sm, int32_t *status) {
     sm.abort_flag = 1;
     asm volatile("st.shared::cluster.s32 [%0], %1;\n" ::"r"(map_to_rank(&sm.abort_flag, cluster_rank() ^ 1u)), "r"(1)
                  : "memory");
@@ -619,8 +619,10 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
     }
     __syncthreads();
     cluster_sync();   // neither CTA issues another copy from here on
-    const bool aborted = sm.abort_flag || ld_peer_s32(&sm.abort_flag);   // same answer in both CTAs
-    if (aborted) {
+    // set_abort writes the flag into both CTAs before this barrier, so both read the same
+    // value here from their own shared memory (no read of the peer: it may leave after the
+    // barrier unless both take the abort path, which ends with a second barrier).
+    if (sm.abort_flag) {
       if (rank == 0 && threadIdx.x == 0 && n_tiles > 0) {
         // After an abort, every TMA load either CTA issued lands before either CTA leaves:
         // Q (issued by both producers before their loops), and per stage the last K and V
