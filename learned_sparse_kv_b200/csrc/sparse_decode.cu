@@ -381,9 +381,10 @@ using CfgMla64 = DecodeCfg<64, 576, 512, 8, true>;
 namespace mla2 {
 int launch(const uint16_t *q, const uint16_t *kv_pool, int64_t k_stride, int64_t n_slots, const int32_t *table,
            int table_stride, const int32_t *topk_idx, const int32_t *topk_count, int k, const int32_t *window_start,
-           const int32_t *window_len, int B, float scale, int n_splits, float *o_part, float *m_part, float *l_part,
-           int32_t *status, cudaStream_t stream);
+           const int32_t *window_len, int max_window_len, int B, float scale, int n_splits, float *o_part,
+           float *m_part, float *l_part, uint8_t *stage, int32_t *status, cudaStream_t stream);
 int max_splits(int B);
+size_t stage_bytes(int B, int k, int max_window_len);
 }  // namespace mla2
 
 // Sep16: 16 heads, separate K/V rows of 128 (mma.sync).  Mla64: 64 latent heads
@@ -455,6 +456,7 @@ extern "C" size_t lsa_sparse_decode_workspace_size(int B, int Hq, int dqk, int d
     c.take<float>((size_t)B * ns * Hq * dv);
     c.take<float>((size_t)B * ns * Hq);
     c.take<float>((size_t)B * ns * Hq);
+    if (v == Variant::Mla128) c.take<uint8_t>(mla2::stage_bytes(B, k, max_window_len));   // staged tiles
     return align_up(c.used, 256);
 }
 
@@ -487,9 +489,11 @@ extern "C" int lsa_sparse_decode(const lsa_bf16 *q, const lsa_bf16 *k_pool, int6
     float *o_part = c.take<float>((size_t)B * ns * Hq * dv);
     float *m_part = c.take<float>((size_t)B * ns * Hq);
     float *l_part = c.take<float>((size_t)B * ns * Hq);
+    uint8_t *stage = v == Variant::Mla128 ? c.take<uint8_t>(mla2::stage_bytes(B, k, max_window_len)) : nullptr;
     int rc = v == Variant::Mla128
                  ? mla2::launch(q, k_pool, k_row_stride, n_slots, chunk_table, table_stride, topk_idx, topk_count, k,
-                                window_start, window_len, B, scale, ns, o_part, m_part, l_part, dev_status, stream)
+                                window_start, window_len, max_window_len, B, scale, ns, o_part, m_part, l_part, stage,
+                                dev_status, stream)
              : v == Variant::Sep16
                  ? launch<CfgSep16>(q, k_pool, k_row_stride, v_pool, v_row_stride, n_slots, chunk_table, table_stride,
                                     topk_idx, topk_count, k, window_start, window_len, B, Hq, scale, ns, o_part, m_part,

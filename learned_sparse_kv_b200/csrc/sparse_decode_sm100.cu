@@ -17,20 +17,22 @@
 // TMEM per CTA: two S buffers of 32 columns and O = 64 heads x 512 values in
 // 256 columns.
 //
-// Loading a tile is one operation per operand wherever the rows are a whole
-// chunk slot of the pool: a 3D TMA box {64 columns, 32 rows, 9 column chunks}
-// fetches a CTA's K rows (36 KB) and a 4D box {64, 64 rows, 2, 2} its value
-// columns (32 KB), both straight into the 128-byte-swizzled operand layout.
-// Gathered tiles (top-k rows, and window tiles that are not a whole aligned
-// chunk) are copied by two warpgroups with 16-byte cp.async into the same layout;
-// missing rows are zero-filled.  Two stages of each operand are in flight.
+// Loading a tile is one operation per operand: a 3D TMA box {64 columns, 32
+// rows, 9 column chunks} fetches a CTA's K rows (36 KB) and a 4D box {64, 64
+// rows, 2, 2} its value columns (32 KB), both straight into the 128-byte-swizzled
+// operand layout.  Window tiles that are a whole aligned chunk slot are read
+// from the pool; the other tiles (top-k rows, and window tiles that are not a
+// whole aligned chunk) are first copied, 64 rows at a time, by stage_kernel
+// into a contiguous staging buffer (missing rows zero-filled), so that they are
+// TMA boxes too: that copy runs on every multiprocessor at the memory's rate,
+// where row gathers inside this kernel were bound by the copies one
+// multiprocessor keeps in flight and stalled the two-stage pipeline.  Two
+// stages of each operand are in flight.
 // Warp roles:
 //   0      K producer (TMA), tile-validity masks
 //   1      S = Q K^T issuer (even CTA)        2   O += P V issuer (even CTA)
 //   3      TMEM allocator, V producer (TMA)
 //   4..7   softmax, O rescale, epilogue (one thread per TMEM lane)
-//   8..15  row gather for gathered tiles (256 threads: the copy rate of one
-//          multiprocessor grows with the number of copying warps)
 // The online softmax is evaluated in the log2 domain; the reference maximum
 // is only moved when a row maximum grows by more than 2^8, which keeps P <= 256
 // in bf16 and makes O rescales rare.  Every mbarrier wait is bounded: on
@@ -54,8 +56,7 @@ constexpr int NTILE = 64;         // kv rows per tile
 constexpr int KCH = DQK / 64;     // 9 column chunks of 64
 constexpr int STAGES = 2;         // tiles in flight per operand
 constexpr int INFO = 4;           // tile-validity ring
-constexpr int THREADS = 512;
-constexpr int GATHER_THREADS = 256;
+constexpr int THREADS = 256;
 constexpr uint32_t Q_BYTES = KCH * HPC * 128;          // per CTA
 constexpr uint32_t K_BYTES = KCH * 32 * 128;           // per CTA and tile
 constexpr uint32_t V_BYTES = 2 * 2 * NTILE * 128;      // per CTA and tile
@@ -73,13 +74,11 @@ struct __align__(1024) Smem {
     uint8_t p[2][HPC * 128];                   // P = hi + lo: [part][64 heads][64 kv], K-major
     uint64_t k_full[STAGES], k_empty[STAGES];
     uint64_t v_full[STAGES], v_empty[STAGES];
-    uint64_t k_go[2], v_go[2];       // producer -> gather: stage free for the n-th gathered tile
     uint64_t q_full;
     uint64_t s_full[2], s_empty[2], p_full[2];
     uint64_t pv_done[2], mma_done;   // pv_done[u & 1]: P.V of tile u
     uint64_t info_full[INFO], info_empty[INFO];
     unsigned long long info_mask[INFO];
-    int32_t grow[STAGES][NTILE];     // pool rows of a gathered tile (-1: zero row)
     float red[128];
     uint32_t tmem_base;
     int abort_flag;
@@ -103,6 +102,7 @@ struct Params {
     int32_t *status;
     int64_t n_rows_pool;   // n_slots * 64
     int table_stride, k, n_splits;
+    int stage_tiles;       // staging slots per sequence
     float scale_log2;
     int stall;             // failure-path test: the first wait waits on a barrier nothing arrives on
 };
@@ -133,6 +133,15 @@ struct SeqTiles {
         const int64_t g = (int64_t)slot * LSA_CHUNK;
         if (slot < 0 || g >= p.n_rows_pool) return -2;
         return g;
+    }
+    // Staging slot of gathered tile t: top-k tiles first, then (aligned window) the
+    // last, partial window tile, or (unaligned window) every window tile in order.
+    __device__ int stage_index(int t) const { return t < t_topk ? t : (aligned ? t_topk : t); }
+    // Inverse: the gathered tile staged in slot g, or -1.
+    __device__ int staged_tile(int g) const {
+        if (g < t_topk) return g;
+        if (aligned) return (g == t_topk && total > t_topk && gathered(total - 1)) ? total - 1 : -1;
+        return g < total ? g : -1;
     }
     // Global pool row of row i (0..63) of tile t, -1 past the end of the row set, -2 if unmapped.
     __device__ int64_t row(const Params &p, int b, int t, int i) const {
@@ -192,16 +201,6 @@ __device__ __forceinline__ bool warp_wait_cluster(Smem &sm, const uint64_t *bar,
     return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
-// Gather-group-uniform bounded wait: one thread polls, the group agrees by barrier reduction.
-__device__ __forceinline__ bool group_wait(Smem &sm, const uint64_t *bar, uint32_t parity, int32_t *status, int g) {
-    bool ok = true;
-    if (g == 0) {
-        ok = sm.abort_flag == 0 && mbar_wait(bar, parity, WAIT_NS, &sm.abort_flag);
-        if (!ok && sm.abort_flag == 0) set_abort(sm, status);
-    }
-    return named_barrier_and(2, GATHER_THREADS, ok);
-}
-
 // Waits until the TMA load of the last tile issued into a stage has landed, if no issuer
 // saw its full phase complete.  u0 / u1: that tile as issued by the even / odd CTA.
 __device__ __forceinline__ void drain_stage(uint64_t *full, int u0, int u1, int consumed) {
@@ -212,13 +211,34 @@ __device__ __forceinline__ void drain_stage(uint64_t *full, int u0, int u1, int 
     (void)mbar_wait(full, (uint32_t)(u >> 1) & 1u, WAIT_NS);
 }
 
-__device__ __forceinline__ int32_t gather_row(const SeqTiles &st, const Params &p, int b, int t, int i) {
-    const int64_t g = st.row(p, b, t, i);
-    return g >= 0 ? (int32_t)g : -1;
+// grid (stage_tiles, B), 256 threads: staging slot g of sequence b receives the 64 rows of
+// the gathered tile staged there (rows past the row set, or without a slot, as zeros).
+// Each thread keeps its 18 loads of 16 bytes in flight before storing.
+__global__ void __launch_bounds__(256) stage_kernel(const Params p, uint8_t *__restrict__ stage) {
+    constexpr int PIECES = DQK * 2 / 16;                  // 72 pieces of 16 bytes per row
+    constexpr int PER_THREAD = NTILE * PIECES / 256;      // 18
+    __shared__ int64_t rows[NTILE];
+    const int g = blockIdx.x, b = blockIdx.y;
+    const SeqTiles st(p, b);
+    const int t = st.staged_tile(g);
+    if (t < 0) return;
+    if (threadIdx.x < NTILE) rows[threadIdx.x] = st.row(p, b, t, threadIdx.x);
+    __syncthreads();
+    uint4 v[PER_THREAD];
+#pragma unroll
+    for (int i = 0; i < PER_THREAD; ++i) {
+        const int q = threadIdx.x + 256 * i, r = q / PIECES, w = q - r * PIECES;
+        const int64_t pr = rows[r];
+        v[i] = pr >= 0 ? __ldg(reinterpret_cast<const uint4 *>(p.pool + pr * p.row_bytes) + w) : make_uint4(0, 0, 0, 0);
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(stage + ((size_t)b * p.stage_tiles + g) * NTILE * (DQK * 2));
+#pragma unroll
+    for (int i = 0; i < PER_THREAD; ++i) dst[threadIdx.x + 256 * i] = v[i];
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
 mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap v_map,
+                  const __grid_constant__ CUtensorMap ks_map, const __grid_constant__ CUtensorMap vs_map,
                   const __grid_constant__ CUtensorMap q_map, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>(smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023));
@@ -231,7 +251,6 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             mbar_init(&sm.k_full[i], 2); mbar_init(&sm.k_empty[i], 1);
             mbar_init(&sm.v_full[i], 2); mbar_init(&sm.v_empty[i], 1);
         }
-        for (int i = 0; i < 2; ++i) { mbar_init(&sm.k_go[i], 1); mbar_init(&sm.v_go[i], 1); }
         mbar_init(&sm.q_full, 2);
         for (int i = 0; i < 2; ++i) { mbar_init(&sm.s_full[i], 1); mbar_init(&sm.s_empty[i], 2); mbar_init(&sm.p_full[i], 2); }
         mbar_init(&sm.pv_done[0], 1);
@@ -253,25 +272,12 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
 
     const SeqTiles st(p, b);
     // Tiles are dealt round-robin: split s takes tiles s, s + n_splits, ...  The
-    // gathered top-k tiles (first in the tile list, and dearer to load than the
-    // chunk-aligned window tiles) are thereby spread evenly over the splits.
+    // staged top-k tiles (first in the tile list) are thereby spread evenly over
+    // the splits.  K (warp 0) and V (warp 3) have a producer each, so K of a later
+    // tile never waits behind the P.V that frees a V stage.
     const int n_tiles = split < st.total ? (st.total - 1 - split) / p.n_splits + 1 : 0;
     const int u0 = split, ustride = p.n_splits;
-    // The split's gathered top-k tiles come first in its share; the first window
-    // tile is moved ahead of them, so the tensor pipe starts on a TMA-loaded tile
-    // while the gathered rows are being copied.
-    const int n_gath = min(n_tiles, split < st.t_topk ? (st.t_topk - 1 - split) / ustride + 1 : 0);
-    const bool lead = n_gath > 0 && n_gath < n_tiles;
-    auto tile_of = [&](int u) {
-        const int k = !lead ? u : (u == 0 ? n_gath : (u <= n_gath ? u - 1 : u));
-        return u0 + k * ustride;
-    };
-
-    // Every tile's stage is waited for by its producer in tile order: a parity wait is
-    // only unambiguous one phase behind the barrier, so the gather group (which
-    // skips the TMA tiles) is handed its stages through k_go / v_go, whose phases count
-    // gathered tiles only.  K (warp 0) and V (warp 3) have a producer each, so K of a
-    // later tile never waits behind the P.V that frees a V stage.
+    auto tile_of = [&](int u) { return u0 + u * ustride; };
     if ((warp == 0 || warp == 3) && n_tiles > 0) {
         // ------------------------------------------------ TMA producers (K + masks, V)
         const bool kprod = warp == 0;
@@ -283,13 +289,14 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         // row indices of the next gathered tile are loaded while the current tile is issued
         int64_t n0 = -1, n1 = -1;
         if (kprod && st.gathered(tile_of(0))) { n0 = st.row(p, b, tile_of(0), lane); n1 = st.row(p, b, tile_of(0), lane + 32); }
-        int gi = 0;   // gathered tiles handed to the gather group so far
         for (int u = 0; u < n_tiles; ++u) {
             const int t = tile_of(u);
             const bool gath = st.gathered(t);
             const int64_t slot_row = gath ? -2 : st.window_slot_row(p, b, t);
-            // an unmapped slot is read out of range: TMA fills zeros
-            const int wy = slot_row >= 0 ? (int)slot_row : (int)p.n_rows_pool;
+            // an unmapped slot is read out of range: TMA fills zeros; a staged tile is read
+            // from its staging slot
+            const int wy = gath ? (b * p.stage_tiles + st.stage_index(t)) * NTILE
+                                : (slot_row >= 0 ? (int)slot_row : (int)p.n_rows_pool);
             const int s = u & 1;
             const uint32_t par = ((u >> 1) + 1) & 1;
             if (kprod) {
@@ -314,29 +321,20 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 }
                 if (!warp_wait(sm, &sm.k_empty[s], par, p.status)) break;
                 if (lane == 0) {
-                    if (gath) {
-                        mbar_arrive_local(&sm.k_go[gi & 1]);
-                    } else {
-                        const uint32_t full = map_to_rank(&sm.k_full[s], 0);
-                        mbar_arrive_expect_tx_cluster(full, K_BYTES);
-                        tma_load_3d(sm.k[s][0], &k_map, 0, wy + 32 * (int)rank, 0, full);
-                        sm.last_k_tma[s] = u;
-                    }
+                    const uint32_t full = map_to_rank(&sm.k_full[s], 0);
+                    mbar_arrive_expect_tx_cluster(full, K_BYTES);
+                    tma_load_3d(sm.k[s][0], gath ? &ks_map : &k_map, 0, wy + 32 * (int)rank, 0, full);
+                    sm.last_k_tma[s] = u;
                 }
             } else {
                 if (!warp_wait(sm, &sm.v_empty[s], par, p.status)) break;
                 if (lane == 0) {
-                    if (gath) {
-                        mbar_arrive_local(&sm.v_go[gi & 1]);
-                    } else {
-                        const uint32_t full = map_to_rank(&sm.v_full[s], 0);
-                        mbar_arrive_expect_tx_cluster(full, V_BYTES);
-                        tma_load_4d(sm.v[s][0][0], &v_map, 0, wy, 2 * (int)rank, 0, full);
-                        sm.last_v_tma[s] = u;
-                    }
+                    const uint32_t full = map_to_rank(&sm.v_full[s], 0);
+                    mbar_arrive_expect_tx_cluster(full, V_BYTES);
+                    tma_load_4d(sm.v[s][0][0], gath ? &vs_map : &v_map, 0, wy, 2 * (int)rank, 0, full);
+                    sm.last_v_tma[s] = u;
                 }
             }
-            gi += gath ? 1 : 0;
             __syncwarp();
         }
     } else if ((warp == 1 || warp == 2) && rank == 0 && n_tiles > 0) {
@@ -407,83 +405,6 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         }
         if (lane == 0) umma_commit_pair(&sm.mma_done, 0x3);
         __syncwarp();
-    } else if (warp >= 8 && n_tiles > 0) {
-        // ------------------------------------------------ row gather (cp.async)
-        // Thread g copies 16-byte pieces: K pieces q = g + 256 i of the CTA's 32
-        // rows x 72 pieces, V pieces of 64 rows x 4 value atoms x 8 pieces.  A
-        // tile is signalled once its copies (and those of the tile before) have
-        // landed: after the next tile's K copies are issued when the next
-        // gathered tile follows directly, else at once.
-        const int g = threadIdx.x - 256;
-        auto next_gathered = [&](int u) {
-            for (; u < n_tiles; ++u)
-                if (st.gathered(tile_of(u))) return u;
-            return n_tiles;
-        };
-        auto signal = [&](int s) {
-            cp_async_wait<0>();
-            fence_proxy_async_smem();
-            named_barrier(2, GATHER_THREADS);
-            if (g == 0) {
-                mbar_arrive_release_cluster(map_to_rank(&sm.k_full[s], 0));
-                mbar_arrive_release_cluster(map_to_rank(&sm.v_full[s], 0));
-            }
-        };
-        int u = next_gathered(0);
-        int32_t nxt = (u < n_tiles && g < NTILE) ? gather_row(st, p, b, tile_of(u), g) : -1;
-        int pending = -1, gi = 0;
-        bool ok = true;
-        while (u < n_tiles) {
-            const int s = u & 1;
-            if (g < NTILE) sm.grow[s][g] = nxt;   // unmapped rows are flagged by the producer warp
-            const int un = next_gathered(u + 1);
-            if (un < n_tiles && g < NTILE) nxt = gather_row(st, p, b, tile_of(un), g);
-            ok = group_wait(sm, &sm.k_go[gi & 1], (gi >> 1) & 1, p.status, g);   // also publishes grow[s]
-            if (!ok) break;
-            const int32_t *gr = sm.grow[s];
-            const uint32_t kb = smem_addr(sm.k[s][0]);
-#pragma unroll
-            for (int i = 0; i < 32 * 72 / GATHER_THREADS; ++i) {
-                const int q = g + GATHER_THREADS * i;   // < 32 x 72
-                const int row = q / 72, w = q - row * 72;
-                const int32_t pr = gr[32 * (int)rank + row];
-                const uint32_t dst = kb + (w >> 3) * (32 * 128) + row * 128 + (((w & 7) ^ (row & 7)) << 4);
-                const uint8_t *src = pr >= 0 ? p.pool + (size_t)pr * p.row_bytes + w * 16 : p.pool;
-                cp_async16(dst, src, pr >= 0 ? 16u : 0u);
-            }
-            cp_async_commit();
-            if (pending >= 0) {
-                // the tile before is complete once at most this tile's K copies are in flight
-                cp_async_wait<1>();
-                fence_proxy_async_smem();
-                named_barrier(2, GATHER_THREADS);
-                if (g == 0) {
-                    mbar_arrive_release_cluster(map_to_rank(&sm.k_full[pending & 1], 0));
-                    mbar_arrive_release_cluster(map_to_rank(&sm.v_full[pending & 1], 0));
-                }
-                pending = -1;
-            }
-            ok = group_wait(sm, &sm.v_go[gi & 1], (gi >> 1) & 1, p.status, g);
-            if (!ok) break;
-            const uint32_t vb = smem_addr(sm.v[s][0][0]);
-#pragma unroll
-            for (int i = 0; i < 64 * 32 / GATHER_THREADS; ++i) {
-                const int q = g + GATHER_THREADS * i;   // < 64 x 32
-                const int row = q >> 5, w = q & 31, a = w >> 3, pp = w & 7;   // a = 2 j + atom
-                const int32_t pr = gr[row];
-                const uint32_t dst = vb + a * (NTILE * 128) + row * 128 + ((pp ^ (row & 7)) << 4);
-                const int col_chunk = 4 * (a >> 1) + 2 * (int)rank + (a & 1);
-                const uint8_t *src = pr >= 0 ? p.pool + (size_t)pr * p.row_bytes + col_chunk * 128 + pp * 16 : p.pool;
-                cp_async16(dst, src, pr >= 0 ? 16u : 0u);
-            }
-            cp_async_commit();
-            if (un == u + 1) pending = u;
-            else signal(s);
-            u = un;
-            ++gi;
-        }
-        cp_async_wait<0>();   // no copy may land after the CTA has left
-        if (ok && pending >= 0) signal(pending & 1);
     } else if (warp >= 4 && warp < 8) {
         // ------------------------------------------------ softmax + epilogue
         const int L = threadIdx.x - 128;        // TMEM lane of this thread
@@ -684,19 +605,28 @@ int max_splits(int B) {
     return max(1, clusters / max(B, 1));
 }
 
+// Staging slots per sequence that a call may need: every top-k tile plus every
+// window tile (a window that does not start on a chunk boundary is staged whole).
+int stage_tiles(int k, int max_window_len) { return (k + NTILE - 1) / NTILE + (max_window_len + NTILE - 1) / NTILE + 1; }
+size_t stage_bytes(int B, int k, int max_window_len) {
+    return (size_t)B * stage_tiles(k, max_window_len) * NTILE * DQK * 2;
+}
+
 int launch(const uint16_t *q, const uint16_t *kv_pool, int64_t k_stride, int64_t n_slots, const int32_t *table,
            int table_stride, const int32_t *topk_idx, const int32_t *topk_count, int k, const int32_t *window_start,
-           const int32_t *window_len, int B, float scale, int n_splits, float *o_part, float *m_part, float *l_part,
-           int32_t *status, cudaStream_t stream) {
+           const int32_t *window_len, int max_window_len, int B, float scale, int n_splits, float *o_part,
+           float *m_part, float *l_part, uint8_t *stage, int32_t *status, cudaStream_t stream) {
     // Column chunk c of a row is 128 bytes at offset 128 c, so a row is also a
     // [9][64] array and boxes can span chunks as a third (and fourth) dimension:
     //   K: {64 columns, rows, 9 chunks}, box {64, 32, 9}  -> [chunk][32 rows][128 B]
     //   V: {64 columns, rows, 4 chunks, 2 groups of 4}, box {64, 64, 2, 2} at chunk 2r
     //      -> [group j][chunk 4j + 2r + a][64 rows][128 B]
     //   Q: {64 columns, B x 128 heads, 9 chunks}, box {64, 64, 9}
-    CUtensorMap k_map, v_map, q_map;
+    CUtensorMap k_map, v_map, ks_map, vs_map, q_map;
     const uint64_t pool_rows = (uint64_t)n_slots * LSA_CHUNK;
-    if (pool_rows + 64 >= (1ull << 31) || (uint64_t)B * HQ >= (1ull << 31))
+    const int G = stage_tiles(k, max_window_len);
+    const uint64_t stage_rows = (uint64_t)B * G * NTILE;
+    if (pool_rows + 64 >= (1ull << 31) || (uint64_t)B * HQ >= (1ull << 31) || stage_rows >= (1ull << 31))
         return fail(LSA_ERR_SHAPE, "lsa_sparse_decode: pool rows must stay below 2^31 for the latent kernel");
     const uint64_t rb = (uint64_t)k_stride * 2;
     const uint64_t kd[3] = {64, pool_rows, KCH}, ks[2] = {rb, 128};
@@ -707,6 +637,11 @@ int launch(const uint16_t *q, const uint16_t *kv_pool, int64_t k_stride, int64_t
     const uint32_t qbox[3] = {64, HPC, KCH};
     if (!make_map(&k_map, kv_pool, 3, kd, ks, kbox) || !make_map(&v_map, kv_pool, 4, vd, vs, vbox))
         return fail(LSA_ERR_CUDA, "lsa_sparse_decode: cuTensorMapEncodeTiled failed for the KV pool");
+    // the staging buffer: the same boxes over dense rows of DQK elements
+    const uint64_t skd[3] = {64, stage_rows, KCH}, sks[2] = {DQK * 2, 128};
+    const uint64_t svd[4] = {64, stage_rows, 4, 2}, svs[3] = {DQK * 2, 128, 512};
+    if (!make_map(&ks_map, stage, 3, skd, sks, kbox) || !make_map(&vs_map, stage, 4, svd, svs, vbox))
+        return fail(LSA_ERR_CUDA, "lsa_sparse_decode: cuTensorMapEncodeTiled failed for the staging buffer");
     if (!make_map(&q_map, q, 3, qd, qs, qbox))
         return fail(LSA_ERR_CUDA, "lsa_sparse_decode: cuTensorMapEncodeTiled failed for q");
     Params prm;
@@ -715,8 +650,12 @@ int launch(const uint16_t *q, const uint16_t *kv_pool, int64_t k_stride, int64_t
     prm.pool = reinterpret_cast<const uint8_t *>(kv_pool); prm.row_bytes = (int64_t)rb;
     prm.o_part = o_part; prm.m_part = m_part; prm.l_part = l_part; prm.status = status;
     prm.n_rows_pool = n_slots * LSA_CHUNK; prm.table_stride = table_stride; prm.k = k; prm.n_splits = n_splits;
+    prm.stage_tiles = G;
     prm.scale_log2 = scale * 1.4426950408889634f;
     prm.stall = take_test_stall(LSA_TEST_STALL_ATTENTION);
+    stage_kernel<<<dim3(G, B), 256, 0, stream>>>(prm, stage);
+    int rc = check_launch("stage_kernel");
+    if (rc) return rc;
     const size_t smem = smem_bytes();
     LSA_CUDA(cudaFuncSetAttribute(mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     cudaLaunchConfig_t cfg = {};
@@ -731,7 +670,7 @@ int launch(const uint16_t *q, const uint16_t *kv_pool, int64_t k_stride, int64_t
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    LSA_CUDA(cudaLaunchKernelEx(&cfg, mla_decode_kernel, k_map, v_map, q_map, prm));
+    LSA_CUDA(cudaLaunchKernelEx(&cfg, mla_decode_kernel, k_map, v_map, ks_map, vs_map, q_map, prm));
     return LSA_OK;
 }
 

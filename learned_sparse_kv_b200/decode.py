@@ -314,19 +314,25 @@ class Window:
 
     def launches_per_window(self) -> int:
         """Kernels this library launches per window of resident pools (select: 2, or 0 for the
-        recency baseline, which only fills memory; per step: append 1, top-k 2 or 3, decode 2).
+        recency baseline, which only fills memory; per step: append 1, top-k 2 or 3, decode 2 or 3).
 
         The top-k call counts the kept cold chunks inside the tcgen05 indexer kernel when
         that kernel serves the indexer shape, else in a kernel of its own."""
         sel = 0 if (self.selector is not None and self.selector["mode"] == lsa.SELECT_RECENT) else 2
-        return sel + self.s.steps * (1 + lsa.topk_kernel_count(self.s.B, self.s.Hl, self.s.dl) + 2)
+        return sel + self.s.steps * (1 + lsa.topk_kernel_count(self.s.B, self.s.Hl, self.s.dl) + self._decode_kernels())
+
+    def _decode_kernels(self) -> int:
+        """Kernels of one attention call: the 128-head latent shape stages its gathered tiles,
+        runs the split-K kernel and merges; the other shapes run split-K and merge."""
+        return 3 if (self.s.latent and self.s.Hq == 128) else 2
 
     def launches_cold(self, n_windows: int) -> int:
         """Kernels of run_cold over n_windows: per window its gate (2), plan (1) and fetch (1);
         window 0's first step is append, two attention calls, top-k and a merge; the other
         steps as launches_per_window; one window advance per later window."""
-        per_step = 1 + lsa.topk_kernel_count(self.s.B, self.s.Hl, self.s.dl) + 2
-        first = 1 + 2 + lsa.topk_kernel_count(self.s.B, self.s.Hl, self.s.dl) + 2 + 1
+        dk = self._decode_kernels()
+        per_step = 1 + lsa.topk_kernel_count(self.s.B, self.s.Hl, self.s.dl) + dk
+        first = 1 + dk + lsa.topk_kernel_count(self.s.B, self.s.Hl, self.s.dl) + dk + 1
         sel = 0 if (self.selector is not None and self.selector["mode"] == lsa.SELECT_RECENT) else 2
         return n_windows * (sel + 2) + first + (n_windows * self.s.steps - 1) * per_step + (n_windows - 1)
 
