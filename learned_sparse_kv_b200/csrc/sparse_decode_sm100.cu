@@ -8,32 +8,28 @@
 // cta_group::2 tcgen05.mma with M = 128 query heads: CTA r holds heads
 // 64r..64r+63 of Q and of P in its shared memory, the B operand is split by
 // N between the pair, and each CTA's tensor memory receives its own heads'
-// rows of the result.  Rows are taken 64 at a time ("units": a chunk slot of
-// the pool, or a slot of the staging buffer) and two units form a tile:
-//   S = Q K^T   N = 128 kv rows per tile (CTA r holds unit r: 64 rows, all 576
-//               columns); 36 MMAs per tile -- at N = 64 an MMA costs nearly as
-//               much as at N = 128, so the wider tile halves the Q.K^T
-//               instructions per row
-//   O += P V    N = 256 value columns per MMA (CTA r holds all 128 rows of value
+// rows of the result.
+//   S = Q K^T   N = 64 kv rows per tile (CTA r holds rows 32r..32r+31, all 576 columns)
+//   O += P V    N = 256 value columns per MMA (CTA r holds all 64 rows of value
 //               columns 128r..128r+127 and 256+128r..); P is passed as the sum
 //               of two bf16 parts, hi = bf16(P) and lo = bf16(P - hi), so every
-//               K step takes two MMAs per value block and P keeps ~16 bits
-// K arrives in nine column chunks of 8 KB (64 rows x 64 columns), each with its
-// own barrier: the ring holds one tile, and chunk c of the next tile is loaded
-// as soon as the Q.K^T step that reads chunk c of this tile is done.  V arrives
-// in 32-row chunks of 16 KB through a ring of two.  Shared memory per CTA:
-// Q 72 KB, K 72 KB, V 32 KB, P 32 KB.
-// TMEM per CTA: two S buffers of 64 columns and O = 64 heads x 512 values in
+//               K step takes four MMAs and P keeps ~16 bits of precision
+// TMEM per CTA: two S buffers of 32 columns and O = 64 heads x 512 values in
 // 256 columns.
 //
-// Every load is one TMA box straight into the 128-byte-swizzled operand layout.
-// Window units that are a whole aligned chunk slot are read from the pool;
-// the other units (top-k rows, and window units that are not a whole aligned
-// chunk) are first copied, 64 rows at a time, by stage_kernel into a
-// contiguous staging buffer (missing rows zero-filled): that copy runs on every
-// multiprocessor at the memory's rate.
+// Loading a tile is one operation per operand: a 3D TMA box {64 columns, 32
+// rows, 9 column chunks} fetches a CTA's K rows (36 KB) and a 4D box {64, 64
+// rows, 2, 2} its value columns (32 KB), both straight into the 128-byte-swizzled
+// operand layout.  Window tiles that are a whole aligned chunk slot are read
+// from the pool; the other tiles (top-k rows, and window tiles that are not a
+// whole aligned chunk) are first copied, 64 rows at a time, by stage_kernel
+// into a contiguous staging buffer (missing rows zero-filled), so that they are
+// TMA boxes too: that copy runs on every multiprocessor at the memory's rate,
+// where row gathers inside this kernel were bound by the copies one
+// multiprocessor keeps in flight and stalled the two-stage pipeline.  Two
+// stages of each operand are in flight.
 // Warp roles:
-//   0      K producer (TMA), unit-validity masks
+//   0      K producer (TMA), tile-validity masks
 //   1      S = Q K^T issuer (even CTA)        2   O += P V issuer (even CTA)
 //   3      TMEM allocator, V producer (TMA)
 //   4..7   softmax, O rescale, epilogue (one thread per TMEM lane)
@@ -56,41 +52,40 @@ using namespace sm100;
 constexpr int HPC = 64;           // heads per CTA
 constexpr int HQ = 128;           // heads per cluster
 constexpr int DQK = 576, DV = 512;
-constexpr int NTILE = 64;         // kv rows per unit (a chunk slot or a staging slot)
+constexpr int NTILE = 64;         // kv rows per tile
 constexpr int KCH = DQK / 64;     // 9 column chunks of 64
-constexpr int VCH = 4;            // 32-row V chunks per tile (two units)
-constexpr int VSLOTS = 2;         // V ring
-constexpr int INFO = 4;           // unit-validity ring (one entry per tile)
+constexpr int STAGES = 2;         // tiles in flight per operand
+constexpr int INFO = 4;           // tile-validity ring
 constexpr int THREADS = 256;
 constexpr uint32_t Q_BYTES = KCH * HPC * 128;          // per CTA
-constexpr uint32_t KC_BYTES = NTILE * 128;             // one K column chunk of one unit
-constexpr uint32_t VC_BYTES = 2 * 2 * 32 * 128;        // one V chunk: [value block][atom][32 rows][128 B]
+constexpr uint32_t K_BYTES = KCH * 32 * 128;           // per CTA and tile
+constexpr uint32_t V_BYTES = 2 * 2 * NTILE * 128;      // per CTA and tile
 constexpr float RESCALE_LOG2 = 8.f;
 
 // TMEM columns
-constexpr uint32_t TM_S = 0;      // S buffers at 0 and 64 (N = 128 over the pair: 64 columns per CTA)
-constexpr uint32_t TM_O = 128;    // O at 128..383
+constexpr uint32_t TM_S = 0;      // S buffers at 0 and 32
+constexpr uint32_t TM_O = 64;     // O at 64..319
 constexpr uint32_t TM_COLS = 512;
 
 struct __align__(1024) Smem {
     uint8_t q[KCH][HPC * 128];                 // 9 x [64 heads][128 B], 128B-swizzled, K-major
-    uint8_t k[KCH][NTILE * 128];               // chunk c of this CTA's unit: [64 kv rows][64 cols], K-major
-    uint8_t v[VSLOTS][2][2][32 * 128];         // [slot][value block j][atom][32 kv rows][64 value cols], MN-major
-    uint8_t p[2][2][HPC * 128];                // P = hi + lo: [part][unit][64 heads][64 kv], K-major
-    uint64_t k_full[KCH], k_empty[KCH];
-    uint64_t v_full[VSLOTS], v_empty[VSLOTS];
+    uint8_t k[STAGES][KCH][32 * 128];          // [chunk][32 kv rows][64 cols]
+    uint8_t v[STAGES][2][2][NTILE * 128];      // [value block j][atom][64 kv rows][64 value cols], MN-major
+    uint8_t p[2][HPC * 128];                   // P = hi + lo: [part][64 heads][64 kv], K-major
+    uint64_t k_full[STAGES], k_empty[STAGES];
+    uint64_t v_full[STAGES], v_empty[STAGES];
     uint64_t q_full;
-    uint64_t s_full[2], s_empty[2], p_full;
-    uint64_t pv_done, mma_done;     // pv_done: P.V of a tile
+    uint64_t s_full[2], s_empty[2], p_full[2];
+    uint64_t pv_done[2], mma_done;   // pv_done[u & 1]: P.V of tile u
     uint64_t info_full[INFO], info_empty[INFO];
-    unsigned long long info_mask[INFO][2];
+    unsigned long long info_mask[INFO];
     float red[128];
     uint32_t tmem_base;
     int abort_flag;
-    // drain bookkeeping: the tile (K) or chunk (V) of the last TMA load this CTA issued into
-    // each slot (-1: none), and (even CTA) how far the issuers consumed them
-    int last_k_tma[KCH], last_v_tma[VSLOTS];
-    int k_cons[KCH], v_consumed, q_seen;
+    // drain bookkeeping: the tile of the last TMA load this CTA issued into each stage
+    // (-1: none), and (even CTA) the tiles whose K / V full phase an issuer saw complete
+    int last_k_tma[STAGES], last_v_tma[STAGES];
+    int k_consumed, v_consumed, q_seen;
     uint64_t never;                  // no arrival ever: the failure-path test's wait
 };
 static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory of one CTA");
@@ -206,16 +201,14 @@ __device__ __forceinline__ bool warp_wait_cluster(Smem &sm, const uint64_t *bar,
     return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
-// Waits until the TMA load last issued into a slot has landed, if no issuer saw its full
-// phase complete.  u0 / u1: that load's index as issued by the even / odd CTA (-1: none);
-// consumed: loads of this slot the issuer saw complete (as an index bound); the phase
-// parity of load u is parity(u).
-__device__ __forceinline__ void drain_slot(uint64_t *full, int u0, int u1, int consumed, uint32_t parity_of_u) {
+// Waits until the TMA load of the last tile issued into a stage has landed, if no issuer
+// saw its full phase complete.  u0 / u1: that tile as issued by the even / odd CTA.
+__device__ __forceinline__ void drain_stage(uint64_t *full, int u0, int u1, int consumed) {
     const int u = max(u0, u1);
-    if (u < consumed) return;               // completed and consumed, or nothing issued (u = -1)
-    if (u0 != u) mbar_arrive_local(full);   // the even CTA did not issue load u
-    if (u1 != u) mbar_arrive_local(full);   // the odd CTA did not issue load u
-    (void)mbar_wait(full, parity_of_u, WAIT_NS);
+    if (u < consumed) return;            // completed and consumed, or nothing issued (u = -1)
+    if (u0 != u) mbar_arrive_local(full);   // the even CTA did not issue tile u
+    if (u1 != u) mbar_arrive_local(full);   // the odd CTA did not issue tile u
+    (void)mbar_wait(full, (uint32_t)(u >> 1) & 1u, WAIT_NS);
 }
 
 // grid (stage_tiles, B), 256 threads: staging slot g of sequence b receives the 64 rows of
@@ -243,33 +236,6 @@ __global__ void __launch_bounds__(256) stage_kernel(const Params p, uint8_t *__r
     for (int i = 0; i < PER_THREAD; ++i) dst[threadIdx.x + 256 * i] = v[i];
 }
 
-// Rows of unit t: its first row in the pool or the staging buffer, and which map to read.
-struct UnitSrc {
-    int y;        // first row (out of range for a missing unit or slot: TMA fills zeros)
-    bool staged;
-};
-__device__ __forceinline__ UnitSrc unit_src(const SeqTiles &st, const Params &p, int b, int t) {
-    if (t >= st.total) return {(int)p.n_rows_pool, false};
-    if (st.gathered(t)) return {(b * p.stage_tiles + st.stage_index(t)) * NTILE, true};
-    const int64_t slot_row = st.window_slot_row(p, b, t);
-    return {slot_row >= 0 ? (int)slot_row : (int)p.n_rows_pool, false};
-}
-
-// Validity of the 64 rows of unit t (bit i: row i exists and has a slot); lane i looks
-// at rows i and i + 32.  A missing slot sets LSA_DEV_TABLE.
-__device__ __forceinline__ unsigned long long unit_mask(const SeqTiles &st, const Params &p, int b, int t, int lane) {
-    if (t >= st.total) return 0ull;
-    if (!st.gathered(t)) {
-        const int64_t slot_row = st.window_slot_row(p, b, t);
-        if (slot_row == -2 && lane == 0) flag(p.status, LSA_DEV_TABLE);
-        return slot_row < 0 ? 0ull : ~0ull;
-    }
-    const int64_t g0 = st.row(p, b, t, lane), g1 = st.row(p, b, t, lane + 32);
-    if (g0 == -2 || g1 == -2) flag(p.status, LSA_DEV_TABLE);
-    const unsigned lo = __ballot_sync(0xffffffffu, g0 >= 0), hi = __ballot_sync(0xffffffffu, g1 >= 0);
-    return (unsigned long long)lo | ((unsigned long long)hi << 32);
-}
-
 __global__ void __launch_bounds__(THREADS, 1)
 mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap v_map,
                   const __grid_constant__ CUtensorMap ks_map, const __grid_constant__ CUtensorMap vs_map,
@@ -281,18 +247,19 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
     const int split = blockIdx.x >> 1, b = blockIdx.y;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < KCH; ++i) { mbar_init(&sm.k_full[i], 2); mbar_init(&sm.k_empty[i], 1); }
-        for (int i = 0; i < VSLOTS; ++i) { mbar_init(&sm.v_full[i], 2); mbar_init(&sm.v_empty[i], 1); }
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(&sm.k_full[i], 2); mbar_init(&sm.k_empty[i], 1);
+            mbar_init(&sm.v_full[i], 2); mbar_init(&sm.v_empty[i], 1);
+        }
         mbar_init(&sm.q_full, 2);
-        for (int i = 0; i < 2; ++i) { mbar_init(&sm.s_full[i], 1); mbar_init(&sm.s_empty[i], 2); }
-        mbar_init(&sm.p_full, 2);
-        mbar_init(&sm.pv_done, 1);
+        for (int i = 0; i < 2; ++i) { mbar_init(&sm.s_full[i], 1); mbar_init(&sm.s_empty[i], 2); mbar_init(&sm.p_full[i], 2); }
+        mbar_init(&sm.pv_done[0], 1);
+        mbar_init(&sm.pv_done[1], 1);
         mbar_init(&sm.mma_done, 2);   // one commit from each MMA issuer
         for (int i = 0; i < INFO; ++i) { mbar_init(&sm.info_full[i], 1); mbar_init(&sm.info_empty[i], 1); }
         mbar_init(&sm.never, 1);
-        for (int i = 0; i < KCH; ++i) { sm.last_k_tma[i] = -1; sm.k_cons[i] = 0; }
-        for (int i = 0; i < VSLOTS; ++i) sm.last_v_tma[i] = -1;
-        sm.v_consumed = sm.q_seen = 0;
+        for (int i = 0; i < STAGES; ++i) sm.last_k_tma[i] = sm.last_v_tma[i] = -1;
+        sm.k_consumed = sm.v_consumed = sm.q_seen = 0;
         sm.abort_flag = 0;
         fence_mbar_init_cluster();
     }
@@ -304,59 +271,68 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
     const uint32_t tmem = sm.tmem_base;
 
     const SeqTiles st(p, b);
-    // Tiles are pairs of units (2j, 2j + 1), dealt round-robin: split s takes tiles s,
-    // s + n_splits, ...  The staged top-k units (first in the unit list) are thereby
-    // spread evenly over the splits.  K (warp 0) and V (warp 3) have a producer each.
-    const int n_pairs = (st.total + 1) >> 1;
-    const int n_tiles = split < n_pairs ? (n_pairs - 1 - split) / p.n_splits + 1 : 0;
-    auto tile_of = [&](int u) { return split + u * p.n_splits; };
-
-    if (warp == 0 && n_tiles > 0) {
-        // ------------------------------------------------ K producer + unit masks
-        if (lane == 0) {
+    // Tiles are dealt round-robin: split s takes tiles s, s + n_splits, ...  The
+    // staged top-k tiles (first in the tile list) are thereby spread evenly over
+    // the splits.  K (warp 0) and V (warp 3) have a producer each, so K of a later
+    // tile never waits behind the P.V that frees a V stage.
+    const int n_tiles = split < st.total ? (st.total - 1 - split) / p.n_splits + 1 : 0;
+    const int u0 = split, ustride = p.n_splits;
+    auto tile_of = [&](int u) { return u0 + u * ustride; };
+    if ((warp == 0 || warp == 3) && n_tiles > 0) {
+        // ------------------------------------------------ TMA producers (K + masks, V)
+        const bool kprod = warp == 0;
+        if (kprod && lane == 0) {
             const uint32_t qf = map_to_rank(&sm.q_full, 0);
             mbar_arrive_expect_tx_cluster(qf, Q_BYTES);
             tma_load_3d(sm.q[0], &q_map, 0, b * HQ + HPC * (int)rank, 0, qf);
         }
+        // row indices of the next gathered tile are loaded while the current tile is issued
+        int64_t n0 = -1, n1 = -1;
+        if (kprod && st.gathered(tile_of(0))) { n0 = st.row(p, b, tile_of(0), lane); n1 = st.row(p, b, tile_of(0), lane + 32); }
         for (int u = 0; u < n_tiles; ++u) {
-            const int j = tile_of(u);
-            const unsigned long long m0 = unit_mask(st, p, b, 2 * j, lane), m1 = unit_mask(st, p, b, 2 * j + 1, lane);
-            if (!warp_wait(sm, &sm.info_empty[u % INFO], ((u / INFO) + 1) & 1, p.status)) break;
-            if (lane == 0) {
-                sm.info_mask[u % INFO][0] = m0;
-                sm.info_mask[u % INFO][1] = m1;
-                asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];\n" ::"r"(smem_addr(&sm.info_full[u % INFO])) : "memory");
-            }
-            const UnitSrc src = unit_src(st, p, b, 2 * j + (int)rank);
-            bool ok = true;
-            for (int c = 0; c < KCH && ok; ++c) {
-                ok = warp_wait(sm, &sm.k_empty[c], (u + 1) & 1, p.status);
-                if (ok && lane == 0) {
-                    const uint32_t full = map_to_rank(&sm.k_full[c], 0);
-                    mbar_arrive_expect_tx_cluster(full, KC_BYTES);
-                    tma_load_3d(sm.k[c], src.staged ? &ks_map : &k_map, 0, src.y, c, full);
-                    sm.last_k_tma[c] = u;
+            const int t = tile_of(u);
+            const bool gath = st.gathered(t);
+            const int64_t slot_row = gath ? -2 : st.window_slot_row(p, b, t);
+            // an unmapped slot is read out of range: TMA fills zeros; a staged tile is read
+            // from its staging slot
+            const int wy = gath ? (b * p.stage_tiles + st.stage_index(t)) * NTILE
+                                : (slot_row >= 0 ? (int)slot_row : (int)p.n_rows_pool);
+            const int s = u & 1;
+            const uint32_t par = ((u >> 1) + 1) & 1;
+            if (kprod) {
+                const int64_t g0 = n0, g1 = n1;
+                if (u + 1 < n_tiles && st.gathered(tile_of(u + 1))) {
+                    n0 = st.row(p, b, tile_of(u + 1), lane);
+                    n1 = st.row(p, b, tile_of(u + 1), lane + 32);
                 }
-            }
-            __syncwarp();
-            if (!ok) break;
-        }
-    } else if (warp == 3 && n_tiles > 0) {
-        // ------------------------------------------------ V producer
-        bool ok = true;
-        for (int u = 0; u < n_tiles && ok; ++u) {
-            const int j = tile_of(u);
-            const UnitSrc s0 = unit_src(st, p, b, 2 * j), s1 = unit_src(st, p, b, 2 * j + 1);
-            for (int i = 0; i < VCH && ok; ++i) {
-                const int g = VCH * u + i, slot = g & 1;
-                const UnitSrc &src = i < 2 ? s0 : s1;
-                ok = warp_wait(sm, &sm.v_empty[slot], ((g >> 1) + 1) & 1, p.status);
-                if (ok && lane == 0) {
-                    const uint32_t full = map_to_rank(&sm.v_full[slot], 0);
-                    mbar_arrive_expect_tx_cluster(full, VC_BYTES);
-                    tma_load_4d(sm.v[slot][0][0], src.staged ? &vs_map : &v_map, 0, src.y + 32 * (i & 1),
-                                2 * (int)rank, 0, full);
-                    sm.last_v_tma[slot] = g;
+                unsigned long long mask;
+                if (!gath) {
+                    if (slot_row == -2) flag(p.status, LSA_DEV_TABLE);
+                    mask = slot_row < 0 ? 0ull : ~0ull;
+                } else {
+                    if ((g0 == -2 || g1 == -2)) flag(p.status, LSA_DEV_TABLE);
+                    const unsigned lo = __ballot_sync(0xffffffffu, g0 >= 0), hi = __ballot_sync(0xffffffffu, g1 >= 0);
+                    mask = (unsigned long long)lo | ((unsigned long long)hi << 32);
+                }
+                if (!warp_wait(sm, &sm.info_empty[u % INFO], ((u / INFO) + 1) & 1, p.status)) break;
+                if (lane == 0) {
+                    sm.info_mask[u % INFO] = mask;
+                    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];\n" ::"r"(smem_addr(&sm.info_full[u % INFO])) : "memory");
+                }
+                if (!warp_wait(sm, &sm.k_empty[s], par, p.status)) break;
+                if (lane == 0) {
+                    const uint32_t full = map_to_rank(&sm.k_full[s], 0);
+                    mbar_arrive_expect_tx_cluster(full, K_BYTES);
+                    tma_load_3d(sm.k[s][0], gath ? &ks_map : &k_map, 0, wy + 32 * (int)rank, 0, full);
+                    sm.last_k_tma[s] = u;
+                }
+            } else {
+                if (!warp_wait(sm, &sm.v_empty[s], par, p.status)) break;
+                if (lane == 0) {
+                    const uint32_t full = map_to_rank(&sm.v_full[s], 0);
+                    mbar_arrive_expect_tx_cluster(full, V_BYTES);
+                    tma_load_4d(sm.v[s][0][0], gath ? &vs_map : &v_map, 0, wy, 2 * (int)rank, 0, full);
+                    sm.last_v_tma[s] = u;
                 }
             }
             __syncwarp();
@@ -367,74 +343,72 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
         // own MMAs, so neither chain waits behind the other's operands.
         // Descriptors are built once; a byte offset o within shared memory is
         // o >> 4 added to the descriptor's start-address field.
-        constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 2 * NTILE, false, false);
+        constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, NTILE, false, false);
         constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 256, false, true);
         constexpr uint64_t K16 = 32 >> 4;
         bool ok = true;
         if (warp == 1) {
-            constexpr uint64_t Q_CHUNK = (HPC * 128) >> 4, K_CHUNK = KC_BYTES >> 4;
+            constexpr uint64_t Q_CHUNK = (HPC * 128) >> 4, K_CHUNK = (32 * 128) >> 4, K_STAGE = K_BYTES >> 4;
             const uint64_t qd0 = smem_desc_sw128(smem_addr(sm.q[0]), 16, 1024);
-            const uint64_t kd0 = smem_desc_sw128(smem_addr(sm.k[0]), 16, 1024);
+            const uint64_t kd0 = smem_desc_sw128(smem_addr(sm.k[0][0]), 16, 1024);
             if (p.stall) ok = warp_wait(sm, &sm.never, 0, p.status, TEST_STALL_NS);
             ok = ok && warp_wait(sm, &sm.q_full, 0, p.status);
             if (ok && lane == 0) sm.q_seen = 1;
             for (int u = 0; u < n_tiles && ok; ++u) {      // S(u) = Q K^T
                 const int sb = u & 1;
-                ok = warp_wait(sm, &sm.s_empty[sb], ((u >> 1) + 1) & 1, p.status);
-                for (int c = 0; c < KCH && ok; ++c) {
-                    ok = warp_wait_cluster(sm, &sm.k_full[c], u & 1, p.status);
-                    if (!ok) break;
-                    tc_fence_after();
-                    if (lane == 0) {
-                        sm.k_cons[c] = u + 1;
+                ok = warp_wait(sm, &sm.s_empty[sb], ((u >> 1) + 1) & 1, p.status) &&
+                     warp_wait_cluster(sm, &sm.k_full[sb], (u >> 1) & 1, p.status);
+                if (!ok) break;
+                if (lane == 0) sm.k_consumed = u + 1;
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t d = tmem + TM_S + 32 * sb;
+                    const uint64_t kb = kd0 + K_STAGE * sb;
+#pragma unroll
+                    for (int c = 0; c < KCH; ++c)
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            umma_pair_ss(tmem + TM_S + 64 * sb, qd0 + Q_CHUNK * c + K16 * kk,
-                                         kd0 + K_CHUNK * c + K16 * kk, IDESC_QK, (c | kk) != 0);
-                        umma_commit_pair(&sm.k_empty[c], 0x3);
-                        if (c == KCH - 1) umma_commit_pair(&sm.s_full[sb], 0x3);
-                    }
-                    __syncwarp();
+                            umma_pair_ss(d, qd0 + Q_CHUNK * c + K16 * kk, kb + K_CHUNK * c + K16 * kk, IDESC_QK,
+                                         (c | kk) != 0);
+                    umma_commit_pair(&sm.k_empty[sb], 0x3);
+                    umma_commit_pair(&sm.s_full[sb], 0x3);
                 }
+                __syncwarp();
             }
         } else {
-            constexpr uint64_t P_PART = (2 * HPC * 128) >> 4, P_UNIT = (HPC * 128) >> 4;
-            constexpr uint64_t V_SLOT = VC_BYTES >> 4, V_J = (2 * 32 * 128) >> 4, V16 = (16 * 128) >> 4;
-            const uint64_t pd0 = smem_desc_sw128(smem_addr(sm.p[0][0]), 16, 1024);
-            const uint64_t vd0 = smem_desc_sw128(smem_addr(sm.v[0][0][0]), 32 * 128, 1024);
+            constexpr uint64_t P_BUF = (HPC * 128) >> 4, V_STAGE = V_BYTES >> 4, V_J = (2 * NTILE * 128) >> 4;
+            constexpr uint64_t V16 = (16 * 128) >> 4;
+            const uint64_t pd0 = smem_desc_sw128(smem_addr(sm.p[0]), 16, 1024);
+            const uint64_t vd0 = smem_desc_sw128(smem_addr(sm.v[0][0][0]), NTILE * 128, 1024);
             for (int u = 0; u < n_tiles && ok; ++u) {      // O += P V for tile u
-                ok = warp_wait(sm, &sm.p_full, u & 1, p.status);
-                for (int i = 0; i < VCH && ok; ++i) {
-                    const int g = VCH * u + i, slot = g & 1;
-                    ok = warp_wait_cluster(sm, &sm.v_full[slot], (g >> 1) & 1, p.status);
-                    if (!ok) break;
-                    tc_fence_after();
-                    if (lane == 0) {
-                        sm.v_consumed = g + 1;
-                        const uint64_t vb = vd0 + V_SLOT * slot;
-                        // chunk i holds kv rows 32 i .. 32 i + 31 of the tile: P unit i / 2, columns 32 (i & 1) ..
+                const int sb = u & 1;
+                ok = warp_wait(sm, &sm.p_full[sb], (u >> 1) & 1, p.status) &&
+                     warp_wait_cluster(sm, &sm.v_full[sb], (u >> 1) & 1, p.status);
+                if (!ok) break;
+                if (lane == 0) sm.v_consumed = u + 1;
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint64_t vb = vd0 + V_STAGE * sb;
 #pragma unroll
-                        for (int jv = 0; jv < 2; ++jv)
+                    for (int j = 0; j < 2; ++j)
 #pragma unroll
-                            for (int kk = 0; kk < 2; ++kk) {
-                                const uint64_t bv = vb + V_J * jv + V16 * kk;
-                                const uint64_t pa = pd0 + P_UNIT * (i >> 1) + K16 * (2 * (i & 1) + kk);
-                                umma_pair_ss(tmem + TM_O + 128 * jv, pa, bv, IDESC_PV, (u | i | kk) != 0);
-                                umma_pair_ss(tmem + TM_O + 128 * jv, pa + P_PART, bv, IDESC_PV, true);
-                            }
-                        umma_commit_pair(&sm.v_empty[slot], 0x3);
-                        if (i == VCH - 1) umma_commit_pair(&sm.pv_done, 0x3);
-                    }
-                    __syncwarp();
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint64_t b = vb + V_J * j + V16 * kk;
+                            umma_pair_ss(tmem + TM_O + 128 * j, pd0 + K16 * kk, b, IDESC_PV, u > 0 || kk > 0);
+                            umma_pair_ss(tmem + TM_O + 128 * j, pd0 + P_BUF + K16 * kk, b, IDESC_PV, true);
+                        }
+                    umma_commit_pair(&sm.v_empty[sb], 0x3);
+                    umma_commit_pair(&sm.pv_done[sb], 0x3);
                 }
+                __syncwarp();
             }
         }
         if (lane == 0) umma_commit_pair(&sm.mma_done, 0x3);
         __syncwarp();
-    } else if (warp >= 4) {
+    } else if (warp >= 4 && warp < 8) {
         // ------------------------------------------------ softmax + epilogue
         const int L = threadIdx.x - 128;        // TMEM lane of this thread
-        const int h = L & 63, half = L >> 6;     // head within the CTA, unit of the tile
+        const int h = L & 63, half = L >> 6;     // head within the CTA, kv half of the tile
         const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
         float m_run = -INFINITY, m_ref = -INFINITY, l = 0.f;
         bool ok = true;
@@ -442,13 +416,12 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             const int s = u & 1;
             ok = ok && sm.abort_flag == 0;
             if (ok) ok = mbar_wait(&sm.info_full[u % INFO], (u / INFO) & 1, WAIT_NS, &sm.abort_flag);
-            const unsigned long long vmask = ok ? sm.info_mask[u % INFO][half] : 0ull;
+            const uint32_t vmask = ok ? (uint32_t)(sm.info_mask[u % INFO] >> (32 * half)) : 0u;
             if (ok) ok = mbar_wait(&sm.s_full[s], (u >> 1) & 1, WAIT_NS, &sm.abort_flag);
             if (!ok && sm.abort_flag == 0) set_abort(sm, p.status);
             tc_fence_after();
-            uint32_t raw[64];
-            tmem_ld32(tmem + lane_base + TM_S + 64 * s, *reinterpret_cast<uint32_t(*)[32]>(raw));
-            tmem_ld32(tmem + lane_base + TM_S + 64 * s + 32, *reinterpret_cast<uint32_t(*)[32]>(raw + 32));
+            uint32_t raw[32];
+            tmem_ld32(tmem + lane_base + TM_S + 32 * s, raw);
             tmem_wait_ld();
             tc_fence_before();
             named_barrier(1, 128);
@@ -456,12 +429,12 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 mbar_arrive_cluster(map_to_rank(&sm.s_empty[s], 0));
                 asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];\n" ::"r"(smem_addr(&sm.info_empty[u % INFO])) : "memory");
             }
+            float sv[32];
             float mx = -INFINITY;
 #pragma unroll
-            for (int i = 0; i < 64; ++i) {
-                const float x = (vmask >> i) & 1ull ? __uint_as_float(raw[i]) * p.scale_log2 : -INFINITY;
-                raw[i] = __float_as_uint(x);
-                mx = fmaxf(mx, x);
+            for (int i = 0; i < 32; ++i) {
+                sv[i] = (vmask >> i) & 1u ? __uint_as_float(raw[i]) * p.scale_log2 : -INFINITY;
+                mx = fmaxf(mx, sv[i]);
             }
             sm.red[L] = mx;
             named_barrier(1, 128);
@@ -477,10 +450,10 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             // P = hi + lo, both bf16: rounding P to one bf16 alone leaves a relative error
             // of 2^-9 on every weight, which peaked rows carry straight into the output.
             float psum = 0.f;
-            uint32_t pk_hi[32], pk_lo[32];
+            uint32_t pk_hi[16], pk_lo[16];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const float p0 = exp2f(__uint_as_float(raw[2 * i]) - m_ref), p1 = exp2f(__uint_as_float(raw[2 * i + 1]) - m_ref);
+            for (int i = 0; i < 16; ++i) {
+                const float p0 = exp2f(sv[2 * i] - m_ref), p1 = exp2f(sv[2 * i + 1] - m_ref);
                 const float q0 = m_ref == -INFINITY ? 0.f : p0, q1 = m_ref == -INFINITY ? 0.f : p1;
                 psum += q0 + q1;
                 const __nv_bfloat162 hi = __floats2bfloat162_rn(q0, q1);
@@ -488,9 +461,9 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 pk_lo[i] = pack_bf16x2(q0 - __low2float(hi), q1 - __high2float(hi));
             }
             l += psum;
-            // The P buffer is rewritten and O may be rescaled: P.V of tile u-1 must be done.
+            // The P buffers are rewritten and O may be rescaled: P.V of tile u-1 must be done.
             if (u > 0 && ok) {
-                ok = mbar_wait(&sm.pv_done, (u - 1) & 1, WAIT_NS, &sm.abort_flag);
+                ok = mbar_wait(&sm.pv_done[(u - 1) & 1], ((u - 1) >> 1) & 1, WAIT_NS, &sm.abort_flag);
                 if (!ok && sm.abort_flag == 0) set_abort(sm, p.status);
             }
             // tcgen05.ld / st are warp-collective: the whole warp takes the rescale when
@@ -508,10 +481,10 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 }
                 tmem_wait_st();
             }
-            uint8_t *prow_hi = sm.p[0][half] + h * 128, *prow_lo = sm.p[1][half] + h * 128;
+            uint8_t *prow_hi = sm.p[0] + h * 128, *prow_lo = sm.p[1] + h * 128;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const int off = (c ^ (h & 7)) << 4;
+            for (int c = 0; c < 4; ++c) {
+                const int chunk = 4 * half + c, off = (chunk ^ (h & 7)) << 4;
                 *reinterpret_cast<uint4 *>(prow_hi + off) =
                     make_uint4(pk_hi[4 * c], pk_hi[4 * c + 1], pk_hi[4 * c + 2], pk_hi[4 * c + 3]);
                 *reinterpret_cast<uint4 *>(prow_lo + off) =
@@ -520,11 +493,11 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             fence_proxy_async_smem();
             tc_fence_before();
             named_barrier(1, 128);
-            if (L == 0) mbar_arrive_cluster(map_to_rank(&sm.p_full, 0));
+            if (L == 0) mbar_arrive_cluster(map_to_rank(&sm.p_full[s], 0));
         }
         // ---- epilogue: wait for the last P.V, then write the partial
         if (n_tiles > 0 && ok) {
-            ok = mbar_wait(&sm.pv_done, (n_tiles - 1) & 1, WAIT_NS, &sm.abort_flag);
+            ok = mbar_wait(&sm.pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, WAIT_NS, &sm.abort_flag);
             if (!ok && sm.abort_flag == 0) set_abort(sm, p.status);
         }
         tc_fence_after();
@@ -549,8 +522,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                 for (int i = 0; i < 32; ++i) o[i] = 0u;
             }
             // O columns 0..127 hold values 0..255 split by lane half; 128..255 hold 256..511
-            const int jv = q >> 2, within = (q & 3) * 32;
-            float4 *dst = reinterpret_cast<float4 *>(orow + 256 * jv + 128 * half + within);
+            const int j = q >> 2, within = (q & 3) * 32;
+            float4 *dst = reinterpret_cast<float4 *>(orow + 256 * j + 128 * half + within);
 #pragma unroll
             for (int i = 0; i < 8; ++i)
                 dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
@@ -571,25 +544,19 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
     // value here from their own shared memory (no read of the peer: it may leave after the
     // barrier unless both take the abort path, which ends with a second barrier).
     if (sm.abort_flag) {
-        if (rank == 0 && threadIdx.x == 0 && n_tiles > 0) {
-            // After an abort, every TMA load either CTA issued lands before either CTA leaves:
-            // Q (issued by both producers before their loops), and per slot the last K chunk
-            // and V chunk that no issuer consumed.  Where only one CTA issued that load, this
-            // thread arrives in place of the other, so the phase completes once the issued
-            // bytes have landed.  Every wait is bounded.
-            if (!sm.q_seen) (void)mbar_wait(&sm.q_full, 0, WAIT_NS);
-            for (int c = 0; c < KCH; ++c) {
-                const int u = max(sm.last_k_tma[c], ld_peer_s32(&sm.last_k_tma[c]));
-                drain_slot(&sm.k_full[c], sm.last_k_tma[c], ld_peer_s32(&sm.last_k_tma[c]), sm.k_cons[c],
-                           (uint32_t)u & 1u);
-            }
-            for (int i = 0; i < VSLOTS; ++i) {
-                const int g = max(sm.last_v_tma[i], ld_peer_s32(&sm.last_v_tma[i]));
-                drain_slot(&sm.v_full[i], sm.last_v_tma[i], ld_peer_s32(&sm.last_v_tma[i]), sm.v_consumed,
-                           (uint32_t)(g >> 1) & 1u);
-            }
+      if (rank == 0 && threadIdx.x == 0 && n_tiles > 0) {
+        // After an abort, every TMA load either CTA issued lands before either CTA leaves:
+        // Q (issued by both producers before their loops), and per stage the last K and V
+        // tiles whose full phase no issuer saw complete.  Where only one CTA issued that
+        // tile, this thread arrives in place of the other, so the phase completes once the
+        // issued bytes have landed.  Every wait is bounded.
+        if (!sm.q_seen) (void)mbar_wait(&sm.q_full, 0, WAIT_NS);
+        for (int s = 0; s < STAGES; ++s) {
+            drain_stage(&sm.k_full[s], sm.last_k_tma[s], ld_peer_s32(&sm.last_k_tma[s]), sm.k_consumed);
+            drain_stage(&sm.v_full[s], sm.last_v_tma[s], ld_peer_s32(&sm.last_v_tma[s]), sm.v_consumed);
         }
-        cluster_sync();   // the odd CTA leaves only after the drain
+      }
+      cluster_sync();   // the odd CTA leaves only after the drain
     }
     if (warp == 3) {
         tc_fence_after();
@@ -651,9 +618,9 @@ int launch(const uint16_t *q, const uint16_t *kv_pool, int64_t k_stride, int64_t
            float *m_part, float *l_part, uint8_t *stage, int32_t *status, cudaStream_t stream) {
     // Column chunk c of a row is 128 bytes at offset 128 c, so a row is also a
     // [9][64] array and boxes can span chunks as a third (and fourth) dimension:
-    //   K: {64 columns, rows, 9 chunks}, box {64, 64, 1} at chunk c -> one unit's chunk c, [64 rows][128 B]
-    //   V: {64 columns, rows, 4 chunks, 2 groups of 4}, box {64, 32, 2, 2} at chunk 2r
-    //      -> [group j][chunk 4j + 2r + a][32 rows][128 B]
+    //   K: {64 columns, rows, 9 chunks}, box {64, 32, 9}  -> [chunk][32 rows][128 B]
+    //   V: {64 columns, rows, 4 chunks, 2 groups of 4}, box {64, 64, 2, 2} at chunk 2r
+    //      -> [group j][chunk 4j + 2r + a][64 rows][128 B]
     //   Q: {64 columns, B x 128 heads, 9 chunks}, box {64, 64, 9}
     CUtensorMap k_map, v_map, ks_map, vs_map, q_map;
     const uint64_t pool_rows = (uint64_t)n_slots * LSA_CHUNK;
@@ -663,9 +630,9 @@ int launch(const uint16_t *q, const uint16_t *kv_pool, int64_t k_stride, int64_t
         return fail(LSA_ERR_SHAPE, "lsa_sparse_decode: pool rows must stay below 2^31 for the latent kernel");
     const uint64_t rb = (uint64_t)k_stride * 2;
     const uint64_t kd[3] = {64, pool_rows, KCH}, ks[2] = {rb, 128};
-    const uint32_t kbox[3] = {64, NTILE, 1};
+    const uint32_t kbox[3] = {64, 32, KCH};
     const uint64_t vd[4] = {64, pool_rows, 4, 2}, vs[3] = {rb, 128, 512};
-    const uint32_t vbox[4] = {64, 32, 2, 2};
+    const uint32_t vbox[4] = {64, NTILE, 2, 2};
     const uint64_t qd[3] = {64, (uint64_t)B * HQ, KCH}, qs[2] = {DQK * 2, 128};
     const uint32_t qbox[3] = {64, HPC, KCH};
     if (!make_map(&k_map, kv_pool, 3, kd, ks, kbox) || !make_map(&v_map, kv_pool, 4, vd, vs, vbox))
