@@ -211,29 +211,32 @@ __device__ __forceinline__ void drain_stage(uint64_t *full, int u0, int u1, int 
     (void)mbar_wait(full, (uint32_t)(u >> 1) & 1u, WAIT_NS);
 }
 
-// grid (stage_tiles, B), 256 threads: staging slot g of sequence b receives the 64 rows of
-// the gathered tile staged there (rows past the row set, or without a slot, as zeros).
-// Each thread keeps its 18 loads of 16 bytes in flight before storing.
-__global__ void __launch_bounds__(256) stage_kernel(const Params p, uint8_t *__restrict__ stage) {
-    constexpr int PIECES = DQK * 2 / 16;                  // 72 pieces of 16 bytes per row
-    constexpr int PER_THREAD = NTILE * PIECES / 256;      // 18
-    __shared__ int64_t rows[NTILE];
-    const int g = blockIdx.x, b = blockIdx.y;
+// grid (4 * stage_tiles, B), 128 threads: CTA (4 g + q, b) copies rows 16 q .. 16 q + 15
+// of the gathered tile staged in slot g of sequence b (rows past the row set, or
+// without a slot, as zeros).  Each thread keeps its 9 loads of 16 bytes in flight
+// before storing; a unit over four CTAs keeps four times the copies in flight of
+// one CTA per unit.
+constexpr int STAGE_ROWS = 16, STAGE_THREADS = 128;
+__global__ void __launch_bounds__(STAGE_THREADS) stage_kernel(const Params p, uint8_t *__restrict__ stage) {
+    constexpr int PIECES = DQK * 2 / 16;                              // 72 pieces of 16 bytes per row
+    constexpr int PER_THREAD = STAGE_ROWS * PIECES / STAGE_THREADS;   // 9
+    __shared__ int64_t rows[STAGE_ROWS];
+    const int g = blockIdx.x >> 2, r0 = STAGE_ROWS * (blockIdx.x & 3), b = blockIdx.y;
     const SeqTiles st(p, b);
     const int t = st.staged_tile(g);
     if (t < 0) return;
-    if (threadIdx.x < NTILE) rows[threadIdx.x] = st.row(p, b, t, threadIdx.x);
+    if (threadIdx.x < STAGE_ROWS) rows[threadIdx.x] = st.row(p, b, t, r0 + threadIdx.x);
     __syncthreads();
     uint4 v[PER_THREAD];
 #pragma unroll
     for (int i = 0; i < PER_THREAD; ++i) {
-        const int q = threadIdx.x + 256 * i, r = q / PIECES, w = q - r * PIECES;
+        const int q = threadIdx.x + STAGE_THREADS * i, r = q / PIECES, w = q - r * PIECES;
         const int64_t pr = rows[r];
         v[i] = pr >= 0 ? __ldg(reinterpret_cast<const uint4 *>(p.pool + pr * p.row_bytes) + w) : make_uint4(0, 0, 0, 0);
     }
-    uint4 *dst = reinterpret_cast<uint4 *>(stage + ((size_t)b * p.stage_tiles + g) * NTILE * (DQK * 2));
+    uint4 *dst = reinterpret_cast<uint4 *>(stage + (((size_t)b * p.stage_tiles + g) * NTILE + r0) * (DQK * 2));
 #pragma unroll
-    for (int i = 0; i < PER_THREAD; ++i) dst[threadIdx.x + 256 * i] = v[i];
+    for (int i = 0; i < PER_THREAD; ++i) dst[threadIdx.x + STAGE_THREADS * i] = v[i];
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
@@ -653,7 +656,7 @@ int launch(const uint16_t *q, const uint16_t *kv_pool, int64_t k_stride, int64_t
     prm.stage_tiles = G;
     prm.scale_log2 = scale * 1.4426950408889634f;
     prm.stall = take_test_stall(LSA_TEST_STALL_ATTENTION);
-    stage_kernel<<<dim3(G, B), 256, 0, stream>>>(prm, stage);
+    stage_kernel<<<dim3(4 * G, B), STAGE_THREADS, 0, stream>>>(prm, stage);
     int rc = check_launch("stage_kernel");
     if (rc) return rc;
     const size_t smem = smem_bytes();
