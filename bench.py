@@ -47,7 +47,39 @@ def parse():
     p.add_argument("--profile-window", action="store_true",
                    help="no timing: run two eager windows of the workload's kernels on 24K-token contexts "
                         "(pools of ~230 MB) for a profiler capture, then exit")
+    p.add_argument("--profile-extras", action="store_true",
+                   help="no timing: run the label vote, the query encoder, the random baseline selector and "
+                        "two windows of the 512K cold pipeline once each, for profiler captures, then exit")
     return p.parse_args()
+
+
+def profile_extras(args):
+    """One run each of the kernels outside the resident decode step, at the workloads' sizes:
+    label vote (label_vote_128k_l32), query encoder (128K workload), random selector (128K
+    window starts), and two windows of the 512K cold pipeline (gate, plan, fetch, steps)."""
+    import lsa_workloads as W
+    from lsa_workloads.device import bf16, host_build, upload
+    from learned_sparse_kv_b200 import lsa
+    from learned_sparse_kv_b200.decode import Shapes, Window
+    dev = torch.device("cuda:0")
+    p = W.LABEL_VOTE
+    d = W.label_vote_scores(p["layers"], p["steps"], p["chunks"], p["planted"], p["seed"])
+    lsa.label_vote(torch.from_numpy(d["scores"]).to(dev), p["top_p"], p["min_layers"], 0)
+    wl = W.workload(DEFAULT_WORKLOAD)
+    e = W.encoder_inputs(wl)
+    lsa.query_encoder(*(bf16(e[k], dev) for k in ("h", "w_down", "w_up", "w_head")), wl.Hn, wl.dn)
+    ws = torch.tensor([L - wl.window for L in wl.ctx], dtype=torch.int32, device=dev)
+    lsa.select_baseline(lsa.SELECT_RANDOM, ws, max(wl.n_ch), max(wl.n_ch), seed=3)
+    cw = W.workload(COLD_WORKLOAD)
+    host = host_build(cw, windows=2)
+    shapes, t, max_ch, kept_cap, cold = upload(host, dev)
+    win = Window(Shapes(**shapes), t, max_ch, kept_cap, cold)
+    win.run(use_graph=False)
+    torch.cuda.synchronize()
+    status = win.device_status()
+    print(json.dumps({"profile_extras": True, "status": status, "fetched": win.fetch_log.cpu().tolist()}))
+    if status != 0:
+        raise SystemExit(1)
 
 
 def profile_window(args):
@@ -685,6 +717,9 @@ def main():
     args = parse()
     if args.profile_window:
         profile_window(args)
+        return
+    if args.profile_extras:
+        profile_extras(args)
         return
     world, rank, local = dist_setup(args)
     try:
