@@ -15,7 +15,10 @@
 namespace lsa {
 
 constexpr int kTopkThreads = 512;   // threads per CTA
-constexpr int kTopkCtas = 8;        // CTAs per sequence: one thread-block cluster (8 measured fastest of 1..16)
+// CTAs per sequence: one thread-block cluster.  8 measured fastest of 1..16 for 8 sequences of
+// ~16K candidates; a single sequence (a batch of one) takes 16, so that twice the multiprocessors
+// share its candidates.
+constexpr int kTopkCtas = 8, kTopkCtasOne = 16;
 
 int launch_li_scores(const uint16_t *, const uint16_t *, const uint16_t *, int64_t, const int32_t *, int,
                      const int32_t *, const int32_t *, int, const int32_t *, int32_t *, int, int, int, float *,
@@ -76,15 +79,15 @@ struct TopkShared {
     int remaining;
 };
 
-// Top-k of the n scores of one sequence by the kTopkCtas CTAs of a cluster.
+// Top-k of the n scores of one sequence by the NC CTAs of a cluster.
 // CTA c takes the contiguous slice [c seg, (c + 1) seg) and stages its keys in
 // shared memory when they fit (stage_cap keys).  Each 8-bit radix pass counts
-// digits locally; after a cluster barrier every CTA sums the kTopkCtas
+// digits locally; after a cluster barrier every CTA sums the NC
 // histograms through distributed shared memory and picks the same digit, so
 // no result has to be broadcast.  The emission is ordered: a CTA's output
 // offset is the number of selected keys in the lower slices, and ties at the
 // threshold go to the lowest candidate indices.
-template <class PosFn>
+template <int NC, class PosFn>
 __device__ void topk_cluster(const float *__restrict__ s, int n, int k, PosFn pos, int32_t *__restrict__ out,
                              int32_t *__restrict__ out_count, int stage_cap) {
     __shared__ TopkShared sh;
@@ -93,11 +96,11 @@ __device__ void topk_cluster(const float *__restrict__ s, int n, int k, PosFn po
     const int c = (int)sm100::cluster_rank();
 
     if (n <= k) {  // everything is selected, already in ascending order
-        for (int j = c * kTopkThreads + t; j < k; j += kTopkCtas * kTopkThreads) out[j] = j < n ? pos(j) : -1;
+        for (int j = c * kTopkThreads + t; j < k; j += NC * kTopkThreads) out[j] = j < n ? pos(j) : -1;
         if (c == 0 && t == 0) *out_count = n;
         return;
     }
-    const int seg = (n + kTopkCtas - 1) / kTopkCtas;
+    const int seg = (n + NC - 1) / NC;
     const int j0 = min(n, c * seg), len = min(n, j0 + seg) - j0;
     const bool staged = len <= stage_cap;
     if (staged)
@@ -123,7 +126,7 @@ __device__ void topk_cluster(const float *__restrict__ s, int n, int k, PosFn po
         sm100::cluster_sync();   // every CTA's histogram of this pass is complete
         int v = 0;               // suffix counts over digits, highest digit first
         if (t < 256) {
-            for (int r = 0; r < kTopkCtas; ++r) v += ld_cluster_s32(&hist[255 - t], (uint32_t)r);
+            for (int r = 0; r < NC; ++r) v += ld_cluster_s32(&hist[255 - t], (uint32_t)r);
             // The other buffer serves the next pass: every CTA finished reading it
             // (in the previous pass) before the cluster barrier above.  Pass 1 finds
             // it zero from the start.
@@ -194,6 +197,7 @@ __device__ void topk_cluster(const float *__restrict__ s, int n, int k, PosFn po
     sm100::cluster_sync();   // no CTA leaves while another may still read its counts
 }
 
+template <int NC>
 __global__ void __launch_bounds__(kTopkThreads) topk_kept_kernel(const float *__restrict__ scores, int kept_cap,
                                                                  const int32_t *__restrict__ kept_idx,
                                                                  const int32_t *__restrict__ cold, int k,
@@ -202,10 +206,11 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kept_kernel(const float *__
     const int b = blockIdx.y;
     const int32_t *kept = kept_idx + (size_t)b * kept_cap;
     const int n = min(max(cold[b], 0), kept_cap) * LSA_CHUNK;
-    topk_cluster(scores + (size_t)b * kept_cap * LSA_CHUNK, n, k, CandFromKept{kept}, topk_idx + (size_t)b * k,
+    topk_cluster<NC>(scores + (size_t)b * kept_cap * LSA_CHUNK, n, k, CandFromKept{kept}, topk_idx + (size_t)b * k,
                  topk_count + b, stage_cap);
 }
 
+template <int NC>
 __global__ void __launch_bounds__(kTopkThreads) topk_scores_kernel(const float *__restrict__ scores,
                                                                    const int64_t *__restrict__ off, int max_cand,
                                                                    int k, int32_t *__restrict__ topk_idx,
@@ -213,7 +218,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_scores_kernel(const float *
     const int b = blockIdx.y;
     const int64_t a = off[b];
     const int n = (int)max((int64_t)0, min(off[b + 1] - a, (int64_t)max_cand));
-    topk_cluster(scores + a, n, k, CandIdentity{}, topk_idx + (size_t)b * k, topk_count + b, stage_cap);
+    topk_cluster<NC>(scores + a, n, k, CandIdentity{}, topk_idx + (size_t)b * k, topk_count + b, stage_cap);
 }
 
 // ------------------------------------------------------- baseline selectors --
@@ -254,6 +259,7 @@ __global__ void __launch_bounds__(256) random_score_kernel(const int32_t *__rest
 
 // One cluster per sequence: the m = round(n_old * num / den) chunks with the largest
 // scores, ascending, then -1 up to kept_cap.
+template <int NC>
 __global__ void __launch_bounds__(kTopkThreads) random_select_kernel(const float *__restrict__ scores,
                                                                      const int32_t *__restrict__ window_start,
                                                                      int max_old, int num, int den,
@@ -265,32 +271,33 @@ __global__ void __launch_bounds__(kTopkThreads) random_select_kernel(const float
     const int m = (int)min(((int64_t)n_old * num + den / 2) / den, (int64_t)n_old);   // <= kept_cap (host check)
     int32_t *out = kept_idx + (size_t)b * kept_cap;
     const int c = (int)sm100::cluster_rank();
-    for (int j = m + c * kTopkThreads + (int)threadIdx.x; j < kept_cap; j += kTopkCtas * kTopkThreads) out[j] = -1;
+    for (int j = m + c * kTopkThreads + (int)threadIdx.x; j < kept_cap; j += NC * kTopkThreads) out[j] = -1;
     if (m == 0) {
         if (c == 0 && threadIdx.x == 0) kept_count[b] = 0;
         return;
     }
-    topk_cluster(scores + (size_t)b * max_old, n_old, m, CandIdentity{}, out, kept_count + b, stage_cap);
+    topk_cluster<NC>(scores + (size_t)b * max_old, n_old, m, CandIdentity{}, out, kept_count + b, stage_cap);
 }
 
 // Keys staged per CTA: a slice of at most ceil(max_n / 8), never more than 24,576 (96 KB).
-static int stage_capacity(int max_n) { return max(0, min((max_n + kTopkCtas - 1) / kTopkCtas, 24576)); }
+static int cluster_ctas(int B) { return B == 1 ? kTopkCtasOne : kTopkCtas; }
+static int stage_capacity(int max_n, int nc) { return max(0, min((max_n + nc - 1) / nc, 24576)); }
 
-// One cluster of kTopkCtas CTAs per sequence.
+// One cluster of nc CTAs per sequence.
 template <class... Args>
-static int launch_topk(void (*kernel)(Args...), int B, int stage_cap, cudaStream_t stream, const char *what,
+static int launch_topk(void (*kernel)(Args...), int nc, int B, int stage_cap, cudaStream_t stream, const char *what,
                        Args... args) {
     const size_t smem = (size_t)stage_cap * sizeof(uint32_t);
     LSA_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     LSA_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(kTopkCtas, B, 1);
+    cfg.gridDim = dim3(nc, B, 1);
     cfg.blockDim = dim3(kTopkThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kTopkCtas;
+    attr[0].val.clusterDim.x = nc;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
@@ -341,9 +348,13 @@ extern "C" int lsa_topk(const lsa_bf16 *q_li, const lsa_bf16 *w_li, const lsa_bf
     rc = launch_li_scores(q_li, w_li, li_pool, n_slots, chunk_table, table_stride, kept_idx, kept_count, kept_cap,
                           window_start, cold, B, Hl, dl, buf, dev_status, stream);
     if (rc) return rc;
-    const int cap = stage_capacity(kept_cap * LSA_CHUNK);
-    return launch_topk(topk_kept_kernel, B, cap, stream, "topk_kept_kernel", (const float *)buf, kept_cap,
-                       kept_idx, (const int32_t *)cold, k, topk_idx, topk_count, cap);
+    const int nc = cluster_ctas(B), cap = stage_capacity(kept_cap * LSA_CHUNK, nc);
+    if (nc == kTopkCtasOne)
+        return launch_topk(topk_kept_kernel<kTopkCtasOne>, nc, B, cap, stream, "topk_kept_kernel",
+                           (const float *)buf, kept_cap, kept_idx, (const int32_t *)cold, k, topk_idx, topk_count,
+                           cap);
+    return launch_topk(topk_kept_kernel<kTopkCtas>, nc, B, cap, stream, "topk_kept_kernel", (const float *)buf,
+                       kept_cap, kept_idx, (const int32_t *)cold, k, topk_idx, topk_count, cap);
 }
 
 extern "C" int lsa_topk_kernel_count(int B, int Hl, int dl) {
@@ -359,9 +370,12 @@ extern "C" int lsa_topk_from_scores(const float *scores, const int64_t *cand_off
                 "lsa_topk_from_scores: null pointer or B <= 0");
     LSA_REQUIRE(max_cand >= 0, LSA_ERR_INVALID_ARG, "lsa_topk_from_scores: max_cand must be >= 0");
     LSA_REQUIRE(k >= 1 && k <= 65536, LSA_ERR_INVALID_ARG, "lsa_topk_from_scores: k=%d outside [1, 65536]", k);
-    const int cap = stage_capacity(max_cand);
-    return launch_topk(topk_scores_kernel, B, cap, stream, "topk_scores_kernel", scores, cand_offset, max_cand, k,
-                       topk_idx, topk_count, cap);
+    const int nc = cluster_ctas(B), cap = stage_capacity(max_cand, nc);
+    if (nc == kTopkCtasOne)
+        return launch_topk(topk_scores_kernel<kTopkCtasOne>, nc, B, cap, stream, "topk_scores_kernel", scores,
+                           cand_offset, max_cand, k, topk_idx, topk_count, cap);
+    return launch_topk(topk_scores_kernel<kTopkCtas>, nc, B, cap, stream, "topk_scores_kernel", scores, cand_offset,
+                       max_cand, k, topk_idx, topk_count, cap);
 }
 
 extern "C" size_t lsa_select_baseline_workspace_size(int B, int max_old_chunks) {
@@ -401,8 +415,12 @@ extern "C" int lsa_select_baseline(int mode, const int32_t *window_start, int B,
         int rc = check_launch("random_score_kernel");
         if (rc) return rc;
     }
-    const int cap = stage_capacity(max_old_chunks);
-    return launch_topk(random_select_kernel, B, cap, stream, "random_select_kernel", (const float *)scores,
-                       window_start, max_old_chunks, keep_num, keep_den, kept_idx, kept_count, kept_cap, dev_status,
-                       cap);
+    const int nc = cluster_ctas(B), cap = stage_capacity(max_old_chunks, nc);
+    if (nc == kTopkCtasOne)
+        return launch_topk(random_select_kernel<kTopkCtasOne>, nc, B, cap, stream, "random_select_kernel",
+                           (const float *)scores, window_start, max_old_chunks, keep_num, keep_den, kept_idx,
+                           kept_count, kept_cap, dev_status, cap);
+    return launch_topk(random_select_kernel<kTopkCtas>, nc, B, cap, stream, "random_select_kernel",
+                       (const float *)scores, window_start, max_old_chunks, keep_num, keep_den, kept_idx, kept_count,
+                       kept_cap, dev_status, cap);
 }

@@ -190,6 +190,13 @@ def test_select_baseline_random_and_recent_exact(L, seed):
             assert np.all(kept[b, cnt[b]:] == -1)
     kept, cnt = L.select_baseline(L.SELECT_RECENT, ws, max_old, 16)
     assert int(cnt.abs().sum()) == 0 and bool((kept == -1).all())
+    # a single sequence (the top-k runs on a larger cluster for a batch of one)
+    one = starts[1:2]
+    m1 = int(one[0]) // CH
+    kept, cnt = L.select_baseline(L.SELECT_RANDOM, i32(one, d), m1, (m1 + 5) // 10, seed=seed)
+    ref, _, rcnt = oracle.select_baseline(oracle.RANDOM, one, seed=seed, kept_cap=(m1 + 5) // 10)
+    assert int(cnt[0]) == rcnt[0]
+    np.testing.assert_array_equal(kept[0, :rcnt[0]].cpu().numpy(), ref[0])
 
 
 def test_select_baseline_rejects_a_too_small_capacity(L):
