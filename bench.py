@@ -270,6 +270,25 @@ def recorded_traffic(*kernel_files):
 
 # ------------------------------------------------------- attention timing --
 
+STEP_KEYS = ("q_li", "w_li", "new_li", "new_kv", "new_k", "new_v")
+
+
+def append_topk(win, src, s):
+    """One step's append and top-k (one fused call with the latent layout) from src's step tensors."""
+    from learned_sparse_kv_b200 import lsa
+    t, sh = win.t, win.s
+    if sh.latent:
+        lsa.append_topk(src["new_kv"], src["new_li"], win.k_pool, win.window_len, src["q_li"], src["w_li"], t["li"],
+                        t["chunk_table"], win.kept_idx, win.kept_count, t["window_start"], sh.k, scores=win.scores,
+                        status=win.status, topk_idx=win.topk_idx[s], topk_count=win.topk_count[s], ws=win.ws_topk)
+        return
+    lsa.append_token(src["new_k"], src["new_v"], src["new_li"], win.k_pool, win.v_pool, t["li"], t["chunk_table"],
+                     t["window_start"], win.window_len, status=win.status)
+    lsa.topk(src["q_li"], src["w_li"], t["li"], t["chunk_table"], win.kept_idx, win.kept_count, t["window_start"],
+             sh.k, scores=win.scores, status=win.status, topk_idx=win.topk_idx[s], topk_count=win.topk_count[s],
+             ws=win.ws_topk)
+
+
 def time_attention_kernels(win, windows):
     """Average device time of the attention launch, from external event nodes in a graph.
 
@@ -299,12 +318,7 @@ def time_attention_kernels(win, windows):
         if win.cold is None:
             win.select()
         for s in range(S):
-            lsa.append_token(t["new_kv"][s] if sh.latent else t["new_k"][s], None if sh.latent else t["new_v"][s],
-                             t["new_li"][s], win.k_pool, win.v_pool, t["li"], t["chunk_table"], t["window_start"],
-                             win.window_len, status=win.status)
-            lsa.topk(t["q_li"][s], t["w_li"][s], t["li"], t["chunk_table"], win.kept_idx, win.kept_count,
-                     t["window_start"], sh.k, scores=win.scores, status=win.status, topk_idx=win.topk_idx[s],
-                     topk_count=win.topk_count[s], ws=win.ws_topk)
+            append_topk(win, {k: t[k][s] for k in STEP_KEYS if k in t}, s)
             rec(evs[s][0])
             lsa.sparse_decode(t["q"][s], win.k_pool, win.v_pool, t["chunk_table"], win.topk_idx[s],
                               win.topk_count[s], t["window_start"], win.window_len, win.max_window_len, sh.dv,
@@ -538,12 +552,7 @@ def run_e2e(win, wl, args, world):
         d = dev_in[s % 2]
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            lsa.append_token(d["new_kv"] if sh.latent else d["new_k"], None if sh.latent else d["new_v"],
-                             d["new_li"], win.k_pool, win.v_pool, t["li"], t["chunk_table"], t["window_start"],
-                             win.window_len, status=win.status)
-            lsa.topk(d["q_li"], d["w_li"], t["li"], t["chunk_table"], win.kept_idx, win.kept_count,
-                     t["window_start"], sh.k, scores=win.scores, status=win.status, topk_idx=win.topk_idx[s],
-                     topk_count=win.topk_count[s], ws=win.ws_topk)
+            append_topk(win, d, s)
             lsa.sparse_decode(d["q"], win.k_pool, win.v_pool, t["chunk_table"], win.topk_idx[s],
                               win.topk_count[s], t["window_start"], win.window_len, win.max_window_len, sh.dv,
                               sh.scale, out=win.out[s], lse=win.lse[s], status=win.status, ws=win.ws_decode)

@@ -232,6 +232,25 @@ size_t lsa_topk_workspace_size(int B, int kept_cap);
 int lsa_topk_kernel_count(int B, int Hl, int dl);
 
 /*
+ * a5 + a2 + a3 in one call: the append of the decoded token (lsa_append_token,
+ * latent layout: one KV row of kv_width in kv_pool and one indexer key in
+ * li_pool per sequence), then the indexer scoring and top-k (lsa_topk).
+ * Passage: as lsa_append_token and lsa_topk.
+ * Where the tcgen05 indexer serves the shape (lsa_topk_kernel_count == 2) the
+ * append is done by the indexer launch itself -- that kernel reads neither the
+ * window's rows nor window_len -- so the step has one launch less; other shapes
+ * launch the append first.  Arguments, alignment rules and results are those
+ * of the two calls (kv_row_stride and kv_width as k_row_stride and k_width).
+ */
+int lsa_append_topk(const lsa_bf16 *new_kv, const lsa_bf16 *new_li, lsa_bf16 *kv_pool, int64_t kv_row_stride,
+                    int kv_width, int32_t *window_len, const lsa_bf16 *q_li, const lsa_bf16 *w_li,
+                    lsa_bf16 *li_pool, int64_t n_slots, const int32_t *chunk_table, int table_stride,
+                    const int32_t *kept_idx, const int32_t *kept_count, int kept_cap,
+                    const int32_t *window_start, int B, int Hl, int dl, int k,
+                    int32_t *topk_idx, int32_t *topk_count, float *scores, int32_t *dev_status,
+                    void *ws, size_t ws_bytes, lsa_stream_t stream);
+
+/*
  * a3 alone, on given fp32 scores (exact unit entry point).
  * Sequence b owns scores[cand_offset[b] .. cand_offset[b+1]); writes the
  * indices (relative to cand_offset[b]) of its min(k, n_b) largest scores,
@@ -299,8 +318,12 @@ int lsa_merge_attention(const float *o_parts, const float *lse_parts, int R, int
  *
  * For each sequence b the token at position p = window_start[b] + window_len[b]
  * gets new_k[b] (and new_v[b], new_li[b]) written into its pool row, then
- * window_len[b] is incremented.  The chunk of p must already have a slot.
+ * window_len[b] is incremented.  The chunk of p must already have a slot; a
+ * chunk without one sets LSA_DEV_TABLE in dev_status and leaves that sequence
+ * unchanged.
  *   new_k [B, k_width], new_v [B, v_width] or NULL, new_li [B, dl] or NULL (device)
+ * Widths and row strides are multiples of 8 elements and every base pointer is
+ * 16-byte aligned (rows move as 16-byte vectors), else LSA_ERR_INVALID_ARG.
  */
 int lsa_append_token(const lsa_bf16 *new_k, const lsa_bf16 *new_v, const lsa_bf16 *new_li,
                      lsa_bf16 *k_pool, int64_t k_row_stride, int k_width,

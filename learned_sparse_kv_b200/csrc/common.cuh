@@ -18,6 +18,16 @@ void set_error(const char *fmt, ...);
 int fail(int code, const char *fmt, ...);
 int check_launch(const char *what);  // returns LSA_ERR_CUDA and records the message on error
 int sm_count();                      // multiprocessor count of the current device (cached per device)
+// The decoded token's rows, appended by the indexer launch of lsa_append_topk (latent
+// layout: one KV row and one indexer key per sequence).
+struct AppendArgs {
+    const uint16_t *new_kv, *new_li;
+    uint16_t *kv_pool, *li_pool;
+    int64_t kv_stride;
+    int kv_width;
+    int32_t *window_len;
+};
+
 // Failure-path test switch (lsa_test_stall_next_wait): true once for the next
 // launch of the named kernel after the switch was set.
 int take_test_stall(int which);

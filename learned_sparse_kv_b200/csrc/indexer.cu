@@ -242,21 +242,23 @@ bool shape_ok(int H, int D, int B);
 int launch(const uint16_t *q_li, const uint16_t *w_li, const uint16_t *li_pool, int64_t n_slots, const int32_t *table,
            int table_stride, const int32_t *kept_idx, const int32_t *kept_count, int kept_cap,
            const int32_t *window_start, int32_t *cold, int B, int H, int D, float *scores, int32_t *status,
-           cudaStream_t stream);
+           cudaStream_t stream, const AppendArgs *app);
 }  // namespace li2
 
 // True when the indexer kernel for this shape counts the kept cold chunks itself
 // (the tcgen05 kernel does, in its prologue); otherwise they are counted first.
 bool indexer_counts_cold(int H, int D, int B) { return li2::shape_ok(H, D, B); }
 
+// app (optional, tcgen05 shapes only): the decoded token's rows, appended by the same launch.
 int launch_li_scores(const uint16_t *q_li, const uint16_t *w_li, const uint16_t *li_pool, int64_t n_slots,
                      const int32_t *table, int table_stride, const int32_t *kept_idx, const int32_t *kept_count,
                      int kept_cap, const int32_t *window_start, int32_t *cold, int B, int H, int D,
-                     float *scores, int32_t *status, cudaStream_t stream) {
+                     float *scores, int32_t *status, cudaStream_t stream, const AppendArgs *app) {
     // Head counts of 32, 64 or 128 run on tcgen05 (M = 128 tokens, N = heads); others on mma.sync.
     if (li2::shape_ok(H, D, B))
         return li2::launch(q_li, w_li, li_pool, n_slots, table, table_stride, kept_idx, kept_count, kept_cap,
-                           window_start, cold, B, H, D, scores, status, stream);
+                           window_start, cold, B, H, D, scores, status, stream, app);
+    if (app) return fail(LSA_ERR_SHAPE, "append with the indexer: only the tcgen05 indexer shapes");
     const size_t smem = sizeof(IdxSmem);
     int per_seq = (sm_count() * 8 + B - 1) / B;
     per_seq = max(1, min(per_seq, kept_cap));

@@ -59,7 +59,40 @@ struct Params {
     int64_t n_slots;
     int B, H, D, table_stride, kept_cap;
     int stall;                    // failure-path test: the first wait waits on a barrier nothing arrives on
+    // optional append of the decoded token (CTA b, b < B, before anything else): its KV row
+    // and indexer key go to position window_start[b] + window_len[b], then window_len[b] += 1
+    const uint16_t *new_kv, *new_li;
+    uint16_t *kv_pool, *li_pool;
+    int64_t kv_stride;
+    int kv_width;
+    int32_t *window_len;
 };
+
+// The append of the decoded token, folded into the indexer launch: this kernel reads neither
+// the window's rows nor window_len, so CTA b can write sequence b's new rows and advance its
+// window; the attention launches that follow read them.
+__device__ void append_token(const Params &p, int b) {
+    __shared__ int64_t s_row;
+    if (threadIdx.x == 0) {
+        const int pos = p.window_start[b] + p.window_len[b];
+        const int chunk = pos / LSA_CHUNK;
+        const int slot = (pos >= 0 && chunk < p.table_stride) ? p.table[(size_t)b * p.table_stride + chunk] : -1;
+        s_row = (slot >= 0 && slot < p.n_slots) ? (int64_t)slot * LSA_CHUNK + pos % LSA_CHUNK : -1;
+        if (s_row < 0) flag(p.status, LSA_DEV_TABLE);
+    }
+    __syncthreads();
+    const int64_t row = s_row;
+    if (row >= 0) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.new_kv + (size_t)b * p.kv_width);
+        uint4 *dst = reinterpret_cast<uint4 *>(p.kv_pool + row * p.kv_stride);
+        for (int c = threadIdx.x; c < p.kv_width / 8; c += blockDim.x) dst[c] = src[c];
+        const uint4 *lsrc = reinterpret_cast<const uint4 *>(p.new_li + (size_t)b * p.D);
+        uint4 *ldst = reinterpret_cast<uint4 *>(p.li_pool + row * p.D);
+        for (int c = threadIdx.x; c < p.D / 8; c += blockDim.x) ldst[c] = lsrc[c];
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && row >= 0) p.window_len[b] += 1;
+}
 
 // 1-CTA MMA and commit
 __device__ __forceinline__ void umma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, bool acc) {
@@ -163,6 +196,7 @@ li_score_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_consta
         sm.abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
+    if (p.new_kv && (int)blockIdx.x < p.B) append_token(p, blockIdx.x);
     count_cold(p, wk, warp, lane);
     if (warp == 1) asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
                                     smem_addr(&sm.tmem_base)), "r"(256));
@@ -375,7 +409,7 @@ bool shape_ok(int H, int D, int B) { return (H == 32 || H == 64 || H == 128) && 
 int launch(const uint16_t *q_li, const uint16_t *w_li, const uint16_t *li_pool, int64_t n_slots, const int32_t *table,
            int table_stride, const int32_t *kept_idx, const int32_t *kept_count, int kept_cap,
            const int32_t *window_start, int32_t *cold, int B, int H, int D, float *scores, int32_t *status,
-           cudaStream_t stream) {
+           cudaStream_t stream, const AppendArgs *app) {
     CUtensorMap key_map, q_map;
     if (!make_map(&key_map, li_pool, D, (uint64_t)n_slots * LSA_CHUNK, LSA_CHUNK))
         return fail(LSA_ERR_CUDA, "lsa_topk: cuTensorMapEncodeTiled failed for the indexer key pool");
@@ -386,6 +420,13 @@ int launch(const uint16_t *q_li, const uint16_t *w_li, const uint16_t *li_pool, 
     prm.window_start = window_start; prm.cold = cold; prm.scores = scores; prm.status = status; prm.n_slots = n_slots;
     prm.B = B; prm.H = H; prm.D = D; prm.table_stride = table_stride; prm.kept_cap = kept_cap;
     prm.stall = take_test_stall(LSA_TEST_STALL_INDEXER);
+    prm.new_kv = app ? app->new_kv : nullptr;
+    prm.new_li = app ? app->new_li : nullptr;
+    prm.kv_pool = app ? app->kv_pool : nullptr;
+    prm.li_pool = app ? app->li_pool : nullptr;
+    prm.kv_stride = app ? app->kv_stride : 0;
+    prm.kv_width = app ? app->kv_width : 0;
+    prm.window_len = app ? app->window_len : nullptr;
     const size_t smem = sizeof(Smem) + 1024;
     LSA_CUDA(cudaFuncSetAttribute(li_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     li_score_kernel<<<sm_count(), THREADS, smem, stream>>>(key_map, q_map, prm);

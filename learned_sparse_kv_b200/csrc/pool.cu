@@ -205,6 +205,9 @@ extern "C" int lsa_append_token(const lsa_bf16 *new_k, const lsa_bf16 *new_v, co
                 LSA_ERR_INVALID_ARG, "lsa_append_token: v width/stride must be positive multiples of 8");
     LSA_REQUIRE(!li_pool || (new_li && dl > 0 && dl % 8 == 0), LSA_ERR_INVALID_ARG,
                 "lsa_append_token: indexer key width must be a positive multiple of 8");
+    auto al16 = [](const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; };
+    LSA_REQUIRE(al16(new_k) && al16(k_pool) && al16(new_v) && al16(v_pool) && al16(new_li) && al16(li_pool),
+                LSA_ERR_INVALID_ARG, "lsa_append_token: rows are copied in 16-byte vectors: 16-byte aligned bases");
     append_kernel<<<B, 128, 0, stream>>>(new_k, new_v, new_li, k_pool, k_row_stride, k_width, v_pool, v_row_stride,
                                          v_width, li_pool, dl, n_slots, chunk_table, table_stride, window_start,
                                          window_len, dev_status);

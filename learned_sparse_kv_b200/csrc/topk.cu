@@ -22,7 +22,7 @@ constexpr int kTopkCtas = 8, kTopkCtasOne = 16;
 
 int launch_li_scores(const uint16_t *, const uint16_t *, const uint16_t *, int64_t, const int32_t *, int,
                      const int32_t *, const int32_t *, int, const int32_t *, int32_t *, int, int, int, float *,
-                     int32_t *, cudaStream_t);
+                     int32_t *, cudaStream_t, const AppendArgs *);
 bool indexer_shape_ok(int H, int D);
 bool indexer_counts_cold(int H, int D, int B);
 
@@ -318,11 +318,11 @@ extern "C" size_t lsa_topk_workspace_size(int B, int kept_cap) {
     return align_up(c.used, 256);
 }
 
-extern "C" int lsa_topk(const lsa_bf16 *q_li, const lsa_bf16 *w_li, const lsa_bf16 *li_pool, int64_t n_slots,
-                        const int32_t *chunk_table, int table_stride, const int32_t *kept_idx,
-                        const int32_t *kept_count, int kept_cap, const int32_t *window_start, int B, int Hl, int dl,
-                        int k, int32_t *topk_idx, int32_t *topk_count, float *scores, int32_t *dev_status, void *ws,
-                        size_t ws_bytes, lsa_stream_t stream) {
+static int topk_impl(const lsa_bf16 *q_li, const lsa_bf16 *w_li, const lsa_bf16 *li_pool, int64_t n_slots,
+                     const int32_t *chunk_table, int table_stride, const int32_t *kept_idx,
+                     const int32_t *kept_count, int kept_cap, const int32_t *window_start, int B, int Hl, int dl,
+                     int k, int32_t *topk_idx, int32_t *topk_count, float *scores, int32_t *dev_status, void *ws,
+                     size_t ws_bytes, lsa_stream_t stream, const AppendArgs *app) {
     LSA_REQUIRE(B > 0 && kept_cap > 0 && table_stride > 0 && n_slots > 0, LSA_ERR_INVALID_ARG,
                 "lsa_topk: bad sizes (B=%d kept_cap=%d table_stride=%d n_slots=%lld)", B, kept_cap, table_stride,
                 (long long)n_slots);
@@ -346,7 +346,7 @@ extern "C" int lsa_topk(const lsa_bf16 *q_li, const lsa_bf16 *w_li, const lsa_bf
         if (rc) return rc;
     }
     rc = launch_li_scores(q_li, w_li, li_pool, n_slots, chunk_table, table_stride, kept_idx, kept_count, kept_cap,
-                          window_start, cold, B, Hl, dl, buf, dev_status, stream);
+                          window_start, cold, B, Hl, dl, buf, dev_status, stream, app);
     if (rc) return rc;
     const int nc = cluster_ctas(B), cap = stage_capacity(kept_cap * LSA_CHUNK, nc);
     if (nc == kTopkCtasOne)
@@ -355,6 +355,44 @@ extern "C" int lsa_topk(const lsa_bf16 *q_li, const lsa_bf16 *w_li, const lsa_bf
                            cap);
     return launch_topk(topk_kept_kernel<kTopkCtas>, nc, B, cap, stream, "topk_kept_kernel", (const float *)buf,
                        kept_cap, kept_idx, (const int32_t *)cold, k, topk_idx, topk_count, cap);
+}
+
+extern "C" int lsa_topk(const lsa_bf16 *q_li, const lsa_bf16 *w_li, const lsa_bf16 *li_pool, int64_t n_slots,
+                        const int32_t *chunk_table, int table_stride, const int32_t *kept_idx,
+                        const int32_t *kept_count, int kept_cap, const int32_t *window_start, int B, int Hl, int dl,
+                        int k, int32_t *topk_idx, int32_t *topk_count, float *scores, int32_t *dev_status, void *ws,
+                        size_t ws_bytes, lsa_stream_t stream) {
+    return topk_impl(q_li, w_li, li_pool, n_slots, chunk_table, table_stride, kept_idx, kept_count, kept_cap,
+                     window_start, B, Hl, dl, k, topk_idx, topk_count, scores, dev_status, ws, ws_bytes, stream,
+                     nullptr);
+}
+
+extern "C" int lsa_append_topk(const lsa_bf16 *new_kv, const lsa_bf16 *new_li, lsa_bf16 *kv_pool,
+                               int64_t kv_row_stride, int kv_width, int32_t *window_len, const lsa_bf16 *q_li,
+                               const lsa_bf16 *w_li, lsa_bf16 *li_pool, int64_t n_slots, const int32_t *chunk_table,
+                               int table_stride, const int32_t *kept_idx, const int32_t *kept_count, int kept_cap,
+                               const int32_t *window_start, int B, int Hl, int dl, int k, int32_t *topk_idx,
+                               int32_t *topk_count, float *scores, int32_t *dev_status, void *ws, size_t ws_bytes,
+                               lsa_stream_t stream) {
+    LSA_REQUIRE(new_kv && new_li && kv_pool && window_len && li_pool, LSA_ERR_INVALID_ARG,
+                "lsa_append_topk: null append pointer");
+    LSA_REQUIRE(kv_width > 0 && kv_width % 8 == 0 && kv_row_stride >= kv_width && kv_row_stride % 8 == 0,
+                LSA_ERR_INVALID_ARG, "lsa_append_topk: kv width/stride must be positive multiples of 8");
+    auto al16 = [](const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; };
+    LSA_REQUIRE(al16(new_kv) && al16(new_li) && al16(kv_pool) && al16(li_pool), LSA_ERR_INVALID_ARG,
+                "lsa_append_topk: rows are copied in 16-byte vectors: 16-byte aligned bases");
+    if (!indexer_counts_cold(Hl, dl, B)) {
+        // other indexer shapes: the append is a launch of its own, then the top-k call
+        const int rc = lsa_append_token(new_kv, nullptr, new_li, kv_pool, kv_row_stride, kv_width, nullptr, 0, 0,
+                                        li_pool, dl, n_slots, chunk_table, table_stride, window_start, window_len, B,
+                                        dev_status, stream);
+        if (rc) return rc;
+        return lsa_topk(q_li, w_li, li_pool, n_slots, chunk_table, table_stride, kept_idx, kept_count, kept_cap,
+                        window_start, B, Hl, dl, k, topk_idx, topk_count, scores, dev_status, ws, ws_bytes, stream);
+    }
+    const AppendArgs app = {new_kv, new_li, kv_pool, li_pool, kv_row_stride, kv_width, window_len};
+    return topk_impl(q_li, w_li, li_pool, n_slots, chunk_table, table_stride, kept_idx, kept_count, kept_cap,
+                     window_start, B, Hl, dl, k, topk_idx, topk_count, scores, dev_status, ws, ws_bytes, stream, &app);
 }
 
 extern "C" int lsa_topk_kernel_count(int B, int Hl, int dl) {

@@ -162,12 +162,17 @@ class Window:
         """Decode step s of window w: append, indexer top-k, attention."""
         t, sh = self.t, self.s
         g = w * sh.steps + s
-        lsa.append_token(t["new_kv"][g] if sh.latent else t["new_k"][g], None if sh.latent else t["new_v"][g],
-                         t["new_li"][g], self.k_pool, self.v_pool, t["li"], t["chunk_table"], t["window_start"],
-                         self.window_len, status=self.status)
-        lsa.topk(t["q_li"][g], t["w_li"][g], t["li"], t["chunk_table"], self.kept_idx, self.kept_count,
-                 t["window_start"], sh.k, scores=self.scores, status=self.status, topk_idx=self.topk_w[w, s],
-                 topk_count=self.topk_count_w[w, s], ws=self.ws_topk)
+        if sh.latent:
+            lsa.append_topk(t["new_kv"][g], t["new_li"][g], self.k_pool, self.window_len, t["q_li"][g],
+                            t["w_li"][g], t["li"], t["chunk_table"], self.kept_idx, self.kept_count,
+                            t["window_start"], sh.k, scores=self.scores, status=self.status,
+                            topk_idx=self.topk_w[w, s], topk_count=self.topk_count_w[w, s], ws=self.ws_topk)
+        else:
+            lsa.append_token(t["new_k"][g], t["new_v"][g], t["new_li"][g], self.k_pool, self.v_pool, t["li"],
+                             t["chunk_table"], t["window_start"], self.window_len, status=self.status)
+            lsa.topk(t["q_li"][g], t["w_li"][g], t["li"], t["chunk_table"], self.kept_idx, self.kept_count,
+                     t["window_start"], sh.k, scores=self.scores, status=self.status, topk_idx=self.topk_w[w, s],
+                     topk_count=self.topk_count_w[w, s], ws=self.ws_topk)
         lsa.sparse_decode(t["q"][g], self.k_pool, self.v_pool, t["chunk_table"], self.topk_w[w, s],
                           self.topk_count_w[w, s], t["window_start"], self.window_len, self.max_window_len, sh.dv,
                           sh.scale, out=self.out_w[w, s], lse=self.lse_w[w, s], status=self.status,
@@ -314,12 +319,19 @@ class Window:
 
     def launches_per_window(self) -> int:
         """Kernels this library launches per window of resident pools (select: 2, or 0 for the
-        recency baseline, which only fills memory; per step: append 1, top-k 2 or 3, decode 2 or 3).
+        recency baseline, which only fills memory; per step: append and top-k 2 to 4, decode 2 or 3).
 
         The top-k call counts the kept cold chunks inside the tcgen05 indexer kernel when
-        that kernel serves the indexer shape, else in a kernel of its own."""
+        that kernel serves the indexer shape, else in a kernel of its own; with the latent
+        layout that kernel also appends the decoded token."""
         sel = 0 if (self.selector is not None and self.selector["mode"] == lsa.SELECT_RECENT) else 2
-        return sel + self.s.steps * (1 + lsa.topk_kernel_count(self.s.B, self.s.Hl, self.s.dl) + self._decode_kernels())
+        return sel + self.s.steps * (self._append_topk_kernels() + self._decode_kernels())
+
+    def _append_topk_kernels(self) -> int:
+        sh = self.s
+        if sh.latent:
+            return lsa.append_topk_kernel_count(sh.B, sh.Hl, sh.dl)
+        return 1 + lsa.topk_kernel_count(sh.B, sh.Hl, sh.dl)
 
     def _decode_kernels(self) -> int:
         """Kernels of one attention call: the 128-head latent shape stages its gathered tiles,
@@ -331,7 +343,7 @@ class Window:
         window 0's first step is append, two attention calls, top-k and a merge; the other
         steps as launches_per_window; one window advance per later window."""
         dk = self._decode_kernels()
-        per_step = 1 + lsa.topk_kernel_count(self.s.B, self.s.Hl, self.s.dl) + dk
+        per_step = self._append_topk_kernels() + dk
         first = 1 + dk + lsa.topk_kernel_count(self.s.B, self.s.Hl, self.s.dl) + dk + 1
         sel = 0 if (self.selector is not None and self.selector["mode"] == lsa.SELECT_RECENT) else 2
         return n_windows * (sel + 2) + first + (n_windows * self.s.steps - 1) * per_step + (n_windows - 1)

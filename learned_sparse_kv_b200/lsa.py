@@ -42,6 +42,7 @@ def _load():
         "lsa_select_baseline_workspace_size": ([I, I], SZ),
         "lsa_topk": ([P, P, P, I64, P, I, P, P, I, P, I, I, I, I, P, P, P, P, P, SZ, P], I),
         "lsa_topk_workspace_size": ([I, I], SZ),
+        "lsa_append_topk": ([P, P, P, I64, I, P, P, P, P, I64, P, I, P, P, I, P, I, I, I, I, P, P, P, P, P, SZ, P], I),
         "lsa_topk_kernel_count": ([I, I, I], I),
         "lsa_topk_from_scores": ([P, P, I, I, I, P, P, P, SZ, P], I),
         "lsa_sparse_decode": ([P, P, I64, P, I64, I64, P, I, P, P, I, P, P, I, I, I, I, I, F, P, P, P, P, SZ, P], I),
@@ -249,6 +250,38 @@ def topk(q_li, w_li, li_pool, chunk_table, kept_idx, kept_count, window_start, k
                          B, Hl, dl, k, _ptr(topk_idx), _ptr(topk_count), _ptr(scores), _ptr(status), _ptr(ws),
                          ws.numel(), _stream(stream)))
     return topk_idx, topk_count
+
+
+def append_topk(new_kv, new_li, kv_pool, window_len, q_li, w_li, li_pool, chunk_table, kept_idx, kept_count,
+                window_start, k, *, scores=None, status=None, topk_idx=None, topk_count=None, ws=None,
+                stream=None):
+    """append_token (latent layout: new_kv [B, Kw] into kv_pool [slots, 64, Kw]) then topk, in the
+    indexer's launch where the tcgen05 indexer serves the shape.  Returns (topk_idx, topk_count)."""
+    B, Hl, dl = q_li.shape
+    _dev(new_kv, torch.bfloat16, "new_kv"); _dev(new_li, torch.bfloat16, "new_li")
+    _dev(kv_pool, torch.bfloat16, "kv_pool"); _dev(window_len, torch.int32, "window_len")
+    _dev(q_li, torch.bfloat16, "q_li"); _dev(w_li, torch.bfloat16, "w_li"); _dev(li_pool, torch.bfloat16, "li_pool")
+    _dev(chunk_table, torch.int32, "chunk_table"); _dev(kept_idx, torch.int32, "kept_idx")
+    _dev(kept_count, torch.int32, "kept_count"); _dev(window_start, torch.int32, "window_start")
+    dev = q_li.device
+    kept_cap = kept_idx.shape[1]
+    if topk_idx is None:
+        topk_idx = torch.empty(B, k, dtype=torch.int32, device=dev)
+    if topk_count is None:
+        topk_count = torch.empty(B, dtype=torch.int32, device=dev)
+    ws = _ws(topk_workspace_size(B, kept_cap), dev, ws)
+    _check(_lib.lsa_append_topk(_ptr(new_kv), _ptr(new_li), _ptr(kv_pool), kv_pool.shape[-1], new_kv.shape[1],
+                                _ptr(window_len), _ptr(q_li), _ptr(w_li), _ptr(li_pool), li_pool.shape[0],
+                                _ptr(chunk_table), chunk_table.shape[1], _ptr(kept_idx), _ptr(kept_count), kept_cap,
+                                _ptr(window_start), B, Hl, dl, k, _ptr(topk_idx), _ptr(topk_count), _ptr(scores),
+                                _ptr(status), _ptr(ws), ws.numel(), _stream(stream)))
+    return topk_idx, topk_count
+
+
+def append_topk_kernel_count(B, Hl, dl):
+    """Launches of one append_topk call: the append rides in the tcgen05 indexer launch."""
+    n = topk_kernel_count(B, Hl, dl)
+    return n if n == 2 else n + 1
 
 
 def topk_from_scores(scores, cand_offset, max_cand, k, *, stream=None):

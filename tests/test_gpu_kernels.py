@@ -318,6 +318,63 @@ def test_li_topk_no_cold_candidates(L):
     assert cnt.cpu().tolist() == [0, 0] and bool((idx == -1).all())
 
 
+def test_append_topk_appends_and_selects_like_the_oracle(L):
+    """The fused append + top-k call (latent layout): at every step the top-k equals the
+    oracle's, the decoded token's KV row and indexer key land bit-exact at window_start +
+    window_len, and the window grows by one.  The device rows of the appended tokens start
+    as bf16 NaN, so a missing write shows."""
+    wl = _small_mla(k=700, steps=4)
+    host = host_build(wl)
+    kept, _, _, _ = H.kept_lists(host)
+    H.open_topk_gap(host, kept, [(b, s) for b in range(wl.B) for s in range(wl.steps)])
+    d = dev()
+    kept_t = torch.full((wl.B, host["kept_cap"]), -1, dtype=torch.int32)
+    cnt_t = torch.zeros(wl.B, dtype=torch.int32)
+    for b in range(wl.B):
+        kept_t[b, :kept[b].size] = torch.from_numpy(kept[b])
+        cnt_t[b] = kept[b].size
+    kept_t, cnt_t = kept_t.to(d), cnt_t.to(d)
+    kv, li = bf16(host["pools"]["kv"], d), bf16(host["pools"]["li"], d)
+    table, wstart = i32(host["chunk_table"], d), i32(host["window_start"], d)
+    wlen = torch.full((wl.B,), wl.window, dtype=torch.int32, device=d)
+    status = torch.zeros(1, dtype=torch.int32, device=d)
+    st = host["step"]
+    for s in range(wl.steps):
+        idx, cnt = L.append_topk(bf16(st["new_kv"][s], d), bf16(st["new_li"][s], d), kv, wlen,
+                                 bf16(st["q_li"][s], d), bf16(st["w_li"][s], d), li, table, kept_t, cnt_t, wstart,
+                                 wl.k, status=status)
+        idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+        assert status.item() == 0
+        assert wlen.cpu().tolist() == [wl.window + s + 1] * wl.B
+        for b in range(wl.B):
+            pos, ref_sc = H.li_scores(host, kept[b], b, s)
+            sel = oracle.topk_select(ref_sc, wl.k)
+            assert cnt[b] == sel.size
+            np.testing.assert_array_equal(idx[b, :cnt[b]], pos[sel])
+            p = wl.ctx[b] + s
+            slot = host["chunk_table"][b, p // CH]
+            np.testing.assert_array_equal(kv[slot, p % CH].cpu().view(torch.int16).numpy().view(np.uint16),
+                                          st["new_kv"][s, b])
+            np.testing.assert_array_equal(li[slot, p % CH].cpu().view(torch.int16).numpy().view(np.uint16),
+                                          st["new_li"][s, b])
+    assert L.append_topk_kernel_count(wl.B, wl.Hl, wl.dl) == 2
+
+
+def test_append_topk_rejects_unaligned_rows(L):
+    d = dev()
+    buf = torch.zeros(2 * 576 + 8, dtype=torch.bfloat16, device=d)
+    kv = torch.zeros(4, CH, 576, dtype=torch.bfloat16, device=d)
+    li = torch.zeros(4, CH, 128, dtype=torch.bfloat16, device=d)
+    with pytest.raises(RuntimeError, match="16-byte"):
+        L.append_topk(buf[1:1 + 576].view(1, 576), torch.zeros(1, 128, dtype=torch.bfloat16, device=d), kv,
+                      torch.zeros(1, dtype=torch.int32, device=d), torch.zeros(1, 64, 128, dtype=torch.bfloat16,
+                                                                               device=d),
+                      torch.zeros(1, 64, dtype=torch.bfloat16, device=d), li,
+                      torch.zeros(1, 4, dtype=torch.int32, device=d), torch.zeros(1, 4, dtype=torch.int32, device=d),
+                      torch.zeros(1, dtype=torch.int32, device=d), torch.zeros(1, dtype=torch.int32, device=d), 8)
+    torch.cuda.synchronize()
+
+
 # ------------------------------------------------------------------- a4 ---
 
 def _decode_case(L, wl, kept, host, s, topk_override=None, table_override=None):
