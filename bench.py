@@ -290,16 +290,19 @@ def append_topk(win, src, s):
 
 
 def time_attention_kernels(win, windows):
-    """Average device time of the attention launch, from external event nodes in a graph.
+    """Average device time of the attention launch and of the append + top-k call, from
+    external event nodes in a graph.
 
     A second graph of the same window carries an event record node before and
-    after every attention launch; replaying it `windows` times gives the mean
-    duration of the attention kernels (split-K pass + LSE merge) inside real steps.
+    after every attention launch and every append + top-k call; replaying it `windows`
+    times gives the mean duration of each inside real steps: (attention ms, append +
+    top-k ms).  The attention launch is the staging copy, the split-K pass and the merge.
     """
     from cuda.bindings import runtime as rt
     from learned_sparse_kv_b200 import lsa
     S = win.s.steps
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(S)]
+    evs_t = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(S)]
 
     def rec(ev):
         st = torch.cuda.current_stream().cuda_stream
@@ -307,7 +310,7 @@ def time_attention_kernels(win, windows):
         if int(err) != 0:
             raise RuntimeError(f"cudaEventRecordWithFlags failed: {err}")
 
-    for a, b in evs:           # create the events before capture
+    for a, b in evs + evs_t:   # create the events before capture
         a.record()
         b.record()
     t, sh = win.t, win.s
@@ -318,19 +321,22 @@ def time_attention_kernels(win, windows):
         if win.cold is None:
             win.select()
         for s in range(S):
+            rec(evs_t[s][0])
             append_topk(win, {k: t[k][s] for k in STEP_KEYS if k in t}, s)
+            rec(evs_t[s][1])
             rec(evs[s][0])
             lsa.sparse_decode(t["q"][s], win.k_pool, win.v_pool, t["chunk_table"], win.topk_idx[s],
                               win.topk_count[s], t["window_start"], win.window_len, win.max_window_len, sh.dv,
                               sh.scale, out=win.out[s], lse=win.lse[s], status=win.status, ws=win.ws_decode)
             rec(evs[s][1])
-    total = 0.0
+    total = total_t = 0.0
     for _ in range(windows):
         g.replay()
         torch.cuda.synchronize()
         total += sum(a.elapsed_time(b) for a, b in evs)
+        total_t += sum(a.elapsed_time(b) for a, b in evs_t)
     del g
-    return total / (windows * S)   # ms per attention launch
+    return total / (windows * S), total_t / (windows * S)   # ms per call
 
 
 # --------------------------------------------------------------- the arms --
@@ -377,7 +383,7 @@ def run_lsa(args, world, rank, local):
     value = tokens / (ms / 1e3)
 
     # dominant kernel: attention, timed by event nodes inside the same window graph
-    att_ms = time_attention_kernels(win, max(1, min(args.steps, 5)))
+    att_ms, at_ms = time_attention_kernels(win, max(1, min(args.steps, 5)))
     att_bytes, att_rows = attention_bytes(win)
     per_launch = att_bytes / wl.steps
     achieved = per_launch / (att_ms / 1e3) / 1e9
@@ -407,6 +413,10 @@ def run_lsa(args, world, rank, local):
                                 "peak": tf_sustained, "unit": "TFLOP/s", "peak_kind": "measured sustained",
                                 "frac_useful": useful / wl.steps / (att_ms / 1e3) / 1e12 / tf_sustained,
                                 "frac_issued": issued / wl.steps / (att_ms / 1e3) / 1e12 / tf_sustained}},
+        "step_breakdown_us": {"append_topk": at_ms * 1e3, "attention": att_ms * 1e3,
+                              "step": ms_local / args.steps / wl.steps * 1e3,
+                              "timing": "event nodes around each call inside the window graph (they add ~1-2 us "
+                                        "per call); step = whole-window graph time / 64"},
         "gpu_launches": args.steps * win.launches_per_window(),
         "clocks": clocks, "device_status": status,
     }

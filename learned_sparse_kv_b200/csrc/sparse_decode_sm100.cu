@@ -103,6 +103,7 @@ struct Params {
     int64_t n_rows_pool;   // n_slots * 64
     int table_stride, k, n_splits;
     int stage_tiles;       // staging slots per sequence
+    uint16_t *stage_mask;  // [B][stage_tiles][4]: valid rows of each staged tile, 16 per piece
     float scale_log2;
     int stall;             // failure-path test: the first wait waits on a barrier nothing arrives on
 };
@@ -213,7 +214,7 @@ __device__ __forceinline__ void drain_stage(uint64_t *full, int u0, int u1, int 
 
 // grid (4 * stage_tiles, B), 128 threads: CTA (4 g + q, b) copies rows 16 q .. 16 q + 15
 // of the gathered tile staged in slot g of sequence b (rows past the row set, or
-// without a slot, as zeros).  Each thread keeps its 9 loads of 16 bytes in flight
+// without a slot, as zeros) and writes which of them are valid into the tile's mask.  Each thread keeps its 9 loads of 16 bytes in flight
 // before storing; a unit over four CTAs keeps four times the copies in flight of
 // one CTA per unit.
 constexpr int STAGE_ROWS = 16, STAGE_THREADS = 128;
@@ -227,6 +228,15 @@ __global__ void __launch_bounds__(STAGE_THREADS) stage_kernel(const Params p, ui
     if (t < 0) return;
     if (threadIdx.x < STAGE_ROWS) rows[threadIdx.x] = st.row(p, b, t, r0 + threadIdx.x);
     __syncthreads();
+    if (threadIdx.x < 32) {
+        // rows 16 q .. 16 q + 15 of the tile's validity mask (the attention's softmax reads it)
+        const int64_t r = threadIdx.x < STAGE_ROWS ? rows[threadIdx.x] : -1;
+        const unsigned valid = __ballot_sync(0xffffffffu, r >= 0), unmapped = __ballot_sync(0xffffffffu, r == -2);
+        if (threadIdx.x == 0) {
+            p.stage_mask[((size_t)b * p.stage_tiles + g) * 4 + (blockIdx.x & 3)] = (uint16_t)valid;
+            if (unmapped) flag(p.status, LSA_DEV_TABLE);
+        }
+    }
     uint4 v[PER_THREAD];
 #pragma unroll
     for (int i = 0; i < PER_THREAD; ++i) {
@@ -248,6 +258,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
     const int split = blockIdx.x >> 1, b = blockIdx.y;
+    // the sequence's row counts are read while the barriers and tensor memory are set up
+    const SeqTiles st(p, b);
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
@@ -273,7 +285,6 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
     cluster_sync();
     const uint32_t tmem = sm.tmem_base;
 
-    const SeqTiles st(p, b);
     // Tiles are dealt round-robin: split s takes tiles s, s + n_splits, ...  The
     // staged top-k tiles (first in the tile list) are thereby spread evenly over
     // the splits.  K (warp 0) and V (warp 3) have a producer each, so K of a later
@@ -289,39 +300,25 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             mbar_arrive_expect_tx_cluster(qf, Q_BYTES);
             tma_load_3d(sm.q[0], &q_map, 0, b * HQ + HPC * (int)rank, 0, qf);
         }
-        // row indices of the next gathered tile are loaded while the current tile is issued
-        int64_t n0 = -1, n1 = -1;
-        if (kprod && st.gathered(tile_of(0))) { n0 = st.row(p, b, tile_of(0), lane); n1 = st.row(p, b, tile_of(0), lane + 32); }
+        auto locate = [&](int u, int64_t &slot_row) -> int {
+            const int t = tile_of(u);
+            if (st.gathered(t)) {
+                slot_row = -2;
+                return (b * p.stage_tiles + st.stage_index(t)) * NTILE;
+            }
+            slot_row = st.window_slot_row(p, b, t);
+            return slot_row >= 0 ? (int)slot_row : (int)p.n_rows_pool;
+        };
+        int64_t sr0 = -2, sr1 = -2;
+        int wy0 = locate(0, sr0), wy1 = n_tiles > 1 ? locate(1, sr1) : 0;
         for (int u = 0; u < n_tiles; ++u) {
             const int t = tile_of(u);
-            const bool gath = st.gathered(t);
-            const int64_t slot_row = gath ? -2 : st.window_slot_row(p, b, t);
-            // an unmapped slot is read out of range: TMA fills zeros; a staged tile is read
-            // from its staging slot
-            const int wy = gath ? (b * p.stage_tiles + st.stage_index(t)) * NTILE
-                                : (slot_row >= 0 ? (int)slot_row : (int)p.n_rows_pool);
             const int s = u & 1;
             const uint32_t par = ((u >> 1) + 1) & 1;
+            const int wy = s ? wy1 : wy0;
+            const int64_t slot_row = s ? sr1 : sr0;
+            const bool gath = st.gathered(t);
             if (kprod) {
-                const int64_t g0 = n0, g1 = n1;
-                if (u + 1 < n_tiles && st.gathered(tile_of(u + 1))) {
-                    n0 = st.row(p, b, tile_of(u + 1), lane);
-                    n1 = st.row(p, b, tile_of(u + 1), lane + 32);
-                }
-                unsigned long long mask;
-                if (!gath) {
-                    if (slot_row == -2) flag(p.status, LSA_DEV_TABLE);
-                    mask = slot_row < 0 ? 0ull : ~0ull;
-                } else {
-                    if ((g0 == -2 || g1 == -2)) flag(p.status, LSA_DEV_TABLE);
-                    const unsigned lo = __ballot_sync(0xffffffffu, g0 >= 0), hi = __ballot_sync(0xffffffffu, g1 >= 0);
-                    mask = (unsigned long long)lo | ((unsigned long long)hi << 32);
-                }
-                if (!warp_wait(sm, &sm.info_empty[u % INFO], ((u / INFO) + 1) & 1, p.status)) break;
-                if (lane == 0) {
-                    sm.info_mask[u % INFO] = mask;
-                    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];\n" ::"r"(smem_addr(&sm.info_full[u % INFO])) : "memory");
-                }
                 if (!warp_wait(sm, &sm.k_empty[s], par, p.status)) break;
                 if (lane == 0) {
                     const uint32_t full = map_to_rank(&sm.k_full[s], 0);
@@ -336,6 +333,26 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
                     mbar_arrive_expect_tx_cluster(full, V_BYTES);
                     tma_load_4d(sm.v[s][0][0], gath ? &vs_map : &v_map, 0, wy, 2 * (int)rank, 0, full);
                     sm.last_v_tma[s] = u;
+                }
+            }
+            if (u + 2 < n_tiles) {
+                if (s) wy1 = locate(u + 2, sr1);
+                else wy0 = locate(u + 2, sr0);
+            }
+            if (kprod) {
+                unsigned long long mask;
+                if (!gath) {
+                    if (slot_row == -2) flag(p.status, LSA_DEV_TABLE);
+                    mask = slot_row < 0 ? 0ull : ~0ull;
+                } else {
+                    // written by the staging copy (which also flagged unmapped rows)
+                    mask = *reinterpret_cast<const unsigned long long *>(
+                        p.stage_mask + ((size_t)b * p.stage_tiles + st.stage_index(t)) * 4);
+                }
+                if (!warp_wait(sm, &sm.info_empty[u % INFO], ((u / INFO) + 1) & 1, p.status)) break;
+                if (lane == 0) {
+                    sm.info_mask[u % INFO] = mask;
+                    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];\n" ::"r"(smem_addr(&sm.info_full[u % INFO])) : "memory");
                 }
             }
             __syncwarp();
@@ -513,7 +530,12 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
             p.m_part[part] = n_tiles > 0 ? m_ref : -INFINITY;
             p.l_part[part] = n_tiles > 0 ? l_tot : 0.f;
         }
-        float *orow = p.o_part + part * DV;
+        // O leaves tensor memory 32 columns at a time (one head row per thread); each warp passes
+        // its 32 x 32 block through shared memory (the P buffers, free once the last P.V is
+        // done; 16-byte pieces XOR-swizzled by row), so that every store instruction writes
+        // four whole 128-byte row pieces instead of 32 scattered 16-byte pieces.
+        float *xbuf = reinterpret_cast<float *>(sm.p[0]) + (warp & 3) * 1024;
+        const size_t prow0 = ((size_t)b * p.n_splits + split) * HQ + HPC * (int)rank + (32 * (warp & 3) & 63);
 #pragma unroll 1
         for (int q = 0; q < 8; ++q) {
             uint32_t o[32];
@@ -524,13 +546,20 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_consta
 #pragma unroll
                 for (int i = 0; i < 32; ++i) o[i] = 0u;
             }
-            // O columns 0..127 hold values 0..255 split by lane half; 128..255 hold 256..511
-            const int j = q >> 2, within = (q & 3) * 32;
-            float4 *dst = reinterpret_cast<float4 *>(orow + 256 * j + 128 * half + within);
 #pragma unroll
             for (int i = 0; i < 8; ++i)
-                dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
-                                     __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+                *reinterpret_cast<uint4 *>(xbuf + lane * 32 + 4 * ((i ^ lane) & 7)) =
+                    make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+            __syncwarp();
+            // O columns 0..127 hold values 0..255 split by lane half; 128..255 hold 256..511
+            const int col = 256 * (q >> 2) + 128 * half + (q & 3) * 32 + 4 * (lane & 7);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int r = 4 * k + (lane >> 3);
+                const float4 v = *reinterpret_cast<const float4 *>(xbuf + r * 32 + 4 * (((lane & 7) ^ r) & 7));
+                *reinterpret_cast<float4 *>(p.o_part + (prow0 + r) * DV + col) = v;
+            }
+            __syncwarp();
         }
         tc_fence_before();
     }
@@ -614,7 +643,8 @@ int max_splits(int B) {
 // window tile (a window that does not start on a chunk boundary is staged whole).
 int stage_tiles(int k, int max_window_len) { return (k + NTILE - 1) / NTILE + (max_window_len + NTILE - 1) / NTILE + 1; }
 size_t stage_bytes(int B, int k, int max_window_len) {
-    return (size_t)B * stage_tiles(k, max_window_len) * NTILE * DQK * 2;
+    // staged rows, then one 64-bit validity mask per staged tile
+    return (size_t)B * stage_tiles(k, max_window_len) * (NTILE * DQK * 2 + 8);
 }
 
 int launch(const uint16_t *q, const uint16_t *kv_pool, int64_t k_stride, int64_t n_slots, const int32_t *table,
@@ -656,6 +686,7 @@ int launch(const uint16_t *q, const uint16_t *kv_pool, int64_t k_stride, int64_t
     prm.o_part = o_part; prm.m_part = m_part; prm.l_part = l_part; prm.status = status;
     prm.n_rows_pool = n_slots * LSA_CHUNK; prm.table_stride = table_stride; prm.k = k; prm.n_splits = n_splits;
     prm.stage_tiles = G;
+    prm.stage_mask = reinterpret_cast<uint16_t *>(stage + (size_t)B * G * NTILE * DQK * 2);
     prm.scale_log2 = scale * 1.4426950408889634f;
     prm.stall = take_test_stall(LSA_TEST_STALL_ATTENTION);
     stage_kernel<<<dim3(4 * G, B), STAGE_THREADS, 0, stream>>>(prm, stage);
