@@ -69,29 +69,28 @@ struct Params {
 };
 
 // The append of the decoded token, folded into the indexer launch: this kernel reads neither
-// the window's rows nor window_len, so CTA b can write sequence b's new rows and advance its
-// window; the attention launches that follow read them.
-__device__ void append_token(const Params &p, int b) {
-    __shared__ int64_t s_row;
-    if (threadIdx.x == 0) {
+// the window's rows nor window_len, so one warp of CTA b writes sequence b's new rows and
+// advances its window while the pipeline fills; the attention launches that follow read them.
+__device__ void append_token(const Params &p, int b, int lane) {
+    int64_t row = -1;
+    if (lane == 0) {
         const int pos = p.window_start[b] + p.window_len[b];
         const int chunk = pos / LSA_CHUNK;
         const int slot = (pos >= 0 && chunk < p.table_stride) ? p.table[(size_t)b * p.table_stride + chunk] : -1;
-        s_row = (slot >= 0 && slot < p.n_slots) ? (int64_t)slot * LSA_CHUNK + pos % LSA_CHUNK : -1;
-        if (s_row < 0) flag(p.status, LSA_DEV_TABLE);
+        row = (slot >= 0 && slot < p.n_slots) ? (int64_t)slot * LSA_CHUNK + pos % LSA_CHUNK : -1;
+        if (row < 0) flag(p.status, LSA_DEV_TABLE);
     }
-    __syncthreads();
-    const int64_t row = s_row;
+    row = __shfl_sync(0xffffffffu, row, 0);
     if (row >= 0) {
         const uint4 *src = reinterpret_cast<const uint4 *>(p.new_kv + (size_t)b * p.kv_width);
         uint4 *dst = reinterpret_cast<uint4 *>(p.kv_pool + row * p.kv_stride);
-        for (int c = threadIdx.x; c < p.kv_width / 8; c += blockDim.x) dst[c] = src[c];
+        for (int c = lane; c < p.kv_width / 8; c += 32) dst[c] = src[c];
         const uint4 *lsrc = reinterpret_cast<const uint4 *>(p.new_li + (size_t)b * p.D);
         uint4 *ldst = reinterpret_cast<uint4 *>(p.li_pool + row * p.D);
-        for (int c = threadIdx.x; c < p.D / 8; c += blockDim.x) ldst[c] = lsrc[c];
+        for (int c = lane; c < p.D / 8; c += 32) ldst[c] = lsrc[c];
     }
-    __syncthreads();
-    if (threadIdx.x == 0 && row >= 0) p.window_len[b] += 1;
+    __syncwarp();
+    if (lane == 0 && row >= 0) p.window_len[b] += 1;
 }
 
 // 1-CTA MMA and commit
@@ -196,7 +195,6 @@ li_score_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_consta
         sm.abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
-    if (p.new_kv && (int)blockIdx.x < p.B) append_token(p, blockIdx.x);
     count_cold(p, wk, warp, lane);
     if (warp == 1) asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
                                     smem_addr(&sm.tmem_base)), "r"(256));
@@ -314,6 +312,7 @@ li_score_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_consta
         __syncwarp();
     } else {
         // ------------------------------------------------ epilogue: one token row per thread
+        if (warp == 2 && p.new_kv && (int)blockIdx.x < p.B) append_token(p, blockIdx.x, lane);
         const int L = threadIdx.x - 64;                       // 0..127
         const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
         const int row = 32 * (warp & 3) + lane;               // TMEM lane = token row of the tile
