@@ -76,7 +76,7 @@ struct TopkShared {
     int cnt[2];                           // this CTA's counts of keys > T and == T
     int base, eq_lower;                   // output offset of this CTA, keys == T in lower CTAs
     uint32_t prefix;
-    int remaining;
+    int remaining, in_bin;
 };
 
 // Top-k of the n scores of one sequence by the NC CTAs of a cluster.
@@ -84,9 +84,11 @@ struct TopkShared {
 // shared memory when they fit (stage_cap keys).  Each 8-bit radix pass counts
 // digits locally; after a cluster barrier every CTA sums the NC
 // histograms through distributed shared memory and picks the same digit, so
-// no result has to be broadcast.  The emission is ordered: a CTA's output
-// offset is the number of selected keys in the lower slices, and ties at the
-// threshold go to the lowest candidate indices.
+// no result has to be broadcast.  The passes stop as soon as the chosen digit's
+// bin holds exactly the keys still to be taken (then every key of the bin is
+// selected and its lower digits do not matter).  The emission is ordered: a
+// CTA's output offset is the number of selected keys in the lower slices, and
+// ties at the threshold go to the lowest candidate indices.
 template <int NC, class PosFn>
 __device__ void topk_cluster(const float *__restrict__ s, int n, int k, PosFn pos, int32_t *__restrict__ out,
                              int32_t *__restrict__ out_count, int stage_cap) {
@@ -137,12 +139,16 @@ __device__ void topk_cluster(const float *__restrict__ s, int n, int k, PosFn po
         if (t < 256 && excl < remaining && excl + v >= remaining) {
             sh.prefix = prefix | (uint32_t(255 - t) << shift);
             sh.remaining = remaining - excl;
+            sh.in_bin = v;
         }
         __syncthreads();
         prefix = sh.prefix;   // rewritten only after the next pass's barriers
         remaining = sh.remaining;
         pmask |= 255u << shift;
+        if (sh.in_bin == remaining) break;   // the same in every CTA: all sum the same histograms
     }
+    // Selected: keys whose digits so far exceed the threshold's, and the first need_eq
+    // (in candidate order) of those equal to it.
     const uint32_t T = prefix;
     const int need_eq = remaining;  // keys equal to T that are taken, >= 1
 
@@ -150,7 +156,7 @@ __device__ void topk_cluster(const float *__restrict__ s, int n, int k, PosFn po
     const int i0 = min(len, t * sub), i1 = min(len, i0 + sub);
     int gt = 0, eq = 0;
     for (int i = i0; i < i1; ++i) {
-        const uint32_t u = key(i);
+        const uint32_t u = key(i) & pmask;
         gt += u > T;
         eq += u == T;
     }
@@ -187,7 +193,7 @@ __device__ void topk_cluster(const float *__restrict__ s, int n, int k, PosFn po
     int dummy;
     int o = sh.base + block_exclusive_scan<kTopkThreads>(gt + take_eq, sh.warp_tot, &dummy);
     for (int i = i0; i < i1; ++i) {
-        const uint32_t u = key(i);
+        const uint32_t u = key(i) & pmask;
         if (u > T || (u == T && take_eq > 0)) {
             if (u == T) --take_eq;
             out[o++] = pos(j0 + i);
