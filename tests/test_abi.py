@@ -112,3 +112,25 @@ def test_topk_kernel_count_follows_the_indexer_shape(lib):
     assert lib.lsa_topk_kernel_count(8, 7, 128) == 0
     assert lib.lsa_topk_kernel_count(8, 64, 96) == 0
     assert lib.lsa_topk_kernel_count(0, 64, 128) == 0
+
+
+def test_append_entry_points_reject_unaligned_rows_before_launch(lib):
+    # Rows move as 16-byte vectors: a base that is not 16-byte aligned is an argument error,
+    # reported before anything is enqueued (the pointers are never dereferenced).
+    P, U = ctypes.c_void_p(4096), ctypes.c_void_p(4096 + 2)
+    f = lib.lsa_append_token
+    f.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                                         ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int,
+                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
+                                         ctypes.c_void_p]
+    rc = f(U, None, P, P, 576, 576, None, 0, 0, P, 128, 16, P, 4, P, P, 1, None, None)
+    assert rc == 1 and "16-byte" in _err(lib)
+    g = lib.lsa_append_topk
+    g.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int64, ctypes.c_int] + [ctypes.c_void_p] * 4 + \
+        [ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+         ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int] + [ctypes.c_void_p] * 5 + \
+        [ctypes.c_size_t, ctypes.c_void_p]
+    rc = g(P, U, P, 576, 576, P, P, P, P, 16, P, 4, P, P, 4, P, 1, 64, 128, 64, P, P, P, None, P, 1 << 20, None)
+    assert rc == 1 and "16-byte" in _err(lib)
+    rc = g(P, P, None, 576, 576, P, P, P, P, 16, P, 4, P, P, 4, P, 1, 64, 128, 64, P, P, P, None, P, 1 << 20, None)
+    assert rc == 1 and "null" in _err(lib)
