@@ -84,7 +84,7 @@ def test_window_128k_b8():
     wl = W.workload("decode_128k_b8_mla")
     host = host_build(wl)
     kept, _, _, _ = H.kept_lists(host)
-    pairs = [(0, 0), (3, 31), (7, 63)]
+    pairs = [(b, 9 * b) for b in range(wl.B)]          # every sequence, steps 0 .. 63
     H.open_topk_gap(host, kept, pairs)
     win = _window(host)
     _check_window(host, win, pairs)
@@ -94,8 +94,9 @@ def test_window_ragged_b32():
     wl = W.workload("decode_ragged_b32_mla")
     host = host_build(wl)
     kept, _, _, _ = H.kept_lists(host)
-    order = np.argsort(wl.ctx)
-    pairs = [(int(order[0]), 0), (int(order[-1]), 63), (int(order[len(order) // 2]), 17)]
+    order = np.argsort(wl.ctx, kind="stable")
+    # eight sequences from the shortest to the longest context, steps spread over the window
+    pairs = [(int(order[i]), s) for i, s in zip((0, 4, 9, 13, 18, 22, 27, 31), (0, 9, 18, 27, 36, 45, 54, 63))]
     H.open_topk_gap(host, kept, pairs)
     win = _window(host)
     _check_window(host, win, pairs)
@@ -105,7 +106,7 @@ def test_window_512k_cold_pool():
     wl = W.workload("decode_512k_b1_mla_cold")
     host = host_build(wl)
     kept, _, _, _ = H.kept_lists(host)
-    pairs = [(0, 0), (0, 63)]
+    pairs = [(0, 0), (0, 21), (0, 42), (0, 63)]
     H.open_topk_gap(host, kept, pairs)
     win = _window(host)
     n_cold = sum(1 for c in kept[0] if c < host["first_window_chunk"])
