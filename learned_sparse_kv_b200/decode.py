@@ -3,9 +3,10 @@
 At the window start the Neural Memory Indexer gate selects chunks once
 (lsa_nmi_select, or lsa_nmi_select_union for several indexers in OR mode, or a
 baseline selector); for each of the next `steps` decode steps the decoded
-token is appended to the recent window (lsa_append_token), the Lightning
-Indexer picks the fine top-k inside the kept chunks (lsa_topk) and attention
-runs over top-k plus window (lsa_sparse_decode).  (arXiv 2606.09079:
+token is appended to the recent window and the Lightning Indexer picks the
+fine top-k inside the kept chunks (one call, lsa_append_topk, with the latent
+layout; lsa_append_token and lsa_topk otherwise), then attention runs over
+top-k plus window (lsa_sparse_decode).  (arXiv 2606.09079:
 gist.science explainer 2.1, cjcn.com.cn article section 2.)
 
 Cold pools (chunks before the window in pinned host memory, one sequence) are
