@@ -59,7 +59,7 @@ struct Params {
     int64_t n_slots;
     int B, H, D, table_stride, kept_cap;
     int stall;                    // failure-path test: the first wait waits on a barrier nothing arrives on
-    // optional append of the decoded token (CTA b, b < B, before anything else): its KV row
+    // optional append of the decoded token (one epilogue warp of CTA b, b < B): its KV row
     // and indexer key go to position window_start[b] + window_len[b], then window_len[b] += 1
     const uint16_t *new_kv, *new_li;
     uint16_t *kv_pool, *li_pool;
