@@ -274,8 +274,8 @@ sparse_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict_
 }
 
 // Combines the split-K partials of each head (the log-sum-exp merge).  DV / 8
-// threads per head, two float4 columns each, 128 threads per CTA: grid
-// (Hq / heads per CTA, B).  A split that saw no rows wrote m = -inf, l = 0 and
+// threads per head, two float4 columns each (NV = 2), or DV / 4 threads with one
+// each (NV = 1), 128 threads per CTA: grid (Hq / heads per CTA, B).  A split that saw no rows wrote m = -inf, l = 0 and
 // O = 0, so every partial row is read without branching.  The loads of up to
 // MERGE_GROUP splits are issued together before any arithmetic; a longer split
 // list is taken group by group, rescaling the running sums to the new maximum.
@@ -283,31 +283,35 @@ sparse_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict_
 // multiprocessor), so the 512 CTAs of an 8-sequence, 128-head merge are one wave.
 constexpr int MERGE_GROUP = 10;
 
-template <int DV>
+template <int DV, int NV>
 __global__ void __launch_bounds__(128, 4) lse_merge_kernel(const float *__restrict__ o_part,
                                                         const float *__restrict__ m_part,
                                                         const float *__restrict__ l_part, int n_splits, int Hq,
                                                         float *__restrict__ out, float *__restrict__ lse) {
-    constexpr int TPH = DV / 8, HPB = 128 / TPH;
+    // NV float4 columns per thread: TPH threads per head, HPB heads per CTA
+    constexpr int TPH = DV / 4 / NV, HPB = 128 / TPH;
     const int t = threadIdx.x % TPH, h = blockIdx.x * HPB + threadIdx.x / TPH, b = blockIdx.y;
     if (h >= Hq) return;
     const size_t row0 = (size_t)b * n_splits * Hq + h;   // partial row of split s: row0 + s * Hq
     float M = -INFINITY, L = 0.f;
-    float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+    float4 a[NV];
+#pragma unroll
+    for (int c = 0; c < NV; ++c) a[c] = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int s0 = 0; s0 < n_splits; s0 += MERGE_GROUP) {
-        float4 v0[MERGE_GROUP], v1[MERGE_GROUP];
+        float4 v[MERGE_GROUP][NV];
         float ms[MERGE_GROUP], ls[MERGE_GROUP];
 #pragma unroll
         for (int j = 0; j < MERGE_GROUP; ++j) {
             if (s0 + j < n_splits) {
                 const size_t idx = row0 + (size_t)(s0 + j) * Hq;
                 const float4 *src = reinterpret_cast<const float4 *>(o_part + idx * DV);
-                v0[j] = __ldcs(src + t);
-                v1[j] = __ldcs(src + TPH + t);
+#pragma unroll
+                for (int c = 0; c < NV; ++c) v[j][c] = __ldcs(src + TPH * c + t);
                 ms[j] = __ldg(m_part + idx);
                 ls[j] = __ldg(l_part + idx);
             } else {
-                v0[j] = v1[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int c = 0; c < NV; ++c) v[j][c] = make_float4(0.f, 0.f, 0.f, 0.f);
                 ms[j] = -INFINITY;
                 ls[j] = 0.f;
             }
@@ -317,31 +321,40 @@ __global__ void __launch_bounds__(128, 4) lse_merge_kernel(const float *__restri
         for (int j = 0; j < MERGE_GROUP; ++j) Mn = fmaxf(Mn, ms[j]);
         const float r = M == -INFINITY ? 0.f : exp2f(M - Mn);   // the sums so far are 0 while M = -inf
         L *= r;
-        a0.x *= r; a0.y *= r; a0.z *= r; a0.w *= r;
-        a1.x *= r; a1.y *= r; a1.z *= r; a1.w *= r;
+#pragma unroll
+        for (int c = 0; c < NV; ++c) { a[c].x *= r; a[c].y *= r; a[c].z *= r; a[c].w *= r; }
 #pragma unroll
         for (int j = 0; j < MERGE_GROUP; ++j) {
             const float w = ms[j] == -INFINITY ? 0.f : exp2f(ms[j] - Mn);
             L += w * ls[j];
-            a0.x += w * v0[j].x; a0.y += w * v0[j].y; a0.z += w * v0[j].z; a0.w += w * v0[j].w;
-            a1.x += w * v1[j].x; a1.y += w * v1[j].y; a1.z += w * v1[j].z; a1.w += w * v1[j].w;
+#pragma unroll
+            for (int c = 0; c < NV; ++c) {
+                a[c].x += w * v[j][c].x; a[c].y += w * v[j][c].y; a[c].z += w * v[j][c].z; a[c].w += w * v[j][c].w;
+            }
         }
         M = Mn;
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
     float4 *dst = reinterpret_cast<float4 *>(out + ((size_t)b * Hq + h) * DV);
-    dst[t] = make_float4(a0.x * inv, a0.y * inv, a0.z * inv, a0.w * inv);
-    dst[TPH + t] = make_float4(a1.x * inv, a1.y * inv, a1.z * inv, a1.w * inv);
+#pragma unroll
+    for (int c = 0; c < NV; ++c) dst[TPH * c + t] = make_float4(a[c].x * inv, a[c].y * inv, a[c].z * inv, a[c].w * inv);
     if (lse && t == 0)
         lse[(size_t)b * Hq + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
 }
 
+// Two float4 columns per thread, or one where the two-column grid would not fill the GPU
+// twice over (few sequences), so that more CTAs share the partials' loads.
 template <int DV>
 static int launch_merge(const float *o_part, const float *m_part, const float *l_part, int n_splits, int Hq, int B,
                         float *out, float *lse, cudaStream_t stream) {
-    constexpr int HPB = 128 / (DV / 8);
-    lse_merge_kernel<DV><<<dim3((Hq + HPB - 1) / HPB, B), 128, 0, stream>>>(o_part, m_part, l_part, n_splits, Hq,
-                                                                           out, lse);
+    constexpr int HPB2 = 128 / (DV / 8), HPB1 = 128 / (DV / 4) > 0 ? 128 / (DV / 4) : 1;
+    const int ctas2 = (Hq + HPB2 - 1) / HPB2 * B;
+    if (DV / 4 <= 128 && ctas2 < 2 * sm_count())
+        lse_merge_kernel<DV, 1><<<dim3((Hq + HPB1 - 1) / HPB1, B), 128, 0, stream>>>(o_part, m_part, l_part,
+                                                                                    n_splits, Hq, out, lse);
+    else
+        lse_merge_kernel<DV, 2><<<dim3((Hq + HPB2 - 1) / HPB2, B), 128, 0, stream>>>(o_part, m_part, l_part,
+                                                                                    n_splits, Hq, out, lse);
     return check_launch("lse_merge_kernel");
 }
 
