@@ -213,6 +213,7 @@ size_t lsa_select_baseline_workspace_size(int B, int max_old_chunks);
  *   li_pool   [n_slots, 64, dl] bf16 (device): indexer key of every resident token
  *   chunk_table [B, table_stride] int32 (device)
  *   kept_idx  [B, kept_cap], kept_count [B] int32 (device): lsa_nmi_select output
+ *             (strictly ascending chunk indices; the first kept_count[b] entries are read)
  *   window_start [B] int32 (device): first position of the recent window, multiple of 64
  *   topk_idx  [B, k] int32 (device, out); topk_count [B] int32 (device, out)
  *   scores    [B, kept_cap * 64] fp32 (device, out, optional): candidate scores

@@ -93,6 +93,12 @@ __device__ void append_token(const Params &p, int b, int lane) {
     if (lane == 0 && row >= 0) p.window_len[b] += 1;
 }
 
+// Starts fetching a tensor map (a __grid_constant__ parameter) so that the first copy through
+// it does not wait for the descriptor.
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(map) : "memory");
+}
+
 // 1-CTA MMA and commit
 __device__ __forceinline__ void umma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, bool acc) {
     asm volatile(
@@ -126,20 +132,41 @@ struct Work {
 };
 
 // Every CTA counts, per sequence, the kept chunks that lie before the recent
-// window (they hold the indexer's candidates): warp w takes sequences w, w + 6, ...
-// CTA 0 also writes the counts out for the top-k pass that follows.
+// window (they hold the indexer's candidates).  The kept list is ascending, so the
+// count is the rank of the window's first chunk in it: each half-warp takes one
+// sequence, samples 16 evenly spaced entries (one round of loads), and counts
+// inside the one block of entries that straddles the window start (a second
+// round).  CTA 0 also writes the counts out for the top-k pass that follows.
 __device__ void count_cold(const Params &p, Work &wk, int warp, int lane) {
-    for (int b = warp; b < p.B; b += THREADS / 32) {
-        const int cnt = min(max(p.kept_count[b], 0), p.kept_cap);
-        const int fw = p.window_start[b] / LSA_CHUNK;
-        const int32_t *kept = p.kept_idx + (size_t)b * p.kept_cap;
+    const int half = lane >> 4, hl = lane & 15;
+    const unsigned hmask = half ? 0xffff0000u : 0x0000ffffu;
+    for (int b0 = 2 * warp; b0 < p.B; b0 += 2 * (THREADS / 32)) {
+        const int b = b0 + half;
+        const bool act = b < p.B;
+        int cnt = 0, fw = 0;
+        const int32_t *kept = p.kept_idx + (size_t)(act ? b : 0) * p.kept_cap;
+        if (act) {
+            cnt = min(max(p.kept_count[b], 0), p.kept_cap);
+            fw = p.window_start[b] / LSA_CHUNK;
+        }
+        // block i = entries [i step, (i + 1) step); lane i samples the block's last entry
+        const int step = (cnt + 15) / 16;
+        bool below = false;
+        if (act && cnt > 0) below = kept[min(cnt - 1, (hl + 1) * step - 1)] < fw;
+        const int full = __popc(__ballot_sync(0xffffffffu, below) & hmask);   // blocks wholly below
+        const int base = full * step;
         int c = 0;
 #pragma unroll 8
-        for (int i = lane; i < cnt; i += 32) c += kept[i] < fw;
-        c = __reduce_add_sync(0xffffffffu, c);
-        if (lane == 0) {
-            wk.cold[b] = c;
-            if (blockIdx.x == 0) p.cold[b] = c;
+        for (int i = hl; i < step; i += 16) {
+            const int q = base + i;
+            if (act && q < cnt) c += kept[q] < fw;
+        }
+#pragma unroll
+        for (int o = 8; o >= 1; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+        if (act && hl == 0) {
+            const int n = min(cnt, base + c);
+            wk.cold[b] = n;
+            if (blockIdx.x == 0) p.cold[b] = n;
         }
     }
 }
@@ -181,6 +208,10 @@ li_score_kernel(const __grid_constant__ CUtensorMap key_map, const __grid_consta
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int atoms = p.D / 64;
 
+    if (threadIdx.x == 32) {
+        prefetch_tensormap(&key_map);
+        prefetch_tensormap(&q_map);
+    }
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) { mbar_init(&sm.k_full[i], 1); mbar_init(&sm.k_empty[i], 1); }
         for (int i = 0; i < 2; ++i) {

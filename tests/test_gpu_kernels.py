@@ -305,6 +305,45 @@ def test_li_topk_exact(L, k):
             np.testing.assert_allclose(scores[b, :pos.size].cpu().numpy(), ref_sc, rtol=1e-4, atol=1e-3)
 
 
+@pytest.mark.parametrize("case", ["empty", "one", "all_cold", "17", "straddle_33", "window_only"])
+def test_li_topk_kept_list_edges(L, case):
+    """The tcgen05 indexer counts a sequence's cold chunks by their rank in the ascending kept
+    list (sampled blocks, then the one block straddling the window start): lists of 0, 1 and
+    17 entries, all before the window, straddling it at a block edge, and only window chunks
+    give the oracle's candidates and top-k."""
+    wl = _small_mla(k=200)
+    host = host_build(wl)
+    fw = [int(host["window_start"][b]) // CH for b in range(wl.B)]
+    lists = {
+        "empty": [np.zeros(0, np.int32)] * wl.B,
+        "one": [np.array([3], np.int32), np.array([fw[1] - 1], np.int32)],
+        "all_cold": [np.arange(fw[0], dtype=np.int32), np.arange(fw[1], dtype=np.int32)],
+        "17": [np.arange(0, 34, 2, dtype=np.int32), np.arange(17, dtype=np.int32)],
+        "straddle_33": [np.arange(fw[0] - 16, fw[0] + 17, dtype=np.int32), np.arange(fw[1] - 20, fw[1] + 13, dtype=np.int32)],
+        "window_only": [np.arange(fw[0], wl.n_ch[0], dtype=np.int32), np.arange(fw[1], wl.n_ch[1], dtype=np.int32)],
+    }[case]
+    H.open_topk_gap(host, lists, [(b, 0) for b in range(wl.B)])
+    d = dev()
+    kept_t = torch.full((wl.B, host["kept_cap"]), -1, dtype=torch.int32)
+    cnt_t = torch.zeros(wl.B, dtype=torch.int32)
+    for b in range(wl.B):
+        kept_t[b, :lists[b].size] = torch.from_numpy(lists[b])
+        cnt_t[b] = lists[b].size
+    st = host["step"]
+    status = torch.zeros(1, dtype=torch.int32, device=d)
+    idx, cnt = L.topk(bf16(st["q_li"][0], d), bf16(st["w_li"][0], d), bf16(host["pools"]["li"], d),
+                      i32(host["chunk_table"], d), kept_t.to(d), cnt_t.to(d), i32(host["window_start"], d), wl.k,
+                      status=status)
+    idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    assert status.item() == 0
+    for b in range(wl.B):
+        pos, ref_sc = H.li_scores(host, lists[b], b, 0)
+        sel = oracle.topk_select(ref_sc, wl.k)
+        assert cnt[b] == sel.size == min(wl.k, pos.size)
+        np.testing.assert_array_equal(idx[b, :cnt[b]], pos[sel])
+        assert np.all(idx[b, cnt[b]:] == -1)
+
+
 def test_li_topk_no_cold_candidates(L):
     wl = _small_mla(k=32)
     host = host_build(wl)
