@@ -540,8 +540,9 @@ def run_e2e(win, wl, args, world):
     """Same metric through the public API with host buffers: per decode step the step's
     inputs go host->device from pinned memory and the attention output comes back.
 
-    The copies run on a side stream and overlap the steps, as a serving loop would run
-    them: step s + 1's inputs land in the second of two input buffers while step s
+    The copies run on two side streams (host to device, device to host: the two
+    directions use separate copy engines) and overlap the steps, as a serving loop would
+    run them: step s + 1's inputs land in the second of two input buffers while step s
     computes, and step s's output is copied back while step s + 1 computes.  A window
     ends when its last output is on the host.  The whole window -- the gate inputs' copy,
     the gate, 64 steps and every per-step copy with its cross-stream dependencies -- is
@@ -550,22 +551,26 @@ def run_e2e(win, wl, args, world):
     t, sh = win.t, win.s
     S = wl.steps
     keys = ["q_li", "w_li", "q", "new_li"] + (["new_kv"] if sh.latent else ["new_k", "new_v"])
-    host_in = {k: t[k].cpu().pin_memory() for k in keys}
+    # a step's inputs (all bf16) packed in one pinned host row, so that each step is one copy;
+    # every input starts on a 16-byte boundary (each size is a multiple of 8 elements)
+    sizes = [t[k][0].numel() for k in keys]
+    assert all(n % 8 == 0 for n in sizes) and all(t[k].dtype == torch.bfloat16 for k in keys)
+    offs = [sum(sizes[:i]) for i in range(len(keys))]
+    host_in = torch.cat([t[k].reshape(S, -1).cpu() for k in keys], dim=1).pin_memory()
     host_sel = {k: t[k].cpu().pin_memory() for k in ("q_nmi", "w_nmi")}
-    dev_in = [{k: torch.empty_like(t[k][0]) for k in keys} for _ in range(2)]
+    dev_rows = [torch.empty(host_in.shape[1], dtype=torch.bfloat16, device=t["q"].device) for _ in range(2)]
+    dev_in = [{k: row[o:o + n].view(t[k].shape[1:]) for k, o, n in zip(keys, offs, sizes)} for row in dev_rows]
     host_out = torch.empty(S, *win.out.shape[1:], dtype=torch.float32).pin_memory()
-    h2d = sum(host_in[k][0].numel() * host_in[k].element_size() for k in keys) * S + \
-        sum(v.numel() * v.element_size() for v in host_sel.values())
+    h2d = host_in.numel() * 2 + sum(v.numel() * v.element_size() for v in host_sel.values())
     d2h = host_out.numel() * 4
 
-    copy = torch.cuda.Stream()
+    copy, copy_out = torch.cuda.Stream(), torch.cuda.Stream()
     inputs_ready = [torch.cuda.Event() for _ in range(S)]
     step_done = [torch.cuda.Event() for _ in range(S)]
 
     def h2d_step(s):
         with torch.cuda.stream(copy):
-            for k in keys:
-                dev_in[s % 2][k].copy_(host_in[k][s], non_blocking=True)
+            dev_rows[s % 2].copy_(host_in[s], non_blocking=True)
             inputs_ready[s].record(copy)
 
     def window_body():
@@ -576,6 +581,7 @@ def run_e2e(win, wl, args, world):
         if win.cold is None:
             win.select()
         copy.wait_stream(compute)
+        copy_out.wait_stream(compute)
         h2d_step(0)
         for s in range(S):
             if s + 1 < S:
@@ -589,10 +595,11 @@ def run_e2e(win, wl, args, world):
                               win.topk_count[s], t["window_start"], win.window_len, win.max_window_len, sh.dv,
                               sh.scale, out=win.out[s], lse=win.lse[s], status=win.status, ws=win.ws_decode)
             step_done[s].record(compute)
-            copy.wait_event(step_done[s])
-            with torch.cuda.stream(copy):
+            copy_out.wait_event(step_done[s])
+            with torch.cuda.stream(copy_out):
                 host_out[s].copy_(win.out[s], non_blocking=True)
-        compute.wait_stream(copy)   # the window ends when its last output is on the host
+        compute.wait_stream(copy)
+        compute.wait_stream(copy_out)   # the window ends when its last output is on the host
 
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
@@ -616,7 +623,7 @@ def run_e2e(win, wl, args, world):
     return {"value": wl.B * S * args.steps * world / (ms / 1e3), "unit": "tokens/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "timing": "one CUDA graph per window: the pinned-host copies of every step's inputs and "
-                      "outputs on a side stream, overlapping the steps"}
+                      "outputs on two side streams (one per direction), overlapping the steps"}
 
 
 def run_cold(args, device, hbm_peak, n_windows=4):
