@@ -134,3 +134,13 @@ def test_append_entry_points_reject_unaligned_rows_before_launch(lib):
     assert rc == 1 and "16-byte" in _err(lib)
     rc = g(P, P, None, 576, 576, P, P, P, P, 16, P, 4, P, P, 4, P, 1, 64, 128, 64, P, P, P, None, P, 1 << 20, None)
     assert rc == 1 and "null" in _err(lib)
+
+
+def test_append_topk_launch_count_follows_the_indexer_shape():
+    # The tcgen05 indexer shapes append inside the indexer launch (2 kernels per call);
+    # other shapes launch the append, the counting kernel, the indexer and the top-k.
+    from learned_sparse_kv_b200 import lsa
+    assert lsa.append_topk_kernel_count(8, 64, 128) == 2
+    assert lsa.append_topk_kernel_count(1, 32, 64) == 2
+    assert lsa.append_topk_kernel_count(65, 64, 128) == 4
+    assert lsa.append_topk_kernel_count(8, 48, 128) == 4
