@@ -27,6 +27,8 @@
  *     is skipped.  No call traps or aborts.
  *   - Scratch memory is passed in as (ws, ws_bytes); lsa_*_workspace_size()
  *     report the size.  Workspace contents need no initialisation.
+ *   - Every entry point that enqueues work opens an NVTX range named after
+ *     itself for the duration of the call (host side; free without a tool).
  *   - Chunk pools: token position p of sequence b lives in row p % 64 of pool
  *     slot chunk_table[b * table_stride + p / 64]; -1 marks a chunk that is not
  *     on the device.  Pools are [n_slots, 64, row_width] row-major.

@@ -27,6 +27,7 @@
 #include <algorithm>
 
 #include "common.cuh"
+#include "nvtx_range.cuh"
 #include "sm100.cuh"
 
 namespace lsa {
@@ -301,6 +302,7 @@ extern "C" int lsa_query_encoder(const lsa_bf16 *h, int B, int d_model, const ls
                                  const lsa_bf16 *w_up, const lsa_bf16 *w_head, int Hn, int dn, lsa_bf16 *q_out,
                                  lsa_bf16 *w_out, float *q_f32, float *w_f32, int32_t *dev_status, void *ws,
                                  size_t ws_bytes, lsa_stream_t stream) {
+    LSA_ABI_RANGE();
     LSA_REQUIRE(h && w_down && w_up && w_head && q_out && w_out, LSA_ERR_INVALID_ARG,
                 "lsa_query_encoder: null pointer");
     LSA_REQUIRE(B >= 1 && B <= enc::MAX_B, LSA_ERR_SHAPE, "lsa_query_encoder: B=%d outside [1, %d]", B, enc::MAX_B);

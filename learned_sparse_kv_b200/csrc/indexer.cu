@@ -10,6 +10,7 @@
 // cjcn.com.cn article section 2.)
 #include "block_scan.cuh"
 #include "common.cuh"
+#include "nvtx_range.cuh"
 
 namespace lsa {
 
@@ -338,6 +339,7 @@ extern "C" int lsa_nmi_select(const lsa_bf16 *q, const lsa_bf16 *w, const lsa_bf
                               const int64_t *seq_chunk_offset, int B, int Hn, int dn, int64_t total_chunks,
                               int max_chunks_per_seq, int32_t *kept_idx, int32_t *kept_count, int kept_cap,
                               float *logits, int32_t *dev_status, void *ws, size_t ws_bytes, lsa_stream_t stream) {
+    LSA_ABI_RANGE();
     NmiSet set = {};
     set.q[0] = q; set.w[0] = w; set.khat[0] = khat; set.logits[0] = logits;
     return nmi_select_impl("lsa_nmi_select", 1, set, seq_chunk_offset, B, Hn, dn, total_chunks, max_chunks_per_seq,
@@ -349,6 +351,7 @@ extern "C" int lsa_nmi_select_union(int n_idx, const lsa_bf16 *const *q, const l
                                     int64_t total_chunks, int max_chunks_per_seq, int32_t *kept_idx,
                                     int32_t *kept_count, int kept_cap, float *logits, int32_t *dev_status, void *ws,
                                     size_t ws_bytes, lsa_stream_t stream) {
+    LSA_ABI_RANGE();
     LSA_REQUIRE(n_idx >= 1 && n_idx <= kMaxIndexers, LSA_ERR_INVALID_ARG,
                 "lsa_nmi_select_union: n_idx must be 1..%d (got %d)", kMaxIndexers, n_idx);
     LSA_REQUIRE(q && w && khat, LSA_ERR_INVALID_ARG, "lsa_nmi_select_union: null pointer array");

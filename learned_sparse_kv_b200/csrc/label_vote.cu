@@ -10,6 +10,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "nvtx_range.cuh"
 
 namespace lsa {
 
@@ -177,6 +178,7 @@ extern "C" size_t lsa_label_vote_workspace_size(int n_layers, int n_steps, int n
 extern "C" int lsa_label_vote(const float *scores, int n_layers, int n_steps, int n_chunks, float top_p,
                               int min_layers, int mode, uint8_t *labels, int32_t *max_votes, void *ws,
                               size_t ws_bytes, lsa_stream_t stream) {
+    LSA_ABI_RANGE();
     LSA_REQUIRE(scores && labels, LSA_ERR_INVALID_ARG, "lsa_label_vote: null pointer");
     LSA_REQUIRE(n_layers >= 1 && n_layers <= 64 && n_steps >= 1 && n_chunks >= 1 && n_chunks <= kMaxVoteChunks,
                 LSA_ERR_SHAPE, "lsa_label_vote: unsupported sizes (layers=%d steps=%d chunks=%d)", n_layers, n_steps,

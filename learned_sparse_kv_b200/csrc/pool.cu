@@ -8,6 +8,7 @@
 
 #include "block_scan.cuh"
 #include "common.cuh"
+#include "nvtx_range.cuh"
 
 namespace lsa {
 
@@ -196,6 +197,7 @@ extern "C" int lsa_append_token(const lsa_bf16 *new_k, const lsa_bf16 *new_v, co
                                 int64_t v_row_stride, int v_width, lsa_bf16 *li_pool, int dl, int64_t n_slots,
                                 const int32_t *chunk_table, int table_stride, const int32_t *window_start,
                                 int32_t *window_len, int B, int32_t *dev_status, lsa_stream_t stream) {
+    LSA_ABI_RANGE();
     LSA_REQUIRE(B > 0 && n_slots > 0 && table_stride > 0, LSA_ERR_INVALID_ARG, "lsa_append_token: bad sizes");
     LSA_REQUIRE(new_k && k_pool && chunk_table && window_start && window_len, LSA_ERR_INVALID_ARG,
                 "lsa_append_token: null pointer");
@@ -219,6 +221,7 @@ extern "C" int lsa_gather_chunks(int n_pools, const void *const *host_pools, con
                                  const int32_t *kept_idx_host, int kept_count_host, int first_window_chunk,
                                  int first_free_slot, int32_t *chunk_table_host, int32_t *chunk_table_dev,
                                  int table_len, lsa_stream_t stream, lsa_event_t done, int *n_fetched) {
+    LSA_ABI_RANGE();
     LSA_REQUIRE(n_pools >= 1 && n_pools <= 4 && host_pools && chunk_bytes && dev_pools, LSA_ERR_INVALID_ARG,
                 "lsa_gather_chunks: need 1..4 pools with host/device bases and chunk sizes");
     for (int i = 0; i < n_pools; ++i)
@@ -281,6 +284,7 @@ extern "C" int lsa_plan_residency(const int32_t *table_cur, int32_t *table_next,
                                   int first_window_chunk, int window_end_chunk, int64_t n_slots, int32_t *copy_chunk,
                                   int32_t *copy_slot, int32_t *copy_count, int copy_cap, int32_t *dev_status, void *ws,
                                   size_t ws_bytes, lsa_stream_t stream) {
+    LSA_ABI_RANGE();
     LSA_REQUIRE(table_cur && table_next && kept_idx && kept_count && copy_chunk && copy_slot && copy_count,
                 LSA_ERR_INVALID_ARG, "lsa_plan_residency: null pointer");
     LSA_REQUIRE(table_cur != table_next, LSA_ERR_INVALID_ARG,
@@ -306,6 +310,7 @@ extern "C" int lsa_fetch_chunks(int n_pools, const void *const *host_pools, cons
                                 void *const *dev_pools, int64_t n_host_chunks, int64_t n_slots,
                                 const int32_t *copy_chunk, const int32_t *copy_slot, const int32_t *copy_count,
                                 int copy_cap, int32_t *dev_status, lsa_stream_t stream) {
+    LSA_ABI_RANGE();
     LSA_REQUIRE(n_pools >= 1 && n_pools <= kMaxPools && host_pools && chunk_bytes && dev_pools, LSA_ERR_INVALID_ARG,
                 "lsa_fetch_chunks: need 1..%d pools with host/device bases and chunk sizes", kMaxPools);
     LSA_REQUIRE(copy_chunk && copy_slot && copy_count && copy_cap > 0 && n_host_chunks > 0 && n_slots > 0,
@@ -335,6 +340,7 @@ extern "C" int lsa_fetch_chunks(int n_pools, const void *const *host_pools, cons
 
 extern "C" int lsa_advance_window(int32_t *window_start, int32_t *window_len, int B, int by, int new_len,
                                   lsa_stream_t stream) {
+    LSA_ABI_RANGE();
     LSA_REQUIRE(window_start && window_len && B > 0 && by >= 0 && by % LSA_CHUNK == 0 && new_len >= 0,
                 LSA_ERR_INVALID_ARG, "lsa_advance_window: bad arguments (B=%d by=%d new_len=%d)", B, by, new_len);
     advance_kernel<<<(B + 255) / 256, 256, 0, stream>>>(window_start, window_len, B, by, new_len);

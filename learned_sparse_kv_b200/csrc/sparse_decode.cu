@@ -11,6 +11,7 @@
 // is online in the log2 domain.  Each CTA writes an unnormalised partial
 // (O, running max, running sum); a merge kernel combines the splits.
 #include "common.cuh"
+#include "nvtx_range.cuh"
 
 namespace lsa {
 
@@ -480,6 +481,7 @@ extern "C" int lsa_sparse_decode(const lsa_bf16 *q, const lsa_bf16 *k_pool, int6
                                  const int32_t *window_len, int max_window_len, int B, int Hq, int dqk, int dv,
                                  float scale, float *out, float *lse, int32_t *dev_status, void *ws, size_t ws_bytes,
                                  lsa_stream_t stream) {
+    LSA_ABI_RANGE();
     LSA_REQUIRE(B > 0 && n_slots > 0 && table_stride > 0 && k >= 0 && max_window_len >= 1, LSA_ERR_INVALID_ARG,
                 "lsa_sparse_decode: bad sizes (B=%d n_slots=%lld table_stride=%d k=%d max_window_len=%d)", B,
                 (long long)n_slots, table_stride, k, max_window_len);
@@ -521,6 +523,7 @@ extern "C" int lsa_sparse_decode(const lsa_bf16 *q, const lsa_bf16 *k_pool, int6
 
 extern "C" int lsa_merge_attention(const float *o_parts, const float *lse_parts, int R, int B, int Hq, int dv,
                                    float *out, float *lse, lsa_stream_t stream) {
+    LSA_ABI_RANGE();
     LSA_REQUIRE(o_parts && lse_parts && out, LSA_ERR_INVALID_ARG, "lsa_merge_attention: null pointer");
     LSA_REQUIRE(R >= 1 && B >= 1 && Hq >= 1 && dv >= 4 && dv % 4 == 0 && (int64_t)B * Hq < (1 << 30),
                 LSA_ERR_INVALID_ARG, "lsa_merge_attention: bad sizes (R=%d B=%d Hq=%d dv=%d)", R, B, Hq, dv);

@@ -10,6 +10,7 @@
 // key == T, in candidate order, which is ascending position.
 #include "block_scan.cuh"
 #include "common.cuh"
+#include "nvtx_range.cuh"
 #include "sm100.cuh"
 
 namespace lsa {
@@ -368,6 +369,7 @@ extern "C" int lsa_topk(const lsa_bf16 *q_li, const lsa_bf16 *w_li, const lsa_bf
                         const int32_t *kept_count, int kept_cap, const int32_t *window_start, int B, int Hl, int dl,
                         int k, int32_t *topk_idx, int32_t *topk_count, float *scores, int32_t *dev_status, void *ws,
                         size_t ws_bytes, lsa_stream_t stream) {
+    LSA_ABI_RANGE();
     return topk_impl(q_li, w_li, li_pool, n_slots, chunk_table, table_stride, kept_idx, kept_count, kept_cap,
                      window_start, B, Hl, dl, k, topk_idx, topk_count, scores, dev_status, ws, ws_bytes, stream,
                      nullptr);
@@ -380,6 +382,7 @@ extern "C" int lsa_append_topk(const lsa_bf16 *new_kv, const lsa_bf16 *new_li, l
                                const int32_t *window_start, int B, int Hl, int dl, int k, int32_t *topk_idx,
                                int32_t *topk_count, float *scores, int32_t *dev_status, void *ws, size_t ws_bytes,
                                lsa_stream_t stream) {
+    LSA_ABI_RANGE();
     LSA_REQUIRE(new_kv && new_li && kv_pool && window_len && li_pool, LSA_ERR_INVALID_ARG,
                 "lsa_append_topk: null append pointer");
     LSA_REQUIRE(kv_width > 0 && kv_width % 8 == 0 && kv_row_stride >= kv_width && kv_row_stride % 8 == 0,
@@ -409,6 +412,7 @@ extern "C" int lsa_topk_kernel_count(int B, int Hl, int dl) {
 extern "C" int lsa_topk_from_scores(const float *scores, const int64_t *cand_offset, int B, int max_cand, int k,
                                     int32_t *topk_idx, int32_t *topk_count, void *ws, size_t ws_bytes,
                                     lsa_stream_t stream) {
+    LSA_ABI_RANGE();
     (void)ws; (void)ws_bytes;
     LSA_REQUIRE(B > 0 && scores && cand_offset && topk_idx && topk_count, LSA_ERR_INVALID_ARG,
                 "lsa_topk_from_scores: null pointer or B <= 0");
@@ -432,6 +436,7 @@ extern "C" size_t lsa_select_baseline_workspace_size(int B, int max_old_chunks) 
 extern "C" int lsa_select_baseline(int mode, const int32_t *window_start, int B, int max_old_chunks, uint64_t seed,
                                    int keep_num, int keep_den, int32_t *kept_idx, int32_t *kept_count, int kept_cap,
                                    int32_t *dev_status, void *ws, size_t ws_bytes, lsa_stream_t stream) {
+    LSA_ABI_RANGE();
     LSA_REQUIRE(mode == LSA_SELECT_RECENT || mode == LSA_SELECT_RANDOM, LSA_ERR_INVALID_ARG,
                 "lsa_select_baseline: mode must be LSA_SELECT_RECENT or LSA_SELECT_RANDOM (got %d)", mode);
     LSA_REQUIRE(B > 0 && kept_cap >= 1 && max_old_chunks >= 0, LSA_ERR_INVALID_ARG,
