@@ -87,6 +87,14 @@ const char *lsa_version(void);
 int lsa_test_stall_next_wait(int which);
 
 /*
+ * Failure-path test switch (no counterpart in the paper): after `after` more
+ * host-issued copies of lsa_gather_chunks succeed, the next one reports failure
+ * without being enqueued, as a failed cudaMemcpyAsync would; the switch then
+ * turns itself off.  after = -1 turns it off.  Only for tests of that path.
+ */
+int lsa_test_fail_copy(int after);
+
+/*
  * a1 -- Neural Memory Indexer chunk gate.
  * Passage: gist.science explainer 2.1 ("Scoring-Mechanismus", "Dynamisches
  * Fetching"); cjcn.com.cn article section 2 (ReLU replaced by Sigmoid, fixed
@@ -349,7 +357,11 @@ int lsa_append_token(const lsa_bf16 *new_k, const lsa_bf16 *new_v, const lsa_bf1
  * are written into chunk_table_host (pinned, table_len entries, caller-owned),
  * which is then copied to chunk_table_dev on the same stream, and `done` (if
  * not NULL) is recorded after the last copy.  The caller orders later work
- * after `done`.
+ * after `done`, and leaves chunk_table_host unchanged until then (the table
+ * copy reads it asynchronously).
+ * A copy that cannot be enqueued returns LSA_ERR_CUDA with chunk_table_host as
+ * it was and chunk_table_dev not rewritten; chunk copies enqueued before it
+ * still run, into slots that neither table references.
  *   host_pools[i]  pinned host base of pool i, [n_host_chunks, chunk_bytes[i]]
  *   dev_pools[i]   device base of pool i, [n_slots, chunk_bytes[i]]
  *   n_fetched      (host, out) number of chunks copied

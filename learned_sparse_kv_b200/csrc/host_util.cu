@@ -47,6 +47,18 @@ static std::atomic<int> g_test_stall{0};
 
 int take_test_stall(int which) { return (g_test_stall.fetch_and(~which) & which) ? 1 : 0; }
 
+// Host copy failure switch: -1 off; otherwise the number of copies that still succeed
+// before one reports failure (the switch then turns itself off).
+static std::atomic<int> g_fail_copy{-1};
+
+bool take_copy_failure() {
+    int n = g_fail_copy.load();
+    while (n >= 0) {
+        if (g_fail_copy.compare_exchange_weak(n, n - 1)) return n == 0;
+    }
+    return false;
+}
+
 }  // namespace lsa
 
 extern "C" const char *lsa_last_error(void) { return lsa::g_last_error; }
@@ -55,6 +67,12 @@ extern "C" int lsa_test_stall_next_wait(int which) {
     if (which != LSA_TEST_STALL_ATTENTION && which != LSA_TEST_STALL_INDEXER)
         return lsa::fail(LSA_ERR_INVALID_ARG, "lsa_test_stall_next_wait: unknown kernel %d", which);
     lsa::g_test_stall.fetch_or(which);
+    return LSA_OK;
+}
+
+extern "C" int lsa_test_fail_copy(int after) {
+    if (after < -1) return lsa::fail(LSA_ERR_INVALID_ARG, "lsa_test_fail_copy: after must be >= -1 (got %d)", after);
+    lsa::g_fail_copy.store(after);
     return LSA_OK;
 }
 

@@ -4,6 +4,7 @@
 //       "Periodische Triggerung", cjcn.com.cn article section 2);
 //   a6  fetch of kept cold chunks from the pinned host pool (cjcn.com.cn
 //       article section 2; gist.science explainer 2.1 "Dynamisches Fetching").
+#include <algorithm>
 #include <vector>
 
 #include "block_scan.cuh"
@@ -190,6 +191,10 @@ __global__ void advance_kernel(int32_t *window_start, int32_t *window_len, int B
 
 }  // namespace lsa
 
+namespace lsa {
+bool take_copy_failure();   // host copy failure switch (lsa_test_fail_copy)
+}
+
 using namespace lsa;
 
 extern "C" int lsa_append_token(const lsa_bf16 *new_k, const lsa_bf16 *new_v, const lsa_bf16 *new_li,
@@ -246,7 +251,10 @@ extern "C" int lsa_gather_chunks(int n_pools, const void *const *host_pools, con
     LSA_REQUIRE((int64_t)first_free_slot + n_cold <= n_slots, LSA_ERR_CAPACITY,
                 "lsa_gather_chunks: %d chunks do not fit in slots %d..%lld", n_cold, first_free_slot,
                 (long long)n_slots - 1);
-    for (int c = 0; c < first_window_chunk; ++c) chunk_table_host[c] = -1;
+    // The new entries of the host table are built aside and written only once every chunk
+    // copy is enqueued: on an error return the caller's table is as it was.
+    std::vector<int32_t> table(chunk_table_host, chunk_table_host + first_window_chunk);
+    for (int c = 0; c < first_window_chunk; ++c) table[c] = -1;
     int slot = first_free_slot;
     int j = 0;
     while (j < kept_count_host && kept_idx_host[j] < first_window_chunk) {
@@ -258,14 +266,23 @@ extern "C" int lsa_gather_chunks(int n_pools, const void *const *host_pools, con
         for (int i = 0; i < n_pools; ++i) {
             const char *src = static_cast<const char *>(host_pools[i]) + (size_t)c0 * chunk_bytes[i];
             char *dst = static_cast<char *>(dev_pools[i]) + (size_t)slot * chunk_bytes[i];
+            if (take_copy_failure()) return fail(LSA_ERR_CUDA, "lsa_gather_chunks: chunk copy failed (injected)");
             LSA_CUDA(cudaMemcpyAsync(dst, src, (size_t)len * chunk_bytes[i], cudaMemcpyHostToDevice, stream));
         }
-        for (int r = 0; r < len; ++r) chunk_table_host[c0 + r] = slot + r;
+        for (int r = 0; r < len; ++r) table[c0 + r] = slot + r;
         slot += len;
         j = e + 1;
     }
-    LSA_CUDA(cudaMemcpyAsync(chunk_table_dev, chunk_table_host, sizeof(int32_t) * (size_t)table_len,
-                             cudaMemcpyHostToDevice, stream));
+    std::vector<int32_t> before(chunk_table_host, chunk_table_host + first_window_chunk);
+    std::copy(table.begin(), table.end(), chunk_table_host);
+    cudaError_t err = take_copy_failure() ? cudaErrorUnknown
+                                          : cudaMemcpyAsync(chunk_table_dev, chunk_table_host,
+                                                            sizeof(int32_t) * (size_t)table_len,
+                                                            cudaMemcpyHostToDevice, stream);
+    if (err != cudaSuccess) {
+        std::copy(before.begin(), before.end(), chunk_table_host);
+        return fail(LSA_ERR_CUDA, "lsa_gather_chunks: chunk table copy failed: %s", cudaGetErrorString(err));
+    }
     if (done) LSA_CUDA(cudaEventRecord(done, stream));
     if (n_fetched) *n_fetched = n_cold;
     return LSA_OK;

@@ -59,6 +59,7 @@ def _load():
         "lsa_last_error": ([], ctypes.c_char_p),
         "lsa_version": ([], ctypes.c_char_p),
         "lsa_test_stall_next_wait": ([I], I),
+        "lsa_test_fail_copy": ([I], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -81,6 +82,12 @@ def test_stall_next_wait(which):
     """Failure-path test switch: the next launch of the named tcgen05 kernel waits on a barrier
     nothing arrives on, for 2 ms, then reports LSA_DEV_TIMEOUT and returns."""
     _check(_lib.lsa_test_stall_next_wait(int(which)))
+
+
+def test_fail_copy(after):
+    """Failure-path test switch: after `after` more host-issued copies of gather_chunks succeed,
+    the next one fails as a failed cudaMemcpyAsync would (-1: off)."""
+    _check(_lib.lsa_test_fail_copy(int(after)))
 
 
 def _check(rc):

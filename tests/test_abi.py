@@ -144,3 +144,39 @@ def test_append_topk_launch_count_follows_the_indexer_shape():
     assert lsa.append_topk_kernel_count(1, 32, 64) == 2
     assert lsa.append_topk_kernel_count(65, 64, 128) == 4
     assert lsa.append_topk_kernel_count(8, 48, 128) == 4
+
+
+def _gather_args(lib, np, kept, first_window_chunk, table):
+    f = lib.lsa_gather_chunks
+    f.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                  ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                  ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    host = np.zeros((16, 64), np.uint8)
+    HP = (ctypes.c_void_p * 1)(host.ctypes.data)
+    DP = (ctypes.c_void_p * 1)(4096)            # never written: the first copy fails before enqueueing
+    CB = (ctypes.c_size_t * 1)(64)
+    return f, (1, HP, CB, DP, 16, 32, kept.ctypes.data, kept.size, first_window_chunk, 8,
+               table.ctypes.data, ctypes.c_void_p(8192), table.size, None, None, None), host
+
+
+@pytest.mark.parametrize("cold", [True, False])
+def test_gather_copy_failure_leaves_the_host_table_unchanged(lib, cold):
+    """Host-side fault injection: the first copy of lsa_gather_chunks (a chunk run, or the table
+    itself when no kept chunk is cold) reports failure; the call returns LSA_ERR_CUDA before
+    enqueueing anything and the caller's host table is as it was."""
+    import numpy as np
+    kept = np.array([1, 2, 5, 12], np.int32) if cold else np.array([12, 13], np.int32)
+    table = np.arange(100, 116, dtype=np.int32)
+    f, args, _ = _gather_args(lib, np, kept, 10, table)
+    assert lib.lsa_test_fail_copy(0) == 0
+    try:
+        rc = f(*args)
+    finally:
+        lib.lsa_test_fail_copy(-1)
+    assert rc == 3 and "failed" in _err(lib)
+    np.testing.assert_array_equal(table, np.arange(100, 116, dtype=np.int32))
+
+
+def test_fail_copy_switch_rejects_bad_counts(lib):
+    assert lib.lsa_test_fail_copy(-2) == 1
+    assert lib.lsa_test_fail_copy(-1) == 0
