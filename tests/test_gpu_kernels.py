@@ -442,10 +442,14 @@ def _decode_case(L, wl, kept, host, s, topk_override=None, table_override=None):
     return out.cpu().numpy(), lse.cpu().numpy(), refs, int(status.item())
 
 
-@pytest.mark.parametrize("shape", ["mla128", "mla128_many_tiles", "mla64", "sep16"])
+@pytest.mark.parametrize("shape", ["mla128", "mla128_many_tiles", "mla64", "sep16", "window_plus_one_chunk"])
 @pytest.mark.parametrize("q_scale", [1.0, 4.0])
 def test_sparse_decode_matches_oracle(L, shape, q_scale):
-    if shape == "sep16":
+    if shape == "window_plus_one_chunk":
+        # contexts of the window plus one and plus two chunks, every chunk kept: the top-k
+        # takes all 64 or 128 cold candidates (fewer than k), most splits get no tile
+        wl = _small_mla(ctx=(17 * CH, 18 * CH), pass_rate=(1.0, 1.0), k=500, q_scale=q_scale)
+    elif shape == "sep16":
         wl = W.workload("decode_16k_b1_h16", B=2, ctx=(80 * CH, 33 * CH), window=20 * CH, steps=2,
                         pass_rate=(0.3, 0.4), q_scale=q_scale, k=300)
     elif shape == "mla128_many_tiles":
