@@ -180,3 +180,15 @@ def test_gather_copy_failure_leaves_the_host_table_unchanged(lib, cold):
 def test_fail_copy_switch_rejects_bad_counts(lib):
     assert lib.lsa_test_fail_copy(-2) == 1
     assert lib.lsa_test_fail_copy(-1) == 0
+
+
+@pytest.mark.parametrize("k, shape, code, words", [(0, (64, 128), 1, "outside"), (65537, (64, 128), 1, "outside"),
+                                                  (64, (64, 96), 2, "unsupported"), (64, (7, 128), 2, "unsupported")])
+def test_topk_rejects_bad_k_and_indexer_shapes_before_launch(lib, k, shape, code, words):
+    P = ctypes.c_void_p(4096)   # never dereferenced: the call fails validation first
+    f = lib.lsa_topk
+    f.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int64, ctypes.c_void_p, ctypes.c_int] + [ctypes.c_void_p] * 2 + \
+        [ctypes.c_int, ctypes.c_void_p] + [ctypes.c_int] * 4 + [ctypes.c_void_p] * 5 + [ctypes.c_size_t, ctypes.c_void_p]
+    Hl, dl = shape
+    rc = f(P, P, P, 16, P, 4, P, P, 4, P, 2, Hl, dl, k, P, P, None, None, P, 1 << 30, None)
+    assert rc == code and words in _err(lib)
